@@ -1,0 +1,363 @@
+"""Pins for the CPU oracle: checks against facts fixed outside the oracle itself.
+
+Each test pins one part of the oracle to a hand-derived value, an exhaustive
+brute force, a closed form or an invariant, chosen so that a plausible slip
+(a swapped nibble, a wrong bit of the six-bit packing, a dropped min term, a
+transposed operand, a wrong tie-break) fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import q4k as O
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "q4k_block_handmade.txt")
+
+
+def _read_golden():
+    header, pairs, ws = None, {}, {}
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            tok = line.split()
+            if tok[0] == "header":
+                header = bytes(int(t, 16) for t in tok[1:])
+            elif tok[0] == "pair":
+                pairs[int(tok[1])] = (int(tok[2]), int(tok[3]))
+            elif tok[0] == "w":
+                ws[int(tok[1])] = float(tok[2])
+    block = np.zeros(144, np.uint8)
+    block[:16] = np.frombuffer(header, np.uint8)
+    block[16:] = np.arange(128, dtype=np.uint8)
+    return block, pairs, ws
+
+
+def _golden_ok(mod):
+    block, pairs, ws = _read_golden()
+    sc, m = mod.scale_min_pairs(block)
+    if any((int(sc[j]), int(m[j])) != pairs[j] for j in range(8)):
+        return False
+    w = mod.dequant_exact(block[None, :])
+    return all(w[i] == v for i, v in ws.items())
+
+
+def test_golden_handmade_block():
+    """Hand-packed block (tests/golden/q4k_block_handmade.txt) decodes to the hand-worked weights."""
+    assert _golden_ok(O)
+
+
+def test_scale_bits_each_owned_once():
+    """Every one of the 96 bits of the scale field moves exactly one six-bit value by 2^b,
+    and every (value, bit) pair is hit exactly once: the packing is a bijection."""
+    base = np.zeros(144, np.uint8)
+    sc0, m0 = O.scale_min_pairs(base)
+    seen = set()
+    for byte in range(12):
+        for bit in range(8):
+            b = base.copy()
+            b[4 + byte] ^= np.uint8(1 << bit)
+            sc, m = O.scale_min_pairs(b)
+            diff = np.concatenate([sc - sc0, m - m0])
+            nz = np.nonzero(diff)[0]
+            assert nz.size == 1
+            v = int(diff[nz[0]])
+            assert v > 0 and (v & (v - 1)) == 0 and v < 64
+            key = (int(nz[0]), v.bit_length() - 1)
+            assert key not in seen
+            seen.add(key)
+    assert len(seen) == 96
+
+
+def test_scale_pack_unpack_exhaustive():
+    """All 8 x 64 x 64 (j, sc, m) values round-trip through the packer/unpacker,
+    with the other seven pairs random."""
+    rng = np.random.default_rng(123)
+    for j in range(8):
+        scv, mv = np.meshgrid(np.arange(64), np.arange(64), indexing="ij")
+        n = scv.size
+        sc = rng.integers(0, 64, (n, 8))
+        m = rng.integers(0, 64, (n, 8))
+        sc[:, j] = scv.ravel()
+        m[:, j] = mv.ravel()
+        blocks = np.zeros((n, 144), np.uint8)
+        blocks[:, 4:16] = O.pack_scale_min(sc, m)
+        sc2, m2 = O.scale_min_pairs(blocks)
+        assert np.array_equal(sc2, sc) and np.array_equal(m2, m)
+
+
+def test_one_hot_nibble_positions():
+    """Setting only nibble h of quant byte 32c+l changes only weight 64c+32h+l, by d*sc_j*v."""
+    sc = np.arange(1, 9)
+    base = O.make_block(1.0, 0.0, sc, np.zeros(8, int), np.zeros(256, int))
+    w0 = O.dequant_exact(base[None])
+    assert np.all(w0 == 0)
+    for c in range(4):
+        for h in range(2):
+            for l in range(32):
+                for v in (1, 9, 15):
+                    b = base.copy()
+                    b[16 + 32 * c + l] = np.uint8(v << (4 * h))
+                    w = O.dequant_exact(b[None])
+                    i = 64 * c + 32 * h + l
+                    expect = np.zeros(256)
+                    expect[i] = 1.0 * sc[i // 32] * v
+                    assert np.array_equal(w, expect), (c, h, l, v)
+
+
+def test_closed_form_constant_block():
+    """Constant q=c, sc=s, m=t in every position: w = d*s*c - dmin*t everywhere,
+    and y = w * sum(x) exactly."""
+    rng = np.random.default_rng(7)
+    for (d, dmin, s, c, t) in [(1e-3, 2e-3, 17, 5, 40), (0.25, 0.125, 63, 15, 63), (3e-4, 0.0, 1, 1, 0)]:
+        blk = O.make_block(d, dmin, [s] * 8, [t] * 8, [c] * 256)
+        dh, dmh = float(np.float16(d)), float(np.float16(dmin))
+        w = O.dequant_exact(np.stack([blk, blk])[None])  # one row, two blocks
+        assert np.all(w == dh * s * c - dmh * t)
+        X = synth.bf16_normal(rng, (3, 512))
+        Y, S = O.matmul_ref(np.stack([blk, blk])[None], X)
+        xs = O.bf16_to_f64(X).sum(axis=1)
+        np.testing.assert_allclose(Y[:, 0], (dh * s * c - dmh * t) * xs, rtol=1e-13, atol=1e-15)
+
+
+def test_quantize_dequantize_round_trip():
+    """Weights built from known (d, dmin, sc, m, q) are found again by a brute-force
+    quantizer, and its packed block dequantises to the same weights bit for bit."""
+    rng = np.random.default_rng(11)
+    for _ in range(3):
+        d = float(np.float16(abs(rng.standard_normal()) * 1e-3))
+        dmin = float(np.float16(abs(rng.standard_normal()) * 1e-3))
+        sc = rng.integers(0, 64, 8)
+        m = rng.integers(0, 64, 8)
+        q = rng.integers(0, 16, 256)
+        j = np.arange(256) // 32
+        w = d * sc[j] * q - dmin * m[j]          # representable by construction
+        sc2, m2, q2 = O.quantize_brute_force(w, d, dmin)
+        blk = O.make_block(d, dmin, sc2, m2, q2)
+        assert np.array_equal(O.dequant_exact(blk[None]), w)
+
+
+def test_dequant_f32_bf16_single_rounding():
+    """fp32 dequant is the exact value rounded once; bf16 is RN of that fp32 value."""
+    W, _ = synth.gemv_small(0, N=8, K=512)
+    ex = O.dequant_exact(W)
+    f = O.dequant_f32(W)
+    assert np.all(np.abs(f.astype(np.float64) - ex) <= np.abs(ex) * 2.0 ** -24)
+    bf = O.bf16_to_f64(O.dequant_bf16_bits(W))
+    assert np.all(np.abs(bf - f.astype(np.float64)) <= np.abs(f.astype(np.float64)) * 2.0 ** -8)
+
+
+def _scalar_weight(block, i):
+    """Scalar restatement used only as brute force for the matmul pins."""
+    d = float(np.frombuffer(bytes(block[0:2]), "<f2")[0])
+    dmin = float(np.frombuffer(bytes(block[2:4]), "<f2")[0])
+    s = [int(v) for v in block[4:16]]
+    j = i // 32
+    if j < 4:
+        sc, m = s[j] & 63, s[j + 4] & 63
+    else:
+        sc = (s[j + 4] & 0xF) | ((s[j - 4] >> 6) << 4)
+        m = (s[j + 4] >> 4) | ((s[j] >> 6) << 4)
+    c, rem = divmod(i, 64)
+    h, l = divmod(rem, 32)
+    q = (int(block[16 + 32 * c + l]) >> (4 * h)) & 0xF
+    return d * sc * q - dmin * m
+
+
+def test_matmul_brute_force_tiny():
+    """Two rows x one block x two tokens, every product enumerated, exact fsum."""
+    W, X = synth.gemv_small(5, N=2, K=256, M=2)
+    Y, S = O.matmul_ref(W, X)
+    xf = O.bf16_to_f64(X)
+    for n in range(2):
+        for mtok in range(2):
+            prods = [_scalar_weight(W[n, 0], i) * xf[mtok, i] for i in range(256)]
+            assert abs(Y[mtok, n] - math.fsum(prods)) <= 1e-12 * math.fsum(abs(p) for p in prods)
+            assert abs(S[mtok, n] - math.fsum(abs(p) for p in prods)) <= 1e-12 * S[mtok, n]
+
+
+def test_matmul_orientation_and_linearity():
+    """Y[m, n] pairs token m with weight row n (not transposed), and Y is linear in X."""
+    W, X = synth.gemv_small(9, N=4, K=512, M=3)
+    Wd = O.dequant_exact(W)
+    xf = O.bf16_to_f64(X)
+    Y, _ = O.matmul_ref(W, X)
+    assert Y.shape == (3, 4)
+    for mtok in range(3):
+        for n in range(4):
+            assert abs(Y[mtok, n] - math.fsum(Wd[n] * xf[mtok])) < 1e-12 * np.abs(Wd[n] * xf[mtok]).sum()
+    # linearity: X = X1 + X2 exactly representable (bf16 * 2 stays bf16)
+    X2 = synth.f32_to_bf16_bits(2.0 * O.bf16_to_f64(X).astype(np.float32))
+    Y2, _ = O.matmul_ref(W, X2)
+    np.testing.assert_allclose(Y2, 2 * Y, rtol=1e-13, atol=1e-14)
+
+
+def test_batch_rows_independent():
+    """Row m of an M-token product equals the one-token product of row m."""
+    W, X = synth.gemv_small(3, N=16, K=512, M=5)
+    Y, _ = O.matmul_ref(W, X)
+    for mtok in range(5):
+        y1, _ = O.matmul_ref(W, X[mtok:mtok + 1])
+        np.testing.assert_allclose(Y[mtok], y1[0], rtol=1e-14, atol=1e-15)
+
+
+def test_routing_brute_force_and_ties():
+    rng = np.random.default_rng(21)
+    L = (rng.standard_normal((40, 128)) * 2).astype(np.float32)
+    L[0, :] = 0.5                      # all equal -> experts 0..7
+    L[1, [3, 70, 90, 100]] = 9.0       # tie among the top
+    L[2, ::2] = L[2, 1::2]             # pairwise duplicates
+    ids, w = O.route_topk(L, 8)
+    for t in range(L.shape[0]):
+        ranked = sorted(range(128), key=lambda e: (-float(L[t, e]), e))[:8]
+        assert list(ids[t]) == ranked
+        full = np.exp(L[t].astype(np.float64) - L[t].max())
+        full /= full.sum()
+        ren = full[ranked] / full[ranked].sum()
+        np.testing.assert_allclose(w[t], ren, rtol=1e-12)
+        assert abs(w[t].sum() - 1.0) < 1e-12
+    assert list(ids[0]) == list(range(8))
+    assert list(ids[1][:4]) == [3, 70, 90, 100]
+
+
+def test_permutation_invariants():
+    rng = np.random.default_rng(5)
+    L = (rng.standard_normal((64, 128)) * 2).astype(np.float32)
+    ids, _ = O.route_topk(L, 8)
+    offs, perm, inv, row_tok = O.permute(ids, 128)
+    flat = ids.reshape(-1)
+    assert sorted(perm.tolist()) == list(range(flat.size))
+    exp_of_row = flat[perm]
+    assert np.all(np.diff(exp_of_row) >= 0)
+    for e in range(128):
+        seg = perm[offs[e]:offs[e + 1]]
+        assert np.all(flat[seg] == e)
+        assert np.all(np.diff(seg) > 0)
+    assert np.array_equal(np.diff(offs), np.bincount(flat, minlength=128))
+    assert np.array_equal(inv[perm], np.arange(flat.size))
+    assert np.array_equal(row_tok, perm // 8)
+
+
+def _small_moe(seed, M=6, E=4, H=256, F=256, topk=2):
+    return synth.moe_layer(seed, M, E=E, H=H, F=F), topk
+
+
+def test_combine_linear_and_gather():
+    rng = np.random.default_rng(2)
+    M, topk, H = 5, 3, 16
+    O1 = rng.standard_normal((M * topk, H))
+    O2 = rng.standard_normal((M * topk, H))
+    inv = rng.permutation(M * topk).astype(np.int32)
+    w = rng.random((M, topk))
+    y1, _ = O.combine_ref(O1, inv, w)
+    y2, _ = O.combine_ref(O2, inv, w)
+    y12, _ = O.combine_ref(2.0 * O1 - O2, inv, w)
+    np.testing.assert_allclose(y12, 2 * y1 - y2, rtol=1e-12, atol=1e-12)
+    onehot = np.zeros((M, topk))
+    onehot[:, 1] = 1.0
+    yg, _ = O.combine_ref(O1, inv, onehot)
+    np.testing.assert_array_equal(yg, O1[inv.reshape(M, topk)[:, 1]])
+
+
+def test_moe_layer_token_permutation_and_expert_relabel():
+    inp, topk = _small_moe(31)
+    y = O.moe_layer_ref(inp["logits"], inp["X"], inp["W_gate_up"], inp["W_down"], topk)
+    p = np.random.default_rng(0).permutation(inp["logits"].shape[0])
+    yp = O.moe_layer_ref(inp["logits"][p], inp["X"][p], inp["W_gate_up"], inp["W_down"], topk)
+    np.testing.assert_allclose(yp, y[p], rtol=1e-12, atol=1e-14)
+    # relabel experts: permute the weight stacks and logit columns together
+    # (ties are impossible with continuous logits, so the chosen set is unchanged)
+    r = np.array([2, 0, 3, 1])
+    yr = O.moe_layer_ref(inp["logits"][:, r], inp["X"], inp["W_gate_up"][r], inp["W_down"][r], topk)
+    np.testing.assert_allclose(yr, y, rtol=1e-12, atol=1e-14)
+
+
+def test_moe_single_expert_is_dense_swiglu_ffn():
+    """E=1, top-1: the layer reduces to down(SiLU(gate x) * up x) with weight 1."""
+    inp = synth.moe_layer(41, 3, E=1, H=256, F=256)
+    y = O.moe_layer_ref(inp["logits"], inp["X"], inp["W_gate_up"], inp["W_down"], 1)
+    G, _ = O.matmul_ref(inp["W_gate_up"][0][:256], inp["X"])
+    U, _ = O.matmul_ref(inp["W_gate_up"][0][256:], inp["X"])
+    h = G / (1 + np.exp(-G)) * U
+    Wd = O.dequant_exact(inp["W_down"][0])
+    np.testing.assert_allclose(y, h @ Wd.T, rtol=1e-12, atol=1e-12)
+
+
+def test_stagewise_pipeline_matches_end_to_end():
+    """Routing -> permutation -> grouped gate_up -> SwiGLU -> grouped down -> combine
+    (all in fp64, no bf16 step) equals the end-to-end layer."""
+    inp, topk = _small_moe(17, M=7, E=5)
+    ids, w = O.route_topk(inp["logits"], topk)
+    offs, perm, inv, row_tok = O.permute(ids, 5)
+    GU, _ = O.grouped_ref(inp["W_gate_up"], inp["X"], offs, row_gather=row_tok)
+    F = inp["F"]
+    h = O.silu_mul(GU[:, :F], GU[:, F:])
+    Od = np.empty((perm.size, inp["H"]))
+    offs64 = offs.astype(np.int64)
+    for e in range(5):
+        a, b = offs64[e], offs64[e + 1]
+        if b > a:
+            Od[a:b] = h[a:b] @ O.dequant_exact(inp["W_down"][e]).T
+    y, _ = O.combine_ref(Od, inv, w)
+    y_ref = O.moe_layer_ref(inp["logits"], inp["X"], inp["W_gate_up"], inp["W_down"], topk)
+    np.testing.assert_allclose(y, y_ref, rtol=1e-11, atol=1e-13)
+
+
+def test_synth_fields_distribution():
+    """The generator's random bytes decode to q in 0..15 and sc, m in 0..63, all values hit."""
+    W, _ = synth.gemv_small(0)
+    sc, m = O.scale_min_pairs(W)
+    q = O.quants(W)
+    assert set(np.unique(q)) == set(range(16))
+    assert set(np.unique(sc)) == set(range(64)) and set(np.unique(m)) == set(range(64))
+
+
+# ---- planted mistakes: each mutant of the oracle must fail a pin -----------------
+
+class _Mutant:
+    def __init__(self, **over):
+        self.__dict__.update({k: getattr(O, k) for k in ("scale_min_pairs", "quants", "block_d_dmin")})
+        self.__dict__.update(over)
+
+    def dequant_exact(self, blocks):
+        d, dmin = self.block_d_dmin(blocks)
+        sc, m = self.scale_min_pairs(blocks)
+        q = self.quants(blocks)
+        j = np.arange(256) // 32
+        w = d[..., None] * sc[..., j] * q - dmin[..., None] * m[..., j]
+        return w.reshape(w.shape[:-2] + (w.shape[-2] * 256,))
+
+
+def _swap_nibbles(blocks):
+    q = O.quants(blocks)
+    out = q.copy()
+    for c in range(4):
+        out[..., 64 * c:64 * c + 32], out[..., 64 * c + 32:64 * c + 64] = q[..., 64 * c + 32:64 * c + 64], q[..., 64 * c:64 * c + 32]
+    return out
+
+
+def _swap_sc_m(blocks):
+    sc, m = O.scale_min_pairs(blocks)
+    return m, sc
+
+
+def _hi_bits_wrong(blocks):
+    sc, m = O.scale_min_pairs(blocks)
+    sc2, m2 = sc.copy(), m.copy()
+    sc2[..., 4:], m2[..., 4:] = (sc[..., 4:] & 15) | (m[..., 4:] & 48), (m[..., 4:] & 15) | (sc[..., 4:] & 48)
+    return sc2, m2
+
+
+def _d_dmin_swapped(blocks):
+    d, dmin = O.block_d_dmin(blocks)
+    return dmin, d
+
+
+@pytest.mark.parametrize("mut", [dict(quants=_swap_nibbles), dict(scale_min_pairs=_swap_sc_m),
+                                 dict(scale_min_pairs=_hi_bits_wrong), dict(block_d_dmin=_d_dmin_swapped)])
+def test_planted_mistakes_are_caught(mut):
+    assert not _golden_ok(_Mutant(**mut))

@@ -1,0 +1,502 @@
+"""Benchmark of the Q4_K hot path on B200.
+
+One step = one pass over every row of the hot path on seeded synthetic inputs
+shaped like the dense and MoE decode/prefill workloads:
+
+  * decode GEMV   gate+up 34816x5120 and down 5120x17408, M = 1, 4, 8, 16, 32
+  * prefill GEMM  17408x5120 at M = 512 and 4096 tokens (tcgen05 tensor cores)
+  * MoE decode    128 experts, top-8, hidden 2048, expert FFN 768, M = 1, 8, 32
+  * MoE prefill   same layer at M = 4096 with 16 hot experts
+
+The headline metric is the decode GEMV's effective HBM bandwidth (weight bytes
+per second over the ten GEMV launches of a step); the prefill GEMM TFLOP/s and
+the MoE layer tokens/s are reported beside it. Every kernel is timed with CUDA
+events on the stream it runs on, with L2 flushed (a 256 MiB write) before each
+timed launch. Weights and activations are resident in HBM before timing
+starts; the `e2e` figure repeats the GEMV measurement through the C ABI with
+host (pinned) activations copied in and results copied out inside the timing.
+
+`--impl reference` times the CPU oracle instead, on a bounded sample.
+Under torchrun each rank runs an independent replica (the path has no
+exchange step) and rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Q4_K GEMV effective HBM GB/s (% of peak); prefill GEMM TFLOPS; MoE layer tokens/s"
+UNIT = "GB/s"
+BLOCK = 144
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ----------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ GPU harness ---
+
+class Timer:
+    """Per-kernel CUDA-event timing on the current stream, L2 flushed before each launch."""
+
+    def __init__(self, torch):
+        self.torch = torch
+        self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        self.pending = []  # (key, start, end)
+        self.times = {}
+
+    def run(self, key, fn):
+        t = self.torch
+        self.flush_buf.fill_(1)
+        s, e = t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True)
+        s.record()
+        out = fn()
+        e.record()
+        self.pending.append((key, s, e))
+        return out
+
+    def collect(self):
+        self.torch.cuda.synchronize()
+        for key, s, e in self.pending:
+            self.times.setdefault(key, []).append(s.elapsed_time(e) * 1e-3)
+        self.pending.clear()
+
+
+def build_workloads(torch, q, synth):
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    W = {}
+    dd = synth.dense_decode(1)
+    W["dec"] = {k: dev(v) for k, v in dd.items()}
+    W["dec_shapes"] = {p: (dd[f"W_{p}"].shape[0], dd[f"W_{p}"].shape[1] * 256) for p in ("gate_up", "down")}
+    W["dec_host_X"] = {p: torch.from_numpy(dd[f"X_{p}"].view(np.int16)).pin_memory() for p in ("gate_up", "down")}
+    Wp, Xp = synth.dense_prefill(2)
+    W["pre"] = (dev(Wp), dev(Xp), Wp.shape[0], Wp.shape[1] * 256)
+    del Wp, Xp
+    md = synth.moe_decode(3, 32)
+    W["moe_dec"] = {k: dev(md[k]) for k in ("logits", "X", "W_gate_up", "W_down")}
+    mp = synth.moe_prefill(4)
+    W["moe_pre"] = {k: dev(mp[k]) for k in ("logits", "X", "W_gate_up", "W_down")}
+    W["moe_dims"] = (md["E"], md["H"], md["F"])
+    W["moe_pre_hot"] = [int(x) for x in mp["hot_ids"]]
+    return W
+
+
+def moe_layer_gpu(q, tm, key, d, M, dims, topk=8):
+    E, H, F = dims
+    rows = M * topk
+    logits, X = d["logits"][:M], d["X"][:M]
+    r = tm.run(key + ":route", lambda: q.moe_route_permute(logits, topk))
+    h = tm.run(key + ":gate_up", lambda: q.moe_q4k_grouped(d["W_gate_up"], E, 2 * F, H, X, r["expert_offsets"],
+                                                            rows, M, q.ACT_SWIGLU, row_gather=r["row_token"]))
+    o = tm.run(key + ":down", lambda: q.moe_q4k_grouped(d["W_down"], E, H, F, h, r["expert_offsets"], rows, M,
+                                                         q.ACT_NONE))
+    return tm.run(key + ":combine", lambda: q.moe_combine(o, r["inv_perm"], r["topk_w"], M, topk, H)), r
+
+
+def run_step(q, tm, W):
+    launches = 0
+    for M in (1, 4, 8, 16, 32):
+        for p in ("gate_up", "down"):
+            N, K = W["dec_shapes"][p]
+            Wt, Xt = W["dec"][f"W_{p}"], W["dec"][f"X_{p}"][:M]
+            tm.run(f"gemv:{p}:M{M}", lambda: q.q4k_gemv(Wt, Xt, N, K))
+            launches += 1
+    Wt, Xt, N, K = W["pre"]
+    for M in (512, 4096):
+        tm.run(f"gemm:M{M}", lambda: q.q4k_gemm(Wt, Xt[:M], N, K))
+        launches += 1
+    for M in (1, 8, 32):
+        moe_layer_gpu(q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"])
+        launches += 5
+    moe_layer_gpu(q, tm, "moe_pre:M4096", W["moe_pre"], 4096, W["moe_dims"])
+    launches += 5
+    return launches
+
+
+def e2e_gemv(torch, q, W, steps, warmup):
+    """GEMV through the C ABI with host activations: H2D copy, kernel, D2H copy, all timed."""
+    total_bytes, h2d, d2h = 0, 0, 0
+    outs = {}
+    for M in (1, 4, 8, 16, 32):
+        for p in ("gate_up", "down"):
+            N, K = W["dec_shapes"][p]
+            outs[(p, M)] = (torch.empty(M, K, dtype=torch.int16, device="cuda"),
+                            torch.empty(M, N, dtype=torch.float32, device="cuda"),
+                            torch.empty(M, N, dtype=torch.float32).pin_memory())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    times = []
+    for it in range(warmup + steps):
+        t_step = 0.0
+        for M in (1, 4, 8, 16, 32):
+            for p in ("gate_up", "down"):
+                N, K = W["dec_shapes"][p]
+                xd, yd, yh = outs[(p, M)]
+                xh = W["dec_host_X"][p][:M]
+                flush.fill_(1)
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record()
+                xd.copy_(xh, non_blocking=True)
+                q.q4k_gemv(W["dec"][f"W_{p}"], xd, N, K, Y=yd)
+                yh.copy_(yd, non_blocking=True)
+                e.record()
+                e.synchronize()
+                t_step += s.elapsed_time(e) * 1e-3
+                if it == 0:
+                    total_bytes += N * (K // 256) * BLOCK
+                    h2d += xh.numel() * 2
+                    d2h += yd.numel() * 4
+        if it >= warmup:
+            times.append(t_step)
+    return total_bytes, h2d, d2h, times
+
+
+def summarize(tm, W, peaks):
+    T = {k: float(np.mean(v)) for k, v in tm.times.items()}
+    comp = {}
+    gemv_bytes, gemv_time = 0, 0.0
+    for M in (1, 4, 8, 16, 32):
+        for p in ("gate_up", "down"):
+            N, K = W["dec_shapes"][p]
+            b = N * (K // 256) * BLOCK
+            t = T[f"gemv:{p}:M{M}"]
+            gemv_bytes += b
+            gemv_time += t
+            comp[f"gemv_{p}_M{M}_GBps"] = round(b / t / 1e9, 1)
+            comp[f"gemv_{p}_M{M}_us"] = round(t * 1e6, 2)
+    Wt, Xt, N, K = W["pre"]
+    for M in (512, 4096):
+        t = T[f"gemm:M{M}"]
+        comp[f"gemm_M{M}_TFLOPS"] = round(2.0 * M * N * K / t / 1e12, 1)
+        comp[f"gemm_M{M}_us"] = round(t * 1e6, 1)
+    for key, M in (("moe_dec", 1), ("moe_dec", 8), ("moe_dec", 32), ("moe_pre", 4096)):
+        parts = [T[f"{key}:M{M}:{s}"] for s in ("route", "gate_up", "down", "combine")]
+        comp[f"{key}_M{M}_tokens_per_s"] = round(M / sum(parts), 1)
+        comp[f"{key}_M{M}_us"] = {s: round(x * 1e6, 2) for s, x in zip(("route", "gate_up", "down", "combine"), parts)}
+    gbps = gemv_bytes / gemv_time / 1e9
+    # dominant kernel by time in a step
+    dom = max(T.items(), key=lambda kv: kv[1])
+    return gbps, comp, T, dom
+
+
+def roofline_for(key, T, W, peaks, traffic=None):
+    t = T[key]
+    if key.startswith("gemm:"):
+        M = int(key.split("M")[-1])
+        _, _, N, K = W["pre"]
+        a = 2.0 * M * N * K / t / 1e12
+        return {"kernel": key, "bound": "tensor", "achieved": round(a, 1), "peak": peaks["bf16"],
+                "unit": "TFLOP/s", "frac": round(a / peaks["bf16"], 4), "traffic": traffic,
+                "peak_source": peaks["src"] + " (burst bf16)"}
+    if key.startswith("gemv:"):
+        _, p, m = key.split(":")
+        N, K = W["dec_shapes"][p]
+        a = N * (K // 256) * BLOCK / t / 1e9
+        return {"kernel": key, "bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(a / peaks["hbm"], 4), "traffic": traffic, "peak_source": peaks["src"] + " (copy)"}
+    if key.startswith("moe_pre") and key.endswith(("gate_up", "down")):
+        E, H, F = W["moe_dims"]
+        rows = 4096 * 8
+        fl = 2.0 * rows * (2 * F) * H if key.endswith("gate_up") else 2.0 * rows * H * F
+        a = fl / t / 1e12
+        return {"kernel": key, "bound": "tensor", "achieved": round(a, 1), "peak": peaks["bf16"],
+                "unit": "TFLOP/s", "frac": round(a / peaks["bf16"], 4), "traffic": traffic,
+                "peak_source": peaks["src"] + " (burst bf16)"}
+    return {"kernel": key, "bound": "hbm", "achieved": None, "peak": peaks["hbm"], "unit": "GB/s", "frac": None,
+            "traffic": traffic}
+
+
+# ------------------------------------------------------------- CPU oracle ---
+
+def cpu_oracle_gemv_sample(seconds_target=10.0):
+    """The oracle (numpy fp64) on a sample of the gate+up GEMV rows: GB/s of Q4_K weights."""
+    import synth
+    from oracle import q4k as O
+
+    rng = np.random.default_rng(1)
+    K = 5120
+    rows = 512
+    W = synth.q4k_random_blocks(rng, rows, K)
+    X = synth.bf16_normal(rng, (1, K))
+    done, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds_target:
+        O.matmul_ref(W, X)
+        done += 1
+    dt = time.perf_counter() - t0
+    gbps = done * rows * (K // 256) * BLOCK / dt / 1e9
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": round(gbps, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} x (512 rows x 5120 Q4_K gate+up GEMV, M=1, dequant+fp64 matmul) in {dt:.1f} s"}
+
+
+# ------------------------------------------------------------ single kernel ---
+
+def only(args):
+    """One kernel family on its workload, `iters` launches, L2 flushed before each."""
+    import torch
+
+    import q4_weight_only_super_b200 as q
+    import synth
+
+    torch.cuda.set_device(0)
+    q.lib()
+
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    tm = Timer(torch)
+    if args.only == "gemv":
+        M = args.m or 1
+        dd = synth.dense_decode(1)
+        Wt, Xt = dev(dd[f"W_{args.proj}"]), dev(dd[f"X_{args.proj}"][:M])
+        N, K = dd[f"W_{args.proj}"].shape[0], dd[f"W_{args.proj}"].shape[1] * 256
+        fn = lambda: q.q4k_gemv(Wt, Xt, N, K)
+        units = N * (K // 256) * BLOCK / 1e9
+        unit = "GB/s"
+    elif args.only == "gemm":
+        M = args.m or 4096
+        Wp, Xp = synth.dense_prefill(2, M=M)
+        Wt, Xt = dev(Wp), dev(Xp)
+        N, K = Wp.shape[0], Wp.shape[1] * 256
+        fn = lambda: q.q4k_gemm(Wt, Xt, N, K)
+        units = 2.0 * M * N * K / 1e12
+        unit = "TFLOP/s"
+    else:
+        M = args.m or (4096 if args.only == "moe_pre" else 32)
+        inp = synth.moe_prefill(4, M) if args.only == "moe_pre" else synth.moe_decode(3, M)
+        d = {k: dev(inp[k]) for k in ("logits", "X", "W_gate_up", "W_down")}
+        dims = (inp["E"], inp["H"], inp["F"])
+        fn = lambda: moe_layer_gpu(q, tm, "moe", d, M, dims)
+        units = M
+        unit = "tokens/s"
+    for _ in range(args.iters):
+        if args.only.startswith("moe"):
+            fn()
+        else:
+            tm.run("k", fn)
+    tm.collect()
+    st = q.q4k_last_device_status()
+    if args.only.startswith("moe"):
+        t = sum(float(np.mean(v)) for v in tm.times.values())
+    else:
+        t = float(np.mean(tm.times["k"]))
+    print(json.dumps({"only": args.only, "M": M, "proj": args.proj, "iters": args.iters, "us": round(t * 1e6, 2),
+                      "rate": round(units / t, 2), "unit": unit, "status": st}))
+    return 0 if st == 0 else 1
+
+
+# ------------------------------------------------------------------ main ---
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None, choices=["gemv", "gemm", "moe_dec", "moe_pre"],
+                    help="run one kernel family a few times (for profiler captures), print times")
+    ap.add_argument("--m", type=int, default=None, help="tokens for --only")
+    ap.add_argument("--proj", default="gate_up", choices=["gate_up", "down"], help="GEMV matrix for --only")
+    ap.add_argument("--iters", type=int, default=3, help="launches for --only")
+    args = ap.parse_args()
+    if args.only:
+        return only(args)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks = _peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        for _ in range(args.warmup):
+            cpu_oracle_gemv_sample(2.0)
+        for _ in range(args.steps):
+            vals.append(cpu_oracle_gemv_sample(5.0))
+        v = float(np.mean([x["value"] for x in vals]))
+        cb = dict(vals[-1])
+        cb["value"] = round(v, 4)
+        cb["sample"] = f"{args.steps} steps, each " + cb["sample"]
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Q4_K GEMV gate+up 34816x5120 at M=1 (oracle on a 512-row sample)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    import torch
+
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+
+    import q4_weight_only_super_b200 as q
+    import synth
+
+    q.lib()
+    W = build_workloads(torch, q, synth)
+    tm = Timer(torch)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        run_step(q, tm, W)
+    tm.collect()
+    tm.times.clear()
+    st = q.q4k_last_device_status()
+    assert st == 0, f"device status {st} after warm-up"
+
+    clk = ClockSampler(local)
+    barrier()
+    clk.start()
+    t0 = time.perf_counter()
+    s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_ev.record()
+    launches = 0
+    for _ in range(args.steps):
+        launches += run_step(q, tm, W)
+    e_ev.record()
+    barrier()
+    wall = time.perf_counter() - t0
+    clocks = clk.stop()
+    tm.collect()
+    step_s = s_ev.elapsed_time(e_ev) * 1e-3 / args.steps
+    assert q.q4k_last_device_status() == 0
+
+    gbps, comp, T, dom = summarize(tm, W, peaks)
+    total_bytes, h2d, d2h, e2e_times = e2e_gemv(torch, q, W, max(3, args.steps // 2), 2)
+    e2e_gbps = total_bytes / float(np.mean(e2e_times)) / 1e9
+
+    if world > 1:
+        t = torch.tensor([1.0 / gbps, step_s, 1.0 / e2e_gbps], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        gbps_all = world / t[0].item()
+        step_s = t[1].item()
+        e2e_all = world / t[2].item()
+    else:
+        gbps_all, e2e_all = gbps, e2e_gbps
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(gbps_all, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "Q4_K dense decode GEMV gate+up 34816x5120 and down 5120x17408 at "
+                                   "M=1,4,8,16,32 (seed 1); step also runs prefill GEMM 17408x5120 at "
+                                   "M=512,4096 and MoE layers (128 experts, top-8) at M=1,8,32,4096",
+                       "l2": "256 MiB flush write before every timed kernel",
+                       "parallelism": "replicas" if world > 1 else "single GPU",
+                       "moe_prefill_hot_experts": W["moe_pre_hot"]},
+            "frac_of_hbm_peak": round(gbps_all / world / peaks["hbm"], 4),
+            "components": comp,
+            "roofline": roofline_for(dom[0], T, W, peaks),
+            "rooflines": [roofline_for(k, T, W, peaks) for k in ("gemv:gate_up:M1", "gemv:down:M1",
+                                                                  "gemv:gate_up:M32", "gemm:M4096",
+                                                                  "moe_pre:M4096:gate_up", "moe_pre:M4096:down")],
+            "e2e": {"value": round(e2e_all, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "wall_s": round(wall, 3),
+            "peaks": peaks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_gemv_sample(10.0)
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main() or 0)

@@ -1,0 +1,162 @@
+/*
+ * q4k.h -- C ABI of the Q4_K weight-only matrix-product library for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operations are the hot path of GGUF Q4_K inference as the hipEngine
+ * 0.3.0 README describes it ("GGUF Support": Q4_K quant readers, the
+ * bulk-prefill path; "Quickstart": the WMMA-prefill / GEMV-decode session
+ * profile; "Architecture at a glance": the moe kernel family) and as the
+ * hipster README's claims table measures it (GEMV GB/s, "MoE grouped GEMM").
+ *
+ * Q4_K super-block (llama.cpp-style K-quant; 256 weights in 144 bytes):
+ *   bytes 0-1   d     IEEE binary16, little-endian
+ *   bytes 2-3   dmin  IEEE binary16
+ *   bytes 4-15  eight six-bit (sc_j, m_j) pairs:
+ *                 j<4 : sc_j = s[j] & 63, m_j = s[j+4] & 63
+ *                 j>=4: sc_j = (s[j+4] & 15) | (s[j-4] >> 6) << 4
+ *                       m_j  = (s[j+4] >> 4) | (s[j]   >> 6) << 4
+ *   bytes 16-143 quants: weight i = 64c + 32h + l is nibble h (0 = low) of
+ *                 quant byte 32c + l; it uses pair j = i / 32
+ *   w_i = d * sc_j * q_i - dmin * m_j
+ * A Q4_K matrix with N rows and K inputs is stored row-major as
+ * [N][K/256] blocks, so one row is K/256*144 contiguous bytes.
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers (cudaMalloc'd or equivalent),
+ *    owned by the caller. The library allocates no device memory, keeps no
+ *    per-call state except a device status word, and never synchronises
+ *    the stream (except q4k_last_device_status).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Every call is asynchronous on that stream.
+ *  - Activations are bf16 bit patterns (uint16_t), row-major [M][K].
+ *    Matmul outputs are fp32 row-major [M][N].
+ *  - Base pointers must be 16-byte aligned. K must be a multiple of 256.
+ *  - A host-detectable error returns a nonzero q4k_status before anything
+ *    is launched and writes nothing. Unsupported shapes fail with
+ *    Q4K_ERR_UNSUPPORTED; there is no fallback path.
+ *  - Device-side errors (a bounded wait that gave up, an index out of
+ *    range) are latched in a device status word that
+ *    q4k_last_device_status() reads and clears.
+ *  - Results are deterministic: the same inputs give bit-identical outputs
+ *    (no floating-point atomics on any result path).
+ */
+#ifndef Q4K_H
+#define Q4K_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  Q4K_OK = 0,
+  Q4K_ERR_NULL = 1,           /* a required pointer is NULL                        */
+  Q4K_ERR_ALIGN = 2,          /* a pointer is not 16-byte aligned                 */
+  Q4K_ERR_SHAPE = 3,          /* a size is negative/zero where not allowed, or
+                                 K % 256 != 0                                      */
+  Q4K_ERR_UNSUPPORTED = 4,    /* a valid shape outside the supported set           */
+  Q4K_ERR_WORKSPACE = 5,      /* workspace missing or smaller than required        */
+  Q4K_ERR_LAUNCH = 6,         /* the CUDA launch itself failed                     */
+  Q4K_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up                */
+  Q4K_ERR_DEVICE_BOUNDS = 8,  /* a device-side index check failed                  */
+  Q4K_ERR_CUDA = 9            /* a CUDA runtime call returned an error             */
+} q4k_status;
+
+enum { Q4K_ACT_NONE = 0, Q4K_ACT_SWIGLU = 1 };
+enum { Q4K_OP_GEMM = 1, Q4K_OP_ROUTE = 2, Q4K_OP_GROUPED = 3 };
+
+/* Dequantise `nblocks` consecutive Q4_K blocks (hipEngine 0.3.0 README,
+ * "GGUF Support": the Q4_K quant reader).
+ *   W    [nblocks][144] bytes.
+ *   out  out_bf16 == 0: fp32 [nblocks*256], each value RN_fp32 of the exact
+ *        d*sc*q - dmin*m (bit-exact);
+ *        out_bf16 != 0: bf16 bits [nblocks*256] = RN_bf16 of that fp32 value.
+ * nblocks == 0 is a no-op. */
+q4k_status q4k_dequant(const void* W, int64_t nblocks, int out_bf16, void* out, void* stream);
+
+/* Decode GEMV, 1 <= M <= 32 tokens (hipEngine 0.3.0 README, "Quickstart":
+ * the GEMV-decode half of the WMMA-prefill/GEMV-decode session profile).
+ *   Y[m][n] = sum_k w[n][k] * X[m][k],  W [N][K/256] blocks, X bf16 [M][K],
+ *   Y fp32 [M][N].  N % 16 == 0.  M == 0 or N == 0 is a no-op.
+ * Row m of the result does not depend on the other rows of X (bit-identical
+ * to the M == 1 call on that row). */
+q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
+                    void* stream);
+
+/* Prefill GEMM on tcgen05 tensor cores with the Q4_K weights dequantised
+ * tile by tile into shared memory (hipEngine 0.3.0 README, "GGUF Support":
+ * the bulk-prefill path).
+ *   Y[m][n] = sum_k w[n][k] * X[m][k] with w rounded to bf16 (RN of the fp32
+ *   dequant), bf16 x bf16 products, fp32 accumulation.
+ *   N % 256 == 0, K % 256 == 0, M >= 1 (ragged M handled).
+ *   ws/ws_bytes: unused (pass NULL, 0); reserved for split variants. */
+q4k_status q4k_gemm(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Top-k routing and token permutation for a mixture-of-experts layer
+ * (hipEngine 0.3.0 README, "Architecture at a glance": moe kernels).
+ *   logits     fp32 [M][E] router logits.
+ *   topk_ids   int32 [M][topk]: experts ranked by logit, descending, equal
+ *              logits to the lower id.
+ *   topk_w     fp32 [M][topk]: softmax over the selected logits.
+ *   expert_offsets int32 [E+1]: exclusive prefix sum of per-expert counts.
+ *   perm       int32 [M*topk]: sorted row -> flat index t*topk + j, sorted
+ *              by (expert, flat index).
+ *   inv_perm   int32 [M*topk]: flat index -> sorted row.
+ *   row_token  int32 [M*topk]: sorted row -> token.
+ *   ws         device scratch of q4k_workspace_bytes(Q4K_OP_ROUTE, M, 0, 0,
+ *              E, topk) bytes (per-tile expert histograms).
+ * 1 <= E <= 1024, 1 <= topk <= min(E, 16). M == 0 writes expert_offsets
+ * as zeros only. */
+q4k_status moe_route_permute(const float* logits, int M, int E, int topk,
+                             int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                             int32_t* perm, int32_t* inv_perm, int32_t* row_token,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped expert matmul over rows sorted by expert (hipster README, claims
+ * table: "MoE grouped GEMM"; hipEngine 0.3.0 README, moe kernels).
+ *   W_experts  [E][N][K/256] Q4_K blocks.
+ *   A          bf16 activations; row r of the sorted order reads
+ *              A[row_gather[r]] (row_gather may be NULL: A[r]).
+ *   expert_offsets int32 [E+1] (device): rows [off[e], off[e+1]) use expert e.
+ *   rows       total rows = off[E] (host value; must match the device array).
+ *   max_rows_hint  upper bound on any single expert's row count (for a
+ *              top-k layer over M tokens: M). <= 32 selects the GEMV-style
+ *              decode kernel; larger selects the tcgen05 grouped GEMM.
+ *   act == Q4K_ACT_NONE:   out fp32 [rows][N].
+ *   act == Q4K_ACT_SWIGLU: out bf16 [rows][N/2], h = SiLU(g) * u with
+ *              g = columns 0..N/2-1 (gate rows of W) and u = N/2..N-1 (up rows).
+ *   ws: unused by the current kernels (pass NULL, 0).
+ * N % 32 == 0 (SWIGLU: N/2 % 16 == 0), rows == 0 is a no-op. */
+q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uint16_t* A,
+                           const int32_t* row_gather, const int32_t* expert_offsets,
+                           int rows, int max_rows_hint, int act, void* out,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Weighted combine of the expert outputs back into token order
+ * (hipEngine 0.3.0 README, "Core principles": the gate_combine part of the
+ * fused gate_combine_residual composite).
+ *   y[t][h] = sum_{j=0..topk-1} topk_w[t][j] * O[inv_perm[t*topk + j]][h],
+ *   summed in increasing j.  O fp32 [M*topk][H], Y fp32 [M][H].
+ * H % 4 == 0.  M == 0 is a no-op. */
+q4k_status moe_combine(const float* O, const int32_t* inv_perm, const float* topk_w,
+                       int M, int topk, int H, float* Y, void* stream);
+
+/* Bytes of device workspace an entry point needs for these sizes
+ * (Q4K_OP_ROUTE: moe_route_permute; others return 0). */
+size_t q4k_workspace_bytes(int op, int M, int N, int K, int E, int topk);
+
+/* Synchronises `stream`, returns the device status word (Q4K_OK if no
+ * device-side error was latched since the last call) and clears it. */
+q4k_status q4k_last_device_status(void* stream);
+
+/* Static description of a status code. */
+const char* q4k_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4K_H */

@@ -1,0 +1,176 @@
+"""Q4_K weight-only matrix products for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over ``libq4k.so`` (C ABI in ``include/q4k.h``). Every
+function here only marshals arguments: tensors are passed as raw device
+pointers, the current torch CUDA stream is passed as the stream, and any
+non-zero status raises :class:`Q4KError`. All computation happens in the
+library's CUDA kernels; there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemm", "moe_route_permute",
+    "moe_q4k_grouped", "moe_combine", "q4k_workspace_bytes", "q4k_last_device_status",
+    "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "EXPORTS",
+]
+
+ACT_NONE, ACT_SWIGLU = 0, 1
+OP_GEMM, OP_ROUTE, OP_GROUPED = 1, 2, 3
+BLOCK_BYTES = 144
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libq4k.so")
+
+_p, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+# name -> (restype, argtypes); mirrors include/q4k.h
+EXPORTS = {
+    "q4k_dequant": (_i, [_p, _i64, _i, _p, _p]),
+    "q4k_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p]),
+    "q4k_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
+    "moe_route_permute": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "moe_q4k_grouped": (_i, [_p, _i, _i, _i, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
+    "moe_combine": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
+    "q4k_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "q4k_last_device_status": (_i, [_p]),
+    "q4k_status_string": (ctypes.c_char_p, [_i]),
+}
+
+_LIB = None
+
+
+class Q4KError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: status {status} ({lib().q4k_status_string(status).decode()})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libq4k.so (fails loudly if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing; build it with `python -m q4_weight_only_super_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in EXPORTS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, st):
+    if st != 0:
+        raise Q4KError(fn, st)
+
+
+def _bits16(x):
+    """bf16 activations may be given as bfloat16 or as their int16 bit patterns."""
+    assert x.dtype in (torch.bfloat16, torch.int16, torch.uint16), x.dtype
+    return x
+
+
+def q4k_dequant(W, out_bf16: bool = False, out=None, stream=None):
+    """W: uint8 [..., 144] Q4_K blocks on the GPU -> fp32 (or bf16) weights [nblocks*256]."""
+    nb = W.numel() // BLOCK_BYTES
+    if out is None:
+        out = torch.empty(nb * 256, dtype=torch.bfloat16 if out_bf16 else torch.float32, device=W.device)
+    _check("q4k_dequant", lib().q4k_dequant(_ptr(W), nb, int(out_bf16), _ptr(out), _stream(stream)))
+    return out
+
+
+def q4k_gemv(W, X, N: int, K: int, Y=None, stream=None):
+    """Y[M][N] = X[M][K] @ W^T for 1 <= M <= 32 (W: Q4_K [N][K/256][144])."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
+    _check("q4k_gemv", lib().q4k_gemv(_ptr(W), _ptr(_bits16(X)), _ptr(Y), M, N, K, _stream(stream)))
+    return Y
+
+
+def q4k_gemm(W, X, N: int, K: int, Y=None, stream=None):
+    """Prefill GEMM Y[M][N] = X[M][K] @ W^T on tcgen05 tensor cores."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
+    _check("q4k_gemm", lib().q4k_gemm(_ptr(W), _ptr(_bits16(X)), _ptr(Y), M, N, K, None, 0,
+                                      _stream(stream)))
+    return Y
+
+
+def q4k_workspace_bytes(op: int, M: int, N: int = 0, K: int = 0, E: int = 0, topk: int = 0) -> int:
+    return lib().q4k_workspace_bytes(op, M, N, K, E, topk)
+
+
+def moe_route_permute(logits, topk: int, out=None, ws=None, stream=None):
+    """Top-k routing + stable permutation by expert. Returns a dict of device tensors:
+    topk_ids, topk_w, expert_offsets, perm, inv_perm, row_token."""
+    M, E = logits.shape
+    dev = logits.device
+    if out is None:
+        out = dict(
+            topk_ids=torch.empty(M, topk, dtype=torch.int32, device=dev),
+            topk_w=torch.empty(M, topk, dtype=torch.float32, device=dev),
+            expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            perm=torch.empty(M * topk, dtype=torch.int32, device=dev),
+            inv_perm=torch.empty(M * topk, dtype=torch.int32, device=dev),
+            row_token=torch.empty(M * topk, dtype=torch.int32, device=dev),
+        )
+    need = q4k_workspace_bytes(OP_ROUTE, M, E=E, topk=topk)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = lib().moe_route_permute(
+        _ptr(logits), M, E, topk, _ptr(out["topk_ids"]), _ptr(out["topk_w"]),
+        _ptr(out["expert_offsets"]), _ptr(out["perm"]), _ptr(out["inv_perm"]),
+        _ptr(out["row_token"]), _ptr(ws), ws.numel(), _stream(stream))
+    _check("moe_route_permute", st)
+    return out
+
+
+def moe_q4k_grouped(W_experts, E: int, N: int, K: int, A, expert_offsets, rows: int,
+                    max_rows_hint: int, act: int = ACT_NONE, row_gather=None, out=None, stream=None):
+    """Grouped expert matmul over rows sorted by expert (see include/q4k.h)."""
+    if out is None:
+        if act == ACT_SWIGLU:
+            out = torch.empty(rows, N // 2, dtype=torch.bfloat16, device=A.device)
+        else:
+            out = torch.empty(rows, N, dtype=torch.float32, device=A.device)
+    st = lib().moe_q4k_grouped(_ptr(W_experts), E, N, K, _ptr(_bits16(A)), _ptr(row_gather),
+                               _ptr(expert_offsets), rows, max_rows_hint, act, _ptr(out), None, 0,
+                               _stream(stream))
+    _check("moe_q4k_grouped", st)
+    return out
+
+
+def moe_combine(O, inv_perm, topk_w, M: int, topk: int, H: int, Y=None, stream=None):
+    """y[t] = sum_j topk_w[t,j] * O[inv_perm[t*topk+j]]."""
+    if Y is None:
+        Y = torch.empty(M, H, dtype=torch.float32, device=O.device)
+    _check("moe_combine", lib().moe_combine(_ptr(O), _ptr(inv_perm), _ptr(topk_w), M, topk, H,
+                                            _ptr(Y), _stream(stream)))
+    return Y
+
+
+def q4k_last_device_status(stream=None) -> int:
+    """Synchronise the stream, return and clear the device status word (0 = ok)."""
+    return lib().q4k_last_device_status(_stream(stream))

@@ -1,0 +1,643 @@
+// Q4_K prefill GEMM and grouped expert GEMM on 5th-generation tensor cores
+// (tcgen05 + TMEM), with the weights dequantised tile by tile into shared
+// memory (hipEngine 0.3.0 README, "GGUF Support": the bulk-prefill path;
+// hipster README claims table: "MoE grouped GEMM").
+//
+//   D[m][n] = sum_k X[m][k] * w[n][k],  w = RN_bf16(RN_fp32(d*sc*q - dmin*m))
+//
+// CTA tile 256 (tokens) x 256 (weight rows), K step 64, one tile per CTA:
+//   warp 0      TMA producer: activation tile (bf16, 128-byte swizzle) and the
+//               raw Q4_K bytes of the weight tile (block headers + 32 quant
+//               bytes per row per K step), into a 3-deep ring.
+//   warp 1      allocates 512 TMEM columns; lane 0 issues tcgen05.mma
+//               (M=128, N=256, K=16, bf16 x bf16 -> fp32) for both 128-row
+//               halves of the token tile; frees TMEM at the end.
+//   warps 2-9   dequantise one weight row each per K step into the canonical
+//               K-major 128-byte-swizzled bf16 layout the MMA reads (2-deep
+//               ring); afterwards they drain TMEM (tcgen05.ld) to global.
+//   warps 10-13 (gathered-row variant only) load activation rows by index
+//               with cp.async into the same swizzled layout.
+// Every wait is bounded; on expiry the kernel latches Q4K_ERR_DEVICE_TIMEOUT,
+// stops all roles, drains its own copies (bounded), frees TMEM and returns.
+#pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "common.cuh"
+
+namespace q4k {
+
+constexpr int kGemmBM = 256;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 64;
+constexpr int kStagesAW = 3;
+constexpr int kStagesB = 2;
+constexpr int kDqWarps = 8;
+constexpr int kGatherWarps = 4;
+constexpr uint32_t kATileBytes = kGemmBM * 128;       // 32 KB per K step
+constexpr uint32_t kBTileBytes = kGemmBN * 128;       // 32 KB per K step
+constexpr uint32_t kWRawPart = kGemmBN * 16;          // 4 KB: one 16-byte column per row
+constexpr uint32_t kWRawBytes = 3 * kWRawPart;        // header, quants 0-15, quants 16-31
+constexpr uint32_t kSmemA = 0;
+constexpr uint32_t kSmemB = kSmemA + kStagesAW * kATileBytes;
+constexpr uint32_t kSmemW = kSmemB + kStagesB * kBTileBytes;
+constexpr uint32_t kSmemBar = kSmemW + kStagesAW * kWRawBytes;
+constexpr uint32_t kSmemTotal = kSmemBar + 256;
+constexpr size_t kGemmSmemLaunch = kSmemTotal + 1024;  // + alignment slack
+
+struct GemmParams {
+  const uint8_t* W;        // dense [N][nkb][144]; grouped [E][N][nkb][144]
+  const uint16_t* X;       // activations bf16 (dense [M][K]; grouped: rows of A)
+  void* Y;                 // dense fp32 [M][N]; grouped fp32 [rows][N] or bf16 [rows][N/2]
+  int M, N, K;
+  int E;
+  const int32_t* offsets;  // grouped: [E+1]
+  const int32_t* gather;   // grouped: optional sorted row -> A row
+  int rows;                // grouped: total rows
+  int act;
+  int64_t expert_stride;
+  int n_tiles;             // N / 256
+  int m_tiles;             // dense: ceil(M/256); grouped: upper bound of (expert, m-tile) tasks
+};
+
+// ---- PTX wrappers -----------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
+
+// Bounded wait; returns false (after latching a timeout) if the phase never
+// completes or another role has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        latch_status(Q4K_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major, 128-byte swizzle shared-memory matrix descriptor: 8-row atoms of
+// 128-byte rows, atoms 1024 bytes apart (stride byte offset), descriptor
+// version 1, swizzle mode 2 (128B).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M=128, N=256.
+constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                                ((uint32_t)(128 >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIdescBf16), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
+        "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
+        "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Byte offset of 16-byte chunk `c` (0..7) of row `r` in a K-major 128-byte
+// swizzled tile (rows of 128 bytes, 8-row atoms of 1024 bytes).
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// ---- dequantisation of one row's 64-weight K step ---------------------------
+
+// Four consecutive weights (l = 4p .. 4p+3 of one sub-block) from the nibbles
+// of one quant word, as exact fp32 q*ds - dm. Each nibble is placed in the
+// mantissa of a float whose exponent makes the nibble's lowest bit worth 1
+// (2^E + q), so q*ds = fma(2^E + q, ds, -2^E*ds) exactly.
+__device__ __forceinline__ void dq4(uint32_t word, int h, float ds, float dm, float cA, float cB,
+                                    float (&w)[4]) {
+  // bytes 0,1 of the word in bits 0..15; bytes 2,3 after a 16-bit shift
+  const uint32_t lo = word, hi = word >> 16;
+  // nibble h of byte b (b in {0,1} of a 16-bit half) sits at bit 8b + 4h
+  const uint32_t mA = 0x0Fu << (4 * h), mB = 0x0F00u << (4 * h);
+  // exponents: bit 4h -> 2^(23-4h) unit; bit 8+4h -> 2^(15-4h) unit
+  const uint32_t eA = (uint32_t)(127 + 23 - 4 * h) << 23, eB = (uint32_t)(127 + 15 - 4 * h) << 23;
+  w[0] = fmaf(__uint_as_float((lo & mA) | eA), ds, cA) - dm;
+  w[1] = fmaf(__uint_as_float((lo & mB) | eB), ds, cB) - dm;
+  w[2] = fmaf(__uint_as_float((hi & mA) | eA), ds, cA) - dm;
+  w[3] = fmaf(__uint_as_float((hi & mB) | eB), ds, cB) - dm;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+// Dequantise weight row `r` for K step `ks` (super-block ks/4, chunk ks%4)
+// from its raw header (16 B) and 32 quant bytes into the swizzled B tile.
+__device__ __forceinline__ void dequant_row_step(uint8_t* btile, int r, int chunk, uint4 hdr, uint4 qa,
+                                                 uint4 qb) {
+  const float d = half_bits_to_float(hdr.x), dmin = half_bits_to_float(hdr.x >> 16);
+  const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};  // bytes l = 4i..4i+3
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t sc, m;
+    scale_min(hdr.y, hdr.z, hdr.w, 2 * chunk + h, sc, m);
+    const float ds = d * (float)sc;   // exact
+    const float dm = dmin * (float)m; // exact
+    const float cA = -ds * __uint_as_float((uint32_t)(127 + 23 - 4 * h) << 23);
+    const float cB = -ds * __uint_as_float((uint32_t)(127 + 15 - 4 * h) << 23);
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {  // 8 weights: l = 8*c8 .. 8*c8+7 of sub-block 2*chunk+h
+      float w0[4], w1[4];
+      dq4(qw[2 * c8], h, ds, dm, cA, cB, w0);
+      dq4(qw[2 * c8 + 1], h, ds, dm, cA, cB, w1);
+      // dq4 returns weights in byte order (b0, b1, b2, b3)
+      uint4 o;
+      o.x = pack_bf16x2(w0[0], w0[1]);
+      o.y = pack_bf16x2(w0[2], w0[3]);
+      o.z = pack_bf16x2(w1[0], w1[1]);
+      o.w = pack_bf16x2(w1[2], w1[3]);
+      *reinterpret_cast<uint4*>(btile + sw128_offset(r, 4 * h + c8)) = o;
+    }
+  }
+}
+
+// ---- the kernel -----------------------------------------------------------------
+
+template <bool GROUPED, bool GATHER, bool SWIGLU>
+__global__ void __launch_bounds__(32 * (2 + kDqWarps + (GATHER ? kGatherWarps : 0)), 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+               GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // barriers (8 bytes each) at kSmemBar: [0..2] full_aw, [3..5] empty_aw, [6..7] fullB,
+  // [8..9] emptyB, [10] tmem_full
+  auto bar_full_aw = [&](int s) { return sbase + kSmemBar + 8u * s; };
+  auto bar_empty_aw = [&](int s) { return sbase + kSmemBar + 8u * (3 + s); };
+  auto bar_full_b = [&](int s) { return sbase + kSmemBar + 8u * (6 + s); };
+  auto bar_empty_b = [&](int s) { return sbase + kSmemBar + 8u * (8 + s); };
+  const uint32_t bar_tmem_full = sbase + kSmemBar + 8u * 10;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kSmemBar + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemBar + 132);
+  int* task_info = reinterpret_cast<int*>(smem + kSmemBar + 136);  // expert, row_base, count, m0
+
+  // ---- tile coordinates ----
+  const int n_tile = (int)(blockIdx.x % (unsigned)p.n_tiles);
+  const int task = (int)(blockIdx.x / (unsigned)p.n_tiles);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesAW; ++s) {
+      mbar_init(bar_full_aw(s), GATHER ? 1 + kGatherWarps : 1);
+      mbar_init(bar_empty_aw(s), 1 + kDqWarps);
+    }
+    for (int s = 0; s < kStagesB; ++s) {
+      mbar_init(bar_full_b(s), kDqWarps);
+      mbar_init(bar_empty_b(s), 1);
+    }
+    mbar_init(bar_tmem_full, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    // Resolve the task: dense -> m tile; grouped -> (expert, m tile within expert).
+    int expert = 0, row_base = 0, count = p.M, m0 = task * kGemmBM;
+    if (GROUPED) {
+      int seen = 0;
+      expert = -1;
+      for (int e0 = 0; e0 < p.E && expert < 0; e0 += 32) {
+        const int e = e0 + lane;
+        int c = 0;
+        if (e < p.E) c = p.offsets[e + 1] - p.offsets[e];
+        const int t = (c + kGemmBM - 1) / kGemmBM;
+        int incl = t;
+        for (int off = 1; off < 32; off <<= 1) {
+          const int o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, task < seen + incl && t > 0);
+        if (hit) {
+          const int L = __ffs(hit) - 1;
+          expert = e0 + L;
+          const int incl_l = __shfl_sync(0xffffffffu, incl, L);
+          const int t_l = __shfl_sync(0xffffffffu, t, L);
+          m0 = (task - (seen + incl_l - t_l)) * kGemmBM;
+        }
+        seen += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (expert >= 0) {
+        row_base = p.offsets[expert];
+        count = p.offsets[expert + 1] - row_base;
+      }
+    }
+    if (lane == 0) {
+      task_info[0] = expert;
+      task_info[1] = row_base;
+      task_info[2] = count;
+      task_info[3] = m0;
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(const_cast<uint32_t*>(tmem_slot)))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int expert = task_info[0], row_base = task_info[1], count = task_info[2], m0 = task_info[3];
+  const bool active = GROUPED ? (expert >= 0) : (m0 < p.M);
+  const int nks = p.K / kGemmBK;
+
+  if (active) {
+    if (warp == 0) {
+      // ---------------- TMA producer ----------------
+      if (lane == 0) {
+        int issued = 0;
+        // weight rows of this tile in the [rows][row_bytes] view of W
+        int wy0, wy1;
+        if (SWIGLU) {
+          const int half = p.N / 2;
+          const int g0 = n_tile * (kGemmBN / 2);
+          wy0 = (GROUPED ? expert * p.N : 0) + g0;
+          wy1 = wy0 + half;
+        } else {
+          wy0 = (GROUPED ? expert * p.N : 0) + n_tile * kGemmBN;
+          wy1 = wy0 + kGemmBN / 2;
+        }
+        const int ay = GROUPED ? row_base + m0 : m0;
+        for (int ks = 0; ks < nks; ++ks) {
+          const int s = ks % kStagesAW, u = ks / kStagesAW;
+          if (u >= 1 && !mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag)) break;
+          const uint32_t bytes = (GATHER ? 0u : kATileBytes) + kWRawBytes;
+          mbar_arrive_expect_tx(bar_full_aw(s), bytes);
+          const uint32_t a_dst = sbase + kSmemA + s * kATileBytes;
+          if (!GATHER) {
+            tma_load_2d(a_dst, &tmap_x, ks * kGemmBK, ay, bar_full_aw(s));
+            tma_load_2d(a_dst + kATileBytes / 2, &tmap_x, ks * kGemmBK, ay + 128, bar_full_aw(s));
+          }
+          const int kb = ks >> 2, c = ks & 3;
+          const int xh = kb * BLOCK_BYTES, xq = xh + 16 + 32 * c;
+          const uint32_t w_dst = sbase + kSmemW + s * kWRawBytes;
+          tma_load_2d(w_dst, &tmap_w, xh, wy0, bar_full_aw(s));
+          tma_load_2d(w_dst + 2048, &tmap_w, xh, wy1, bar_full_aw(s));
+          tma_load_2d(w_dst + kWRawPart, &tmap_w, xq, wy0, bar_full_aw(s));
+          tma_load_2d(w_dst + kWRawPart + 2048, &tmap_w, xq, wy1, bar_full_aw(s));
+          tma_load_2d(w_dst + 2 * kWRawPart, &tmap_w, xq + 16, wy0, bar_full_aw(s));
+          tma_load_2d(w_dst + 2 * kWRawPart + 2048, &tmap_w, xq + 16, wy1, bar_full_aw(s));
+          ++issued;
+        }
+        // Drain: every issued stage must have landed before this CTA may exit. On the
+        // normal path the consumers have waited for all of them already.
+        if (*abort_flag) {
+          for (int ks = (issued > kStagesAW ? issued - kStagesAW : 0); ks < issued; ++ks) {
+            const int s = ks % kStagesAW, u = ks / kStagesAW;
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_full_aw(s), u & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+            }
+          }
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------- MMA issuer ----------------
+      if (lane == 0) {
+        bool ok = true;
+        for (int ks = 0; ks < nks && ok; ++ks) {
+          const int s = ks % kStagesAW, sb = ks % kStagesB;
+          ok = mbar_wait(bar_full_aw(s), (ks / kStagesAW) & 1, abort_flag) &&
+               mbar_wait(bar_full_b(sb), (ks / kStagesB) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a0 = sbase + kSmemA + s * kATileBytes;
+          const uint32_t b0 = sbase + kSmemB + sb * kBTileBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+              umma_bf16(tmem + h * 256, umma_desc_sw128(a0 + h * (kATileBytes / 2) + kk * 32),
+                        umma_desc_sw128(b0 + kk * 32), (ks | kk) != 0);
+            }
+          }
+          umma_commit(bar_empty_aw(s));
+          umma_commit(bar_empty_b(sb));
+        }
+        if (ok) umma_commit(bar_tmem_full);
+      }
+    } else if (warp < 2 + kDqWarps) {
+      // ---------------- dequantisation, then epilogue ----------------
+      const int r = (warp - 2) * 32 + lane;  // weight row of the B tile (0..255)
+      bool ok = true;
+      for (int ks = 0; ks < nks; ++ks) {
+        const int s = ks % kStagesAW, sb = ks % kStagesB, ub = ks / kStagesB;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_full_aw(s), (ks / kStagesAW) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        if (ub >= 1 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_empty_b(sb), (ub - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const uint8_t* wr = smem + kSmemW + s * kWRawBytes;
+        const uint4 hdr = *reinterpret_cast<const uint4*>(wr + r * 16);
+        const uint4 qa = *reinterpret_cast<const uint4*>(wr + kWRawPart + r * 16);
+        const uint4 qb = *reinterpret_cast<const uint4*>(wr + 2 * kWRawPart + r * 16);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty_aw(s));
+        dequant_row_step(smem + kSmemB + sb * kBTileBytes, r, ks & 3, hdr, qa, qb);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_full_b(sb));
+      }
+      // epilogue: warp w reads TMEM lanes 32*(w%4).. of accumulator half (w-2)/4
+      if (ok && __all_sync(0xffffffffu, mbar_wait(bar_tmem_full, 0, abort_flag))) {
+        tc_fence_after();
+        const int q = warp & 3, hm = (warp - 2) >> 2;
+        const int ml = hm * 128 + q * 32 + lane;  // row within the 256-row tile
+        const int mrow = m0 + ml;
+        const bool in = GROUPED ? (mrow < count) : (mrow < p.M);
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(hm * 256);
+        if (SWIGLU) {
+          const int half = p.N / 2;
+          uint16_t* out = static_cast<uint16_t*>(p.Y) + (int64_t)(row_base + mrow) * half +
+                          n_tile * (kGemmBN / 2);
+#pragma unroll 1
+          for (int cb = 0; cb < 4; ++cb) {
+            uint32_t g[32], u[32];
+            tmem_ld32(tbase + cb * 32, g);
+            tmem_ld32(tbase + 128 + cb * 32, u);
+            if (in) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 8) {
+                uint4 o;
+                uint32_t* op = &o.x;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float g0 = __uint_as_float(g[i + 2 * e]), g1 = __uint_as_float(g[i + 2 * e + 1]);
+                  const float u0 = __uint_as_float(u[i + 2 * e]), u1 = __uint_as_float(u[i + 2 * e + 1]);
+                  op[e] = pack_bf16x2(silu_mul(g0, u0), silu_mul(g1, u1));
+                }
+                *reinterpret_cast<uint4*>(out + cb * 32 + i) = o;
+              }
+            }
+          }
+        } else {
+          float* out = static_cast<float*>(p.Y) + (int64_t)((GROUPED ? row_base : 0) + mrow) * p.N +
+                       n_tile * kGemmBN;
+#pragma unroll 1
+          for (int cb = 0; cb < 8; ++cb) {
+            uint32_t v[32];
+            tmem_ld32(tbase + cb * 32, v);
+            if (in) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(out + cb * 32 + i) =
+                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+            }
+          }
+        }
+      }
+    } else if (GATHER) {
+      // ---------------- gathered activation rows (cp.async) ----------------
+      const int gt = (warp - 2 - kDqWarps) * 32 + lane;  // 0..127
+      const int ch = gt & 7;                              // 16-byte chunk within the 128-byte row
+      const int r0 = gt >> 3;                             // rows r0, r0+16, ...
+      int64_t src_row[kGemmBM / 16];
+#pragma unroll
+      for (int j = 0; j < kGemmBM / 16; ++j) {
+        const int ml = r0 + 16 * j;
+        const int mrow = m0 + ml;
+        src_row[j] = -1;
+        if (mrow < count) src_row[j] = p.gather ? p.gather[row_base + mrow] : (row_base + mrow);
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int ks = 0; ks < nks; ++ks) {
+        const int s = ks % kStagesAW, u = ks / kStagesAW;
+        if (u >= 1 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const uint32_t a_dst = sbase + kSmemA + s * kATileBytes;
+#pragma unroll
+        for (int j = 0; j < kGemmBM / 16; ++j) {
+          const int ml = r0 + 16 * j;
+          const int64_t sr = src_row[j];
+          const uint16_t* src = p.X + (sr < 0 ? 0 : sr) * p.K + ks * kGemmBK + ch * 8;
+          cp_async_16(a_dst + sw128_offset(ml, ch), src, sr < 0 ? 0u : 16u);
+        }
+        cp_async_commit();
+        ++issued;
+        if (ks >= 1) {
+          cp_async_wait<1>();
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_full_aw((ks - 1) % kStagesAW));
+        }
+      }
+      cp_async_wait<0>();
+      if (ok && issued > 0) {
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_full_aw((issued - 1) % kStagesAW));
+      }
+    }
+  }
+
+  // ---- teardown ----
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ---- host side ----------------------------------------------------------------------
+
+inline PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
+            cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// bf16 [rows][K] activations, box 64 x 128, 128-byte swizzle.
+inline bool make_tmap_x(CUtensorMap* m, const void* base, int64_t rows, int K) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raw Q4_K rows viewed as bytes [rows][row_bytes], box 16 bytes x 128 rows.
+inline bool make_tmap_w(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {16, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool GROUPED, bool GATHER, bool SWIGLU>
+inline q4k_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
+                                cudaStream_t s) {
+  auto* k = gemm_tc_kernel<GROUPED, GATHER, SWIGLU>;
+  static std::atomic<int> attr_set[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return Q4K_ERR_CUDA;
+  if (!attr_set[dev].load()) {
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kGemmSmemLaunch) != cudaSuccess)
+      return Q4K_ERR_LAUNCH;
+    attr_set[dev].store(1);
+  }
+  const dim3 grid((unsigned)(p.n_tiles * p.m_tiles));
+  const dim3 block(32 * (2 + kDqWarps + (GATHER ? kGatherWarps : 0)));
+  k<<<grid, block, kGemmSmemLaunch, s>>>(tx, tw, p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? Q4K_OK : Q4K_ERR_LAUNCH;
+}
+
+inline q4k_status launch_gemm_tc(GemmParams p, cudaStream_t s) {
+  CUtensorMap tx, tw;
+  const int64_t row_bytes = (int64_t)(p.K / QK) * BLOCK_BYTES;
+  if (!make_tmap_x(&tx, p.X, p.M, p.K) || !make_tmap_w(&tw, p.W, p.N, row_bytes))
+    return Q4K_ERR_CUDA;
+  p.n_tiles = p.N / kGemmBN;
+  p.m_tiles = (p.M + kGemmBM - 1) / kGemmBM;
+  return launch_gemm_t<false, false, false>(tx, tw, p, s);
+}
+
+// Grouped: tasks are (expert, 256-row tile of that expert's rows); their number
+// is at most ceil(rows/256) + min(E, rows). CTAs past the real count exit.
+inline q4k_status launch_gemm_tc_grouped(GemmParams p, cudaStream_t s) {
+  CUtensorMap tx, tw;
+  const int64_t row_bytes = (int64_t)(p.K / QK) * BLOCK_BYTES;
+  const bool gather = p.gather != nullptr;
+  // Without a gather the A rows are the sorted rows themselves (TMA); with one they
+  // are fetched by index and the activation tensor map is unused.
+  if (!make_tmap_x(&tx, p.X, gather ? 1 : p.rows, p.K) ||
+      !make_tmap_w(&tw, p.W, (int64_t)p.E * p.N, row_bytes))
+    return Q4K_ERR_CUDA;
+  const bool swiglu = p.act == Q4K_ACT_SWIGLU;
+  if (swiglu && (p.N / 2) % (kGemmBN / 2)) return Q4K_ERR_UNSUPPORTED;
+  p.n_tiles = swiglu ? (p.N / 2) / (kGemmBN / 2) : p.N / kGemmBN;
+  p.m_tiles = (p.rows + kGemmBM - 1) / kGemmBM + std::min(p.E, p.rows);
+  if (gather) {
+    return swiglu ? launch_gemm_t<true, true, true>(tx, tw, p, s)
+                  : launch_gemm_t<true, true, false>(tx, tw, p, s);
+  }
+  return swiglu ? launch_gemm_t<true, false, true>(tx, tw, p, s)
+                : launch_gemm_t<true, false, false>(tx, tw, p, s);
+}
+
+}  // namespace q4k

@@ -1,0 +1,190 @@
+// Mixture-of-experts routing, token permutation and weighted combine
+// (hipEngine 0.3.0 README, "Architecture at a glance": the moe kernel family;
+// "Core principles": the gate_combine_residual composite).
+#pragma once
+#include "common.cuh"
+
+namespace q4k {
+
+constexpr int kRouteWarps = 8;
+constexpr int kRouteTokPerWarp = 4;
+constexpr int kRouteTokPerCta = kRouteWarps * kRouteTokPerWarp;  // tokens per histogram tile
+constexpr int kMaxE = 1024;
+constexpr int kMaxTopk = 16;
+
+// Is (va, ia) ranked before (vb, ib)? Higher logit first; equal logits -> lower id.
+__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+// Routing: one warp per token. Iterated arg-max over the E logits (each lane
+// holds E/32 of them), softmax over the selected logits in fp32. Each CTA
+// also writes the expert histogram of its tile of tokens to counts[cta][E].
+__global__ void __launch_bounds__(32 * kRouteWarps)
+route_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* __restrict__ ids,
+             float* __restrict__ wts, int32_t* __restrict__ counts) {
+  __shared__ int hist[kMaxE];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int per_lane = (E + 31) / 32;  // <= 32
+  for (int tt = 0; tt < kRouteTokPerWarp; ++tt) {
+    const int tok = blockIdx.x * kRouteTokPerCta + warp * kRouteTokPerWarp + tt;
+    if (tok >= M) break;  // uniform per warp
+    const float* row = logits + (int64_t)tok * E;
+    float v[32];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int e = i * 32 + lane;
+      v[i] = (i < per_lane && e < E) ? row[e] : 0.f;
+    }
+    float sel_v[kMaxTopk];
+    int sel_i[kMaxTopk];
+    for (int k = 0; k < topk; ++k) {
+      float bv = -INFINITY;  // a lane with no candidate left never wins
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int e = i * 32 + lane;
+        if (i < per_lane && e < E && !((taken >> i) & 1u) && ranks_before(v[i], e, bv, bi)) {
+          bv = v[i];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (ranks_before(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      sel_v[k] = bv;
+      sel_i[k] = bi;
+    }
+    // softmax over the selected logits; sel_v[0] is the largest
+    float den = 0.f;
+    for (int k = 0; k < topk; ++k) den += expf(sel_v[k] - sel_v[0]);
+    if (lane < topk) {
+      float num = 0.f;
+      int id = 0;
+      for (int k = 0; k < topk; ++k)
+        if (k == lane) { num = expf(sel_v[k] - sel_v[0]); id = sel_i[k]; }
+      ids[(int64_t)tok * topk + lane] = id;
+      wts[(int64_t)tok * topk + lane] = num / den;
+      atomicAdd(&hist[id], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+// Permutation: CTA b places the (token, slot) pairs of its token tile. Its
+// base position for expert e is offsets[e] + (rows of e in tiles < b); inside
+// the tile the pairs are placed in flat-index order (stable sort by expert).
+__global__ void __launch_bounds__(256)
+permute_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ counts, int M, int E,
+               int topk, int ntiles, int32_t* __restrict__ expert_offsets, int32_t* __restrict__ perm,
+               int32_t* __restrict__ inv_perm, int32_t* __restrict__ row_token) {
+  __shared__ int base[kMaxE];
+  __shared__ int total[kMaxE];
+  __shared__ int warp_sums[32];
+  const int b = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int before = 0, all = 0;
+    for (int bb = 0; bb < ntiles; ++bb) {
+      const int c = counts[(int64_t)bb * E + e];
+      all += c;
+      if (bb < b) before += c;
+    }
+    total[e] = all;
+    base[e] = before;
+  }
+  __syncthreads();
+  // exclusive scan of total[] over experts (E <= 1024): thread i owns a run of experts
+  {
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = threadIdx.x * per;
+    int run = 0;
+    for (int e = e0; e < e0 + per && e < E; ++e) run += total[e];
+    // block-wide exclusive scan of run
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = run;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int nw = blockDim.x / 32;
+      int ws = lane < nw ? warp_sums[lane] : 0;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, ws, off);
+        if (lane >= off) ws += o;
+      }
+      if (lane < nw) warp_sums[lane] = ws;  // inclusive
+    }
+    __syncthreads();
+    int excl = incl - run + (warp > 0 ? warp_sums[warp - 1] : 0);
+    for (int e = e0; e < e0 + per && e < E; ++e) {
+      const int tot = total[e];
+      if (b == 0) expert_offsets[e] = excl;
+      base[e] += excl;
+      excl += tot;
+    }
+    if (b == 0 && threadIdx.x == blockDim.x - 1) expert_offsets[E] = excl;  // grand total
+  }
+  __syncthreads();
+  // stable placement by warp 0, 32 pairs at a time in flat-index order
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int f0 = b * kRouteTokPerCta * topk;
+    const int f1 = min(M, (b + 1) * kRouteTokPerCta) * topk;
+    for (int fs = f0; fs < f1; fs += 32) {
+      const int f = fs + lane;
+      const bool act = f < f1;
+      const int e = act ? ids[f] : -1 - lane;
+      const bool ok = !act || (e >= 0 && e < E);
+      if (!ok) latch_status(Q4K_ERR_DEVICE_BOUNDS);
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      if (act && ok) {
+        const int pos = base[e] + rank;
+        perm[pos] = f;
+        inv_perm[f] = pos;
+        row_token[pos] = f / topk;
+      }
+      __syncwarp();
+      if (act && ok && rank == __popc(peers) - 1) base[e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+}
+
+// y[t][h] = sum_j w[t][j] * O[inv_perm[t*topk + j]][h], j in increasing order.
+__global__ void __launch_bounds__(256)
+combine_kernel(const float* __restrict__ O, const int32_t* __restrict__ inv_perm,
+               const float* __restrict__ w, int M, int topk, int H, float* __restrict__ Y) {
+  const int t = blockIdx.y;
+  const int h4 = blockIdx.x * blockDim.x + threadIdx.x;  // index of a float4
+  if (h4 * 4 >= H) return;
+  const int rows = M * topk;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < topk; ++j) {
+    const int r = inv_perm[(int64_t)t * topk + j];
+    if (r < 0 || r >= rows) {
+      latch_status(Q4K_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    const float wj = w[(int64_t)t * topk + j];
+    const float4 o = *reinterpret_cast<const float4*>(O + (int64_t)r * H + 4 * h4);
+    acc.x = fmaf(wj, o.x, acc.x);
+    acc.y = fmaf(wj, o.y, acc.y);
+    acc.z = fmaf(wj, o.z, acc.z);
+    acc.w = fmaf(wj, o.w, acc.w);
+  }
+  *reinterpret_cast<float4*>(Y + (int64_t)t * H + 4 * h4) = acc;
+}
+
+}  // namespace q4k

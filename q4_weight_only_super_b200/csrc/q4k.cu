@@ -1,0 +1,296 @@
+// C ABI of the Q4_K library (declared in include/q4k.h): argument checks,
+// launch configuration and kernel launches. All kernels live in the
+// included headers; this is the only translation unit of libq4k.so.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "common.cuh"
+#include "dequant.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "moe.cuh"
+
+using namespace q4k;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device. `set_to` must be
+// distinct for every kernel (the caller owns one per kernel instantiation).
+template <typename F>
+cudaError_t ensure_smem(F* func, size_t bytes, std::atomic<size_t> (&set_to)[kMaxDevices]) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (bytes <= 48 * 1024 || set_to[dev].load() >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(func),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) set_to[dev].store(bytes);
+  return e;
+}
+
+q4k_status launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return Q4K_OK;
+  cudaGetLastError();  // clear the sticky launch error of this thread
+  return Q4K_ERR_LAUNCH;
+}
+
+// ---------------------------------------------------------------- GEMV ----
+
+struct GemvCfg {
+  int mt, warps, ksplit, kc;
+};
+
+// Launch shape for `tokens` (<= 32) tokens against `rows_out` output rows per
+// matrix and `nkb` super-blocks per row, with `groups` matrices (experts)
+// processed side by side. Depends only on (tokens class, rows, nkb, groups).
+GemvCfg pick_gemv(int tokens, int rows_out, int nkb, int groups) {
+  GemvCfg c;
+  c.mt = tokens <= 8 ? 1 : (tokens <= 16 ? 2 : 4);
+  c.warps = c.mt == 4 ? 8 : 4;
+  c.kc = c.mt == 1 ? 8 : (c.mt == 2 ? 4 : 2);
+  const int tile_rows = 16 * c.warps;
+  const int tiles = (rows_out + tile_rows - 1) / tile_rows;
+  const long target = 4L * 148;
+  long ks = (target + (long)tiles * groups - 1) / ((long)tiles * groups);
+  ks = std::max(1L, std::min<long>(ks, 8));
+  ks = std::min<long>(ks, nkb);
+  c.ksplit = (int)ks;
+  c.kc = std::min(c.kc, (nkb + c.ksplit - 1) / c.ksplit);
+  return c;
+}
+
+template <int MT, int WARPS, bool GROUPED, bool SWIGLU>
+q4k_status launch_gemv_t(const GemvParams& p, int tiles, int groups, cudaStream_t s) {
+  auto* k = gemv_kernel<MT, WARPS, GROUPED, SWIGLU>;
+  static std::atomic<size_t> smem_set[kMaxDevices];  // one per instantiation
+  const size_t smem = gemv_smem_bytes<MT, WARPS>(p.kc);
+  if (ensure_smem(k, smem, smem_set) != cudaSuccess) return Q4K_ERR_LAUNCH;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(tiles * p.ksplit), (unsigned)groups, 1);
+  cfg.blockDim = dim3(32 * WARPS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return launch_status(cudaLaunchKernelEx(&cfg, k, p));
+}
+
+template <bool GROUPED, bool SWIGLU>
+q4k_status launch_gemv(const GemvCfg& c, GemvParams p, int rows_out, int groups, cudaStream_t s) {
+  p.ksplit = c.ksplit;
+  p.kc = c.kc;
+  const int tiles = (rows_out + 16 * c.warps - 1) / (16 * c.warps);
+  if (c.mt == 1) return launch_gemv_t<1, 4, GROUPED, SWIGLU>(p, tiles, groups, s);
+  if (c.mt == 2) return launch_gemv_t<2, 4, GROUPED, SWIGLU>(p, tiles, groups, s);
+  return launch_gemv_t<4, 8, GROUPED, SWIGLU>(p, tiles, groups, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* q4k_status_string(int s) {
+  switch (s) {
+    case Q4K_OK: return "ok";
+    case Q4K_ERR_NULL: return "null pointer";
+    case Q4K_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case Q4K_ERR_SHAPE: return "invalid shape";
+    case Q4K_ERR_UNSUPPORTED: return "unsupported shape";
+    case Q4K_ERR_WORKSPACE: return "workspace missing or too small";
+    case Q4K_ERR_LAUNCH: return "kernel launch failed";
+    case Q4K_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case Q4K_ERR_DEVICE_BOUNDS: return "device-side index out of range";
+    case Q4K_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+q4k_status q4k_dequant(const void* W, int64_t nblocks, int out_bf16, void* out, void* stream) {
+  if (nblocks < 0) return Q4K_ERR_SHAPE;
+  if (nblocks == 0) return Q4K_OK;
+  if (!W || !out) return Q4K_ERR_NULL;
+  if (!aligned16(W) || !aligned16(out)) return Q4K_ERR_ALIGN;
+  const int64_t threads = nblocks * 32;
+  const int64_t grid = (threads + 255) / 256;
+  if (grid > 0x7fffffffLL) return Q4K_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (out_bf16)
+    dequant_kernel<true><<<(unsigned)grid, 256, 0, s>>>(static_cast<const uint8_t*>(W), nblocks, out);
+  else
+    dequant_kernel<false><<<(unsigned)grid, 256, 0, s>>>(static_cast<const uint8_t*>(W), nblocks, out);
+  return launch_status(cudaGetLastError());
+}
+
+q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (M == 0 || N == 0) return Q4K_OK;
+  if (!W || !X || !Y) return Q4K_ERR_NULL;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(Y)) return Q4K_ERR_ALIGN;
+  if (M > 32 || N % 16) return Q4K_ERR_UNSUPPORTED;
+  GemvParams p = {};
+  p.W = static_cast<const uint8_t*>(W);
+  p.X = X;
+  p.out = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nkb = K / QK;
+  const GemvCfg c = pick_gemv(M, N, p.nkb, 1);
+  return launch_gemv<false, false>(c, p, N, 1, static_cast<cudaStream_t>(stream));
+}
+
+q4k_status q4k_gemm(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws,
+                    size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (M == 0 || N == 0) return Q4K_OK;
+  if (!W || !X || !Y) return Q4K_ERR_NULL;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(Y)) return Q4K_ERR_ALIGN;
+  if (N % kGemmBN) return Q4K_ERR_UNSUPPORTED;
+  GemmParams p = {};
+  p.W = static_cast<const uint8_t*>(W);
+  p.X = X;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  return launch_gemm_tc(p, static_cast<cudaStream_t>(stream));
+}
+
+size_t q4k_workspace_bytes(int op, int M, int N, int K, int E, int topk) {
+  (void)N;
+  (void)K;
+  (void)topk;
+  if (op == Q4K_OP_ROUTE) {
+    if (M <= 0 || E <= 0) return 0;
+    const size_t tiles = (size_t)(M + kRouteTokPerCta - 1) / kRouteTokPerCta;
+    return tiles * (size_t)E * sizeof(int32_t);
+  }
+  return 0;
+}
+
+q4k_status moe_route_permute(const float* logits, int M, int E, int topk, int32_t* topk_ids,
+                             float* topk_w, int32_t* expert_offsets, int32_t* perm,
+                             int32_t* inv_perm, int32_t* row_token, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (M < 0 || E <= 0 || topk <= 0) return Q4K_ERR_SHAPE;
+  if (E > kMaxE || topk > kMaxTopk || topk > E) return Q4K_ERR_UNSUPPORTED;
+  if ((int64_t)M * topk > 0x7fffffffLL) return Q4K_ERR_UNSUPPORTED;
+  if (!expert_offsets) return Q4K_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    return cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), s) == cudaSuccess
+               ? Q4K_OK : Q4K_ERR_CUDA;
+  }
+  if (!logits || !topk_ids || !topk_w || !perm || !inv_perm || !row_token || !ws)
+    return Q4K_ERR_NULL;
+  if (!aligned16(logits) || !aligned16(topk_ids) || !aligned16(topk_w) ||
+      !aligned16(expert_offsets) || !aligned16(perm) || !aligned16(inv_perm) ||
+      !aligned16(row_token) || !aligned16(ws))
+    return Q4K_ERR_ALIGN;
+  if (ws_bytes < q4k_workspace_bytes(Q4K_OP_ROUTE, M, 0, 0, E, topk)) return Q4K_ERR_WORKSPACE;
+  const int tiles = (M + kRouteTokPerCta - 1) / kRouteTokPerCta;
+  int32_t* counts = static_cast<int32_t*>(ws);
+  route_kernel<<<tiles, 32 * kRouteWarps, 0, s>>>(logits, M, E, topk, topk_ids, topk_w, counts);
+  q4k_status st = launch_status(cudaGetLastError());
+  if (st != Q4K_OK) return st;
+  permute_kernel<<<tiles, 256, 0, s>>>(topk_ids, counts, M, E, topk, tiles, expert_offsets, perm,
+                                       inv_perm, row_token);
+  return launch_status(cudaGetLastError());
+}
+
+q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uint16_t* A,
+                           const int32_t* row_gather, const int32_t* expert_offsets, int rows,
+                           int max_rows_hint, int act, void* out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (E <= 0 || N <= 0 || K <= 0 || K % QK || rows < 0 || max_rows_hint < 0) return Q4K_ERR_SHAPE;
+  if (act != Q4K_ACT_NONE && act != Q4K_ACT_SWIGLU) return Q4K_ERR_UNSUPPORTED;
+  if (rows == 0) return Q4K_OK;
+  if (!W_experts || !A || !expert_offsets || !out) return Q4K_ERR_NULL;
+  if (!aligned16(W_experts) || !aligned16(A) || !aligned16(out) || !aligned16(expert_offsets) ||
+      (row_gather && !aligned16(row_gather)))
+    return Q4K_ERR_ALIGN;
+  if (N % 32 || E > kMaxE) return Q4K_ERR_UNSUPPORTED;
+  const int nkb = K / QK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int hint = std::min(max_rows_hint == 0 ? rows : max_rows_hint, rows);
+  if (hint <= 32) {
+    GemvParams p = {};
+    p.W = static_cast<const uint8_t*>(W_experts);
+    p.X = A;
+    p.out = out;
+    p.offsets = expert_offsets;
+    p.gather = row_gather;
+    p.N = N;
+    p.K = K;
+    p.nkb = nkb;
+    p.E = E;
+    p.expert_stride = (int64_t)N * nkb * BLOCK_BYTES;
+    const int groups = std::min(E, rows);
+    // The same launch shape (hence the same K partition and summation order) for
+    // the fp32 and the SwiGLU outputs: a SwiGLU CTA covers as many weight rows.
+    const GemvCfg c = pick_gemv(hint, N, nkb, groups);
+    if (act == Q4K_ACT_SWIGLU) return launch_gemv<true, true>(c, p, N, groups, s);
+    return launch_gemv<true, false>(c, p, N, groups, s);
+  }
+  if (N % kGemmBN) return Q4K_ERR_UNSUPPORTED;
+  GemmParams p = {};
+  p.W = static_cast<const uint8_t*>(W_experts);
+  p.X = A;
+  p.Y = out;
+  p.N = N;
+  p.K = K;
+  p.E = E;
+  p.offsets = expert_offsets;
+  p.gather = row_gather;
+  p.rows = rows;
+  p.act = act;
+  p.expert_stride = (int64_t)N * nkb * BLOCK_BYTES;
+  return launch_gemm_tc_grouped(p, s);
+}
+
+q4k_status moe_combine(const float* O, const int32_t* inv_perm, const float* topk_w, int M,
+                       int topk, int H, float* Y, void* stream) {
+  if (M < 0 || topk <= 0 || H <= 0) return Q4K_ERR_SHAPE;
+  if (M == 0) return Q4K_OK;
+  if (!O || !inv_perm || !topk_w || !Y) return Q4K_ERR_NULL;
+  if (!aligned16(O) || !aligned16(inv_perm) || !aligned16(topk_w) || !aligned16(Y))
+    return Q4K_ERR_ALIGN;
+  if (H % 4 || M > 65535 || topk > kMaxTopk) return Q4K_ERR_UNSUPPORTED;
+  const int n4 = H / 4;
+  dim3 grid((n4 + 255) / 256, M);
+  combine_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(O, inv_perm, topk_w, M, topk,
+                                                                       H, Y);
+  return launch_status(cudaGetLastError());
+}
+
+q4k_status q4k_last_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return Q4K_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return Q4K_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return Q4K_ERR_CUDA;
+  return static_cast<q4k_status>(v);
+}
+
+}  // extern "C"

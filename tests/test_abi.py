@@ -1,0 +1,78 @@
+"""CPU checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "q4k.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(?:q4k_status|size_t|const char\*)\s+(\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from q4_weight_only_super_b200 import build
+    build.build()
+    import q4_weight_only_super_b200 as q
+    return q.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("q4k_gemv", "q4k_gemm", "moe_route_permute", "moe_q4k_grouped", "moe_combine"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    import q4_weight_only_super_b200 as q
+    for name in _declared():
+        assert hasattr(L, name), name
+        assert name in q.EXPORTS, f"binding lacks {name}"
+
+
+def test_status_strings(L):
+    assert L.q4k_status_string(0) == b"ok"
+    assert b"unsupported" in L.q4k_status_string(4)
+
+
+def test_argument_errors_return_before_launch(L):
+    fake = 4096  # never dereferenced: every call below fails validation first
+    # K not a multiple of 256
+    assert L.q4k_gemv(fake, fake, fake, 1, 16, 100, None) == 3
+    # null pointers
+    assert L.q4k_gemv(None, fake, fake, 1, 16, 256, None) == 1
+    # misaligned pointer
+    assert L.q4k_gemv(fake + 4, fake, fake, 1, 16, 256, None) == 2
+    # M > 32 is not a GEMV shape
+    assert L.q4k_gemv(fake, fake, fake, 33, 16, 256, None) == 4
+    # N not a multiple of 16
+    assert L.q4k_gemv(fake, fake, fake, 1, 24, 256, None) == 4
+    # GEMM N not a multiple of 256
+    assert L.q4k_gemm(fake, fake, fake, 4, 128, 256, None, 0, None) == 4
+    # routing: too many experts / top-k
+    assert L.moe_route_permute(fake, 4, 2048, 8, fake, fake, fake, fake, fake, fake, fake, 1 << 20,
+                               None) == 4
+    assert L.moe_route_permute(fake, 4, 128, 17, fake, fake, fake, fake, fake, fake, fake, 1 << 20,
+                               None) == 4
+    # routing: workspace too small
+    assert L.moe_route_permute(fake, 64, 128, 8, fake, fake, fake, fake, fake, fake, fake, 16,
+                               None) == 5
+    # grouped: bad activation code, combine: H % 4
+    assert L.moe_q4k_grouped(fake, 4, 64, 256, fake, None, fake, 8, 8, 7, fake, None, 0, None) == 4
+    assert L.moe_combine(fake, fake, fake, 2, 2, 6, fake, None) == 4
+    # empty problems are no-ops
+    assert L.q4k_gemv(None, None, None, 0, 16, 256, None) == 0
+    assert L.moe_combine(None, None, None, 0, 2, 8, None, None) == 0
+
+
+def test_workspace_size(L):
+    assert L.q4k_workspace_bytes(2, 4096, 0, 0, 128, 8) == 128 * 128 * 4
+    assert L.q4k_workspace_bytes(2, 1, 0, 0, 128, 8) == 128 * 4
+    assert L.q4k_workspace_bytes(1, 4096, 17408, 5120, 0, 0) == 0

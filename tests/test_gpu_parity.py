@@ -1,0 +1,257 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Bit-exact for dequantised weights, routing ids, offsets and permutations;
+|y - y_ref| <= 2e-3 * sum|w*x| per fp32 matmul output; routing weights within
+1e-6; combine within 1e-6 * sum|w*O|; SwiGLU output within one bf16 ulp of the
+value rounded from the GPU's own gate/up products.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import q4k as O
+from tests.gpu_util import bf16_ulp, dev, host, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+q = pytest.importorskip("q4_weight_only_super_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    q.lib()
+    yield
+    assert q.q4k_last_device_status() == 0
+
+
+def _assert_tol(y, Y, S, what=""):
+    ok, ratio = O.check_tolerance(y, Y, S)
+    assert ok, f"{what}: worst err/S = {ratio:.3e} (limit 2e-3)"
+    return ratio
+
+
+# ------------------------------------------------------------------ dequant --
+
+def _edge_blocks():
+    blocks = []
+    for d, dmin in [(65504.0, 0.0), (6e-8, 6e-8), (1.0, 65504.0), (0.0, 0.0), (-2.0, -1.5)]:
+        for (sc, m, qv) in [(63, 63, 15), (1, 0, 1), (0, 63, 0)]:
+            blocks.append(O.make_block(d, dmin, [sc] * 8, [m] * 8, [qv] * 256))
+    return np.stack(blocks)
+
+
+@pytest.mark.parametrize("out_bf16", [False, True])
+def test_dequant_bit_exact(out_bf16):
+    W, _ = synth.gemv_small(0)
+    blocks = np.concatenate([W.reshape(-1, 144), _edge_blocks()])
+    out = host(q.q4k_dequant(dev(blocks), out_bf16=out_bf16))
+    if out_bf16:
+        ref = O.dequant_bf16_bits(blocks[None])[0]
+        assert np.array_equal(out, ref)
+    else:
+        ref = O.dequant_f32(blocks[None])[0]
+        assert np.array_equal(out.view(np.uint32), ref.view(np.uint32))
+
+
+def test_dequant_empty():
+    out = torch.empty(16, dtype=torch.float32, device="cuda")
+    assert q.lib().q4k_dequant(out.data_ptr(), 0, 0, out.data_ptr(), None) == 0
+
+
+# --------------------------------------------------------------------- GEMV --
+
+def test_gemv_single_matrix_full():
+    W, X = synth.gemv_small(0)
+    y = host(q.q4k_gemv(dev(W), dev(X), 256, 2048))
+    Y, S = O.matmul_ref(W, X)
+    _assert_tol(y, Y, S, "256x2048 M=1")
+
+
+@pytest.mark.parametrize("N,K", [(16, 256), (48, 512), (80, 1792), (272, 4096), (1040, 256 * 69)])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 17, 32])
+def test_gemv_shapes(N, K, M):
+    W, X = synth.gemv_small(100 + M, N=N, K=K, M=M)
+    y = host(q.q4k_gemv(dev(W), dev(X), N, K))
+    Y, S = O.matmul_ref(W, X)
+    _assert_tol(y, Y, S, f"N={N} K={K} M={M}")
+
+
+@pytest.fixture(scope="module")
+def decode_inputs():
+    inp = synth.dense_decode(1)
+    d = {k: dev(v) for k, v in inp.items()}
+    return inp, d
+
+
+@pytest.mark.parametrize("proj", ["gate_up", "down"])
+@pytest.mark.parametrize("M", [1, 4, 8, 16, 32])
+def test_gemv_dense_decode_sampled(decode_inputs, proj, M):
+    inp, d = decode_inputs
+    W, X = inp[f"W_{proj}"], inp[f"X_{proj}"][:M]
+    N, K = W.shape[0], W.shape[1] * 256
+    y = host(q.q4k_gemv(d[f"W_{proj}"], d[f"X_{proj}"][:M], N, K))
+    rows = sample_rows(N, 384, seed=M)
+    Y, S = O.matmul_rows_ref(W, X, rows)
+    _assert_tol(y[:, rows], Y, S, f"{proj} M={M}")
+
+
+def test_gemv_batch_invariance_and_determinism(decode_inputs):
+    """Row m of an M-token call is bit-identical to the one-token call on row m."""
+    inp, d = decode_inputs
+    N, K = inp["W_down"].shape[0], inp["W_down"].shape[1] * 256
+    W, X = d["W_down"], d["X_down"]
+    y32 = q.q4k_gemv(W, X[:32], N, K)
+    assert torch.equal(y32, q.q4k_gemv(W, X[:32], N, K))
+    for M in (4, 8, 16):
+        assert torch.equal(q.q4k_gemv(W, X[:M], N, K), y32[:M])
+    for m in (0, 7, 13, 31):
+        assert torch.equal(q.q4k_gemv(W, X[m:m + 1], N, K)[0], y32[m])
+
+
+# ---------------------------------------------------------------- MoE route --
+
+def _route_and_check(logits, topk=8):
+    E = logits.shape[1]
+    r = q.moe_route_permute(dev(logits), topk)
+    ids, w = O.route_topk(logits, topk)
+    offs, perm, inv, rt = O.permute(ids, E)
+    assert np.array_equal(host(r["topk_ids"]), ids)
+    assert np.abs(host(r["topk_w"]).astype(np.float64) - w).max() <= 1e-6
+    assert np.array_equal(host(r["expert_offsets"]), offs)
+    assert np.array_equal(host(r["perm"]), perm)
+    assert np.array_equal(host(r["inv_perm"]), inv)
+    assert np.array_equal(host(r["row_token"]), rt)
+    return r
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 33, 100])
+def test_route_permute_decode(M):
+    _route_and_check(synth.moe_layer(3, M, E=128, H=256, F=256)["logits"])
+
+
+def test_route_permute_prefill_skewed():
+    inp = synth.moe_layer(4, 4096, E=128, H=256, F=256, hot=16)
+    _route_and_check(inp["logits"])
+
+
+def test_route_ties_and_small_E():
+    rng = np.random.default_rng(9)
+    L = (rng.standard_normal((70, 128)) * 2).astype(np.float32)
+    L[0] = 0.25
+    L[1, [5, 77, 99]] = 7.0
+    L[2, ::2] = L[2, 1::2]
+    _route_and_check(L)
+    _route_and_check((rng.standard_normal((50, 40))).astype(np.float32), topk=3)
+    _route_and_check((rng.standard_normal((9, 1000))).astype(np.float32), topk=16)
+
+
+def test_route_zero_tokens():
+    offs = torch.full((129,), -1, dtype=torch.int32, device="cuda")
+    st = q.lib().moe_route_permute(None, 0, 128, 8, None, None, offs.data_ptr(), None, None, None,
+                                   None, 0, None)
+    assert st == 0 and torch.count_nonzero(offs).item() == 0
+
+
+# -------------------------------------------------------------- MoE combine --
+
+def test_combine():
+    rng = np.random.default_rng(4)
+    M, topk, H = 37, 8, 2048
+    Od = rng.standard_normal((M * topk, H)).astype(np.float32)
+    inv = rng.permutation(M * topk).astype(np.int32)
+    w = rng.random((M, topk)).astype(np.float32)
+    y = host(q.moe_combine(dev(Od), dev(inv), dev(w), M, topk, H))
+    Y, S = O.combine_ref(Od, inv, w)
+    assert np.all(np.abs(y - Y) <= 1e-6 * S + 1e-30)
+
+
+def test_combine_bad_index_latches_status():
+    M, topk, H = 2, 2, 8
+    Od = torch.zeros(M * topk, H, device="cuda")
+    inv = torch.tensor([0, 1, 2, 99], dtype=torch.int32, device="cuda")
+    w = torch.ones(M, topk, device="cuda")
+    q.moe_combine(Od, inv, w, M, topk, H)
+    assert q.q4k_last_device_status() == 8  # Q4K_ERR_DEVICE_BOUNDS
+    assert q.q4k_last_device_status() == 0
+
+
+# ------------------------------------------------------- MoE expert matmuls --
+
+def _moe_stagewise(inp, M, hint=None):
+    """Run route -> gate_up (fp32 and SwiGLU) -> down -> combine; check every stage."""
+    E, H, F, topk = inp["E"], inp["H"], inp["F"], 8
+    r = _route_and_check(inp["logits"], topk)
+    rows = M * topk
+    hint = M if hint is None else hint
+    Wgu, Wdn, X = dev(inp["W_gate_up"]), dev(inp["W_down"]), dev(inp["X"])
+    offs_h = host(r["expert_offsets"])
+    rt_h = host(r["row_token"])
+    sample = sample_rows(rows, 384, seed=M) if rows > 512 else np.arange(rows)
+
+    GU = q.moe_q4k_grouped(Wgu, E, 2 * F, H, X, r["expert_offsets"], rows, hint, q.ACT_NONE,
+                           row_gather=r["row_token"])
+    Yg, Sg = O.grouped_ref(inp["W_gate_up"], inp["X"], offs_h, row_gather=rt_h, rows=sample)
+    ratio_gu = _assert_tol(host(GU)[sample], Yg, Sg, "gate_up")
+
+    h = q.moe_q4k_grouped(Wgu, E, 2 * F, H, X, r["expert_offsets"], rows, hint, q.ACT_SWIGLU,
+                          row_gather=r["row_token"])
+    h_ref = O.swiglu_bf16_ref(host(GU)[sample], F)
+    diff = np.abs(O.bf16_to_f64(host(h)[sample]) - O.bf16_to_f64(h_ref))
+    ulps = diff / bf16_ulp(h_ref)
+    assert np.all(ulps <= 1.0), f"SwiGLU: {int((ulps > 1).sum())} values beyond one bf16 ulp (max {ulps.max():.1f})"
+
+    Od = q.moe_q4k_grouped(Wdn, E, H, F, h, r["expert_offsets"], rows, hint, q.ACT_NONE)
+    Yd, Sd = O.grouped_ref(inp["W_down"], host(h), offs_h, rows=sample)
+    ratio_dn = _assert_tol(host(Od)[sample], Yd, Sd, "down")
+
+    y = host(q.moe_combine(Od, r["inv_perm"], r["topk_w"], M, topk, H))
+    tok = np.arange(M) if M <= 64 else sample_rows(M, 64, seed=1)
+    Yc, Sc = O.combine_ref(host(Od), host(r["inv_perm"]), host(r["topk_w"]))
+    assert np.all(np.abs(y[tok] - Yc[tok]) <= 1e-6 * Sc[tok] + 1e-30)
+    return ratio_gu, ratio_dn
+
+
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_moe_decode_layer(M):
+    _moe_stagewise(synth.moe_decode(3, M), M)
+
+
+def test_moe_decode_small_experts_tc_path():
+    """The tensor-core grouped path on a small ragged problem (hint forces it)."""
+    inp = synth.moe_layer(13, 40, E=16, H=512, F=256)
+    _moe_stagewise(inp, 40, hint=40)
+
+
+def test_moe_prefill_layer():
+    _moe_stagewise(synth.moe_prefill(4), 4096)
+
+
+# -------------------------------------------------------------------- GEMM --
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (100, 512, 512), (256, 256, 1024),
+                                   (300, 768, 2048), (513, 1024, 5120)])
+def test_gemm_small(M, N, K):
+    W, X = synth.gemv_small(200 + M, N=N, K=K, M=M)
+    y = host(q.q4k_gemm(dev(W), dev(X), N, K))
+    Y, S = O.matmul_ref(W, X)
+    _assert_tol(y, Y, S, f"gemm M={M} N={N} K={K}")
+
+
+@pytest.fixture(scope="module")
+def prefill_inputs():
+    W, X = synth.dense_prefill(2)
+    return W, X, dev(W), dev(X)
+
+
+@pytest.mark.parametrize("M", [512, 4096])
+def test_gemm_dense_prefill_sampled(prefill_inputs, M):
+    W, X, Wd, Xd = prefill_inputs
+    N, K = W.shape[0], W.shape[1] * 256
+    y = q.q4k_gemm(Wd, Xd[:M], N, K)
+    rows = sample_rows(N, 192, seed=M)
+    toks = sample_rows(M, 48, seed=M + 1)
+    yh = host(y[torch.from_numpy(toks).cuda()])
+    Y, S = O.matmul_rows_ref(W, X[toks], rows)
+    _assert_tol(yh[:, rows], Y, S, f"prefill M={M}")
+    assert torch.equal(y, q.q4k_gemm(Wd, Xd[:M], N, K))  # deterministic

@@ -61,7 +61,9 @@ typedef enum {
   Q4K_ERR_LAUNCH = 6,         /* the CUDA launch itself failed                     */
   Q4K_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up                */
   Q4K_ERR_DEVICE_BOUNDS = 8,  /* a device-side index check failed                  */
-  Q4K_ERR_CUDA = 9            /* a CUDA runtime call returned an error             */
+  Q4K_ERR_CUDA = 9,           /* a CUDA runtime call returned an error             */
+  Q4K_ERR_DEVICE_RANGE = 10   /* a value does not fit the fp16 operands of the
+                                 tensor-core grouped path (|x| or |w| > 65504)     */
 } q4k_status;
 
 enum { Q4K_ACT_NONE = 0, Q4K_ACT_SWIGLU = 1 };
@@ -124,7 +126,11 @@ q4k_status moe_route_permute(const float* logits, int M, int E, int topk,
  *   rows       total rows = off[E] (host value; must match the device array).
  *   max_rows_hint  upper bound on any single expert's row count (for a
  *              top-k layer over M tokens: M). <= 32 selects the GEMV-style
- *              decode kernel; larger selects the tcgen05 grouped GEMM.
+ *              decode kernel (exact 4-bit weights, per-32 scales in fp32);
+ *              larger selects the tcgen05 grouped GEMM, whose operands are
+ *              fp16: weights RN_fp16 of the fp32 dequant, activations
+ *              converted from bf16 (|values| must stay below 65504, else
+ *              Q4K_ERR_DEVICE_RANGE is latched).
  *   act == Q4K_ACT_NONE:   out fp32 [rows][N].
  *   act == Q4K_ACT_SWIGLU: out bf16 [rows][N/2], h = SiLU(g) * u with
  *              g = columns 0..N/2-1 (gate rows of W) and u = N/2..N-1 (up rows).

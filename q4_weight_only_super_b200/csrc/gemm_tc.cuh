@@ -15,8 +15,14 @@
 //   warps 2-9   dequantise one weight row each per K step into the canonical
 //               K-major 128-byte-swizzled bf16 layout the MMA reads (2-deep
 //               ring); afterwards they drain TMEM (tcgen05.ld) to global.
-//   warps 10-13 (gathered-row variant only) load activation rows by index
-//               with cp.async into the same swizzled layout.
+//   warps 10-13 (grouped variant) load activation rows by index (gathered or
+//               contiguous), convert bf16 -> fp16 in registers and store them
+//               in the same swizzled layout.
+// The dense GEMM multiplies bf16 x bf16. The grouped (mixture-of-experts) GEMM
+// multiplies fp16 x fp16: its activations can be heavy-tailed (SwiGLU outputs),
+// where bf16-rounded weights (unit roundoff 2^-8) would not keep the
+// 2e-3 * sum|w*x| error bound; fp16 weights (2^-11) do. Values outside the fp16
+// range latch Q4K_ERR_DEVICE_RANGE.
 // Every wait is bounded; on expiry the kernel latches Q4K_ERR_DEVICE_TIMEOUT,
 // stops all roles, drains its own copies (bounded), frees TMEM and returns.
 #pragma once
@@ -144,16 +150,18 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M=128, N=256.
+// Instruction descriptor: fp32 accumulate, A and B both bf16 (format 1) or both
+// fp16 (format 0), both K-major, M=128, N=256.
 constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
                                 ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t kIdescF16 = (1u << 4) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t accumulate) {
+__device__ __forceinline__ void umma_f16kind(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kIdescBf16), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -176,15 +184,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` in a K-major 128-byte
 // swizzled tile (rows of 128 bytes, 8-row atoms of 1024 bytes).
@@ -216,9 +215,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&p);
 }
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  const __half2 p = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  return F16 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
+}
 
 // Dequantise weight row `r` for K step `ks` (super-block ks/4, chunk ks%4)
 // from its raw header (16 B) and 32 quant bytes into the swizzled B tile.
+template <bool F16>
 __device__ __forceinline__ void dequant_row_step(uint8_t* btile, int r, int chunk, uint4 hdr, uint4 qa,
                                                  uint4 qb) {
   const float d = half_bits_to_float(hdr.x), dmin = half_bits_to_float(hdr.x >> 16);
@@ -231,6 +239,7 @@ __device__ __forceinline__ void dequant_row_step(uint8_t* btile, int r, int chun
     const float dm = dmin * (float)m; // exact
     const float cA = -ds * __uint_as_float((uint32_t)(127 + 23 - 4 * h) << 23);
     const float cB = -ds * __uint_as_float((uint32_t)(127 + 15 - 4 * h) << 23);
+    if (F16 && fmaf(15.f, fabsf(ds), fabsf(dm)) > 65504.f) latch_status(Q4K_ERR_DEVICE_RANGE);
 #pragma unroll
     for (int c8 = 0; c8 < 4; ++c8) {  // 8 weights: l = 8*c8 .. 8*c8+7 of sub-block 2*chunk+h
       float w0[4], w1[4];
@@ -238,10 +247,10 @@ __device__ __forceinline__ void dequant_row_step(uint8_t* btile, int r, int chun
       dq4(qw[2 * c8 + 1], h, ds, dm, cA, cB, w1);
       // dq4 returns weights in byte order (b0, b1, b2, b3)
       uint4 o;
-      o.x = pack_bf16x2(w0[0], w0[1]);
-      o.y = pack_bf16x2(w0[2], w0[3]);
-      o.z = pack_bf16x2(w1[0], w1[1]);
-      o.w = pack_bf16x2(w1[2], w1[3]);
+      o.x = pack2<F16>(w0[0], w0[1]);
+      o.y = pack2<F16>(w0[2], w0[3]);
+      o.z = pack2<F16>(w1[0], w1[1]);
+      o.w = pack2<F16>(w1[2], w1[3]);
       *reinterpret_cast<uint4*>(btile + sw128_offset(r, 4 * h + c8)) = o;
     }
   }
@@ -249,8 +258,8 @@ __device__ __forceinline__ void dequant_row_step(uint8_t* btile, int r, int chun
 
 // ---- the kernel -----------------------------------------------------------------
 
-template <bool GROUPED, bool GATHER, bool SWIGLU>
-__global__ void __launch_bounds__(32 * (2 + kDqWarps + (GATHER ? kGatherWarps : 0)), 1)
+template <bool GROUPED, bool SWIGLU>
+__global__ void __launch_bounds__(32 * (2 + kDqWarps + (GROUPED ? kGatherWarps : 0)), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -275,7 +284,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   const int task = (int)(blockIdx.x / (unsigned)p.n_tiles);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesAW; ++s) {
-      mbar_init(bar_full_aw(s), GATHER ? 1 + kGatherWarps : 1);
+      mbar_init(bar_full_aw(s), GROUPED ? 1 + kGatherWarps : 1);
       mbar_init(bar_empty_aw(s), 1 + kDqWarps);
     }
     for (int s = 0; s < kStagesB; ++s) {
@@ -358,10 +367,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         for (int ks = 0; ks < nks; ++ks) {
           const int s = ks % kStagesAW, u = ks / kStagesAW;
           if (u >= 1 && !mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag)) break;
-          const uint32_t bytes = (GATHER ? 0u : kATileBytes) + kWRawBytes;
+          const uint32_t bytes = (GROUPED ? 0u : kATileBytes) + kWRawBytes;
           mbar_arrive_expect_tx(bar_full_aw(s), bytes);
           const uint32_t a_dst = sbase + kSmemA + s * kATileBytes;
-          if (!GATHER) {
+          if (!GROUPED) {
             tma_load_2d(a_dst, &tmap_x, ks * kGemmBK, ay, bar_full_aw(s));
             tma_load_2d(a_dst + kATileBytes / 2, &tmap_x, ks * kGemmBK, ay + 128, bar_full_aw(s));
           }
@@ -403,8 +412,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
           for (int h = 0; h < 2; ++h) {
 #pragma unroll
             for (int kk = 0; kk < kGemmBK / 16; ++kk) {
-              umma_bf16(tmem + h * 256, umma_desc_sw128(a0 + h * (kATileBytes / 2) + kk * 32),
-                        umma_desc_sw128(b0 + kk * 32), (ks | kk) != 0);
+              umma_f16kind(tmem + h * 256, umma_desc_sw128(a0 + h * (kATileBytes / 2) + kk * 32),
+                           umma_desc_sw128(b0 + kk * 32), GROUPED ? kIdescF16 : kIdescBf16,
+                           (ks | kk) != 0);
             }
           }
           umma_commit(bar_empty_aw(s));
@@ -433,7 +443,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         const uint4 qb = *reinterpret_cast<const uint4*>(wr + 2 * kWRawPart + r * 16);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty_aw(s));
-        dequant_row_step(smem + kSmemB + sb * kBTileBytes, r, ks & 3, hdr, qa, qb);
+        dequant_row_step<GROUPED>(smem + kSmemB + sb * kBTileBytes, r, ks & 3, hdr, qa, qb);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_full_b(sb));
@@ -487,51 +497,54 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
           }
         }
       }
-    } else if (GATHER) {
-      // ---------------- gathered activation rows (cp.async) ----------------
+    } else if (GROUPED) {
+      // ---------------- activation rows: load, bf16 -> fp16, store swizzled ----------------
       const int gt = (warp - 2 - kDqWarps) * 32 + lane;  // 0..127
       const int ch = gt & 7;                              // 16-byte chunk within the 128-byte row
       const int r0 = gt >> 3;                             // rows r0, r0+16, ...
-      int64_t src_row[kGemmBM / 16];
+      const uint16_t* src_row[kGemmBM / 16];
 #pragma unroll
       for (int j = 0; j < kGemmBM / 16; ++j) {
-        const int ml = r0 + 16 * j;
-        const int mrow = m0 + ml;
-        src_row[j] = -1;
-        if (mrow < count) src_row[j] = p.gather ? p.gather[row_base + mrow] : (row_base + mrow);
+        const int mrow = m0 + r0 + 16 * j;
+        src_row[j] = nullptr;
+        if (mrow < count) {
+          const int64_t sr = p.gather ? p.gather[row_base + mrow] : (row_base + mrow);
+          src_row[j] = p.X + sr * p.K + ch * 8;
+        }
       }
-      int issued = 0;
-      bool ok = true;
+      uint4 buf[kGemmBM / 16];
+      auto load = [&](int ks) {
+#pragma unroll
+        for (int j = 0; j < kGemmBM / 16; ++j)
+          buf[j] = src_row[j] ? ldg_u4(src_row[j] + ks * kGemmBK) : make_uint4(0u, 0u, 0u, 0u);
+      };
+      uint32_t amax = 0;  // largest |bf16| bit pattern seen, per 16-bit half
+      if (nks > 0) load(0);
       for (int ks = 0; ks < nks; ++ks) {
         const int s = ks % kStagesAW, u = ks / kStagesAW;
         if (u >= 1 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag))) {
-          ok = false;
+            !__all_sync(0xffffffffu, mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag)))
           break;
-        }
-        const uint32_t a_dst = sbase + kSmemA + s * kATileBytes;
+        uint8_t* a_dst = smem + kSmemA + s * kATileBytes;
 #pragma unroll
         for (int j = 0; j < kGemmBM / 16; ++j) {
-          const int ml = r0 + 16 * j;
-          const int64_t sr = src_row[j];
-          const uint16_t* src = p.X + (sr < 0 ? 0 : sr) * p.K + ks * kGemmBK + ch * 8;
-          cp_async_16(a_dst + sw128_offset(ml, ch), src, sr < 0 ? 0u : 16u);
+          const uint32_t w[4] = {buf[j].x, buf[j].y, buf[j].z, buf[j].w};
+          uint4 o;
+          uint32_t* op = &o.x;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            amax = __vmaxu2(amax, w[e] & 0x7FFF7FFFu);
+            op[e] = pack_f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+          }
+          *reinterpret_cast<uint4*>(a_dst + sw128_offset(r0 + 16 * j, ch)) = o;
         }
-        cp_async_commit();
-        ++issued;
-        if (ks >= 1) {
-          cp_async_wait<1>();
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_full_aw((ks - 1) % kStagesAW));
-        }
-      }
-      cp_async_wait<0>();
-      if (ok && issued > 0) {
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_full_aw((issued - 1) % kStagesAW));
+        if (lane == 0) mbar_arrive(bar_full_aw(s));
+        if (ks + 1 < nks) load(ks + 1);  // next stage's rows in flight during the next wait
       }
+      // |x| >= 65536 (bf16 0x4780) does not fit fp16
+      if ((amax & 0xFFFFu) >= 0x4780u || (amax >> 16) >= 0x4780u) latch_status(Q4K_ERR_DEVICE_RANGE);
     }
   }
 
@@ -586,10 +599,10 @@ inline bool make_tmap_w(CUtensorMap* m, const void* base, int64_t rows, int64_t 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GROUPED, bool GATHER, bool SWIGLU>
+template <bool GROUPED, bool SWIGLU>
 inline q4k_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
                                 cudaStream_t s) {
-  auto* k = gemm_tc_kernel<GROUPED, GATHER, SWIGLU>;
+  auto* k = gemm_tc_kernel<GROUPED, SWIGLU>;
   static std::atomic<int> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -601,7 +614,7 @@ inline q4k_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, co
     attr_set[dev].store(1);
   }
   const dim3 grid((unsigned)(p.n_tiles * p.m_tiles));
-  const dim3 block(32 * (2 + kDqWarps + (GATHER ? kGatherWarps : 0)));
+  const dim3 block(32 * (2 + kDqWarps + (GROUPED ? kGatherWarps : 0)));
   k<<<grid, block, kGemmSmemLaunch, s>>>(tx, tw, p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? Q4K_OK : Q4K_ERR_LAUNCH;
@@ -614,30 +627,23 @@ inline q4k_status launch_gemm_tc(GemmParams p, cudaStream_t s) {
     return Q4K_ERR_CUDA;
   p.n_tiles = p.N / kGemmBN;
   p.m_tiles = (p.M + kGemmBM - 1) / kGemmBM;
-  return launch_gemm_t<false, false, false>(tx, tw, p, s);
+  return launch_gemm_t<false, false>(tx, tw, p, s);
 }
 
 // Grouped: tasks are (expert, 256-row tile of that expert's rows); their number
 // is at most ceil(rows/256) + min(E, rows). CTAs past the real count exit.
+// Activation rows are fetched by the loader warps (by index when `gather` is
+// set), so the activation tensor map is unused.
 inline q4k_status launch_gemm_tc_grouped(GemmParams p, cudaStream_t s) {
   CUtensorMap tx, tw;
   const int64_t row_bytes = (int64_t)(p.K / QK) * BLOCK_BYTES;
-  const bool gather = p.gather != nullptr;
-  // Without a gather the A rows are the sorted rows themselves (TMA); with one they
-  // are fetched by index and the activation tensor map is unused.
-  if (!make_tmap_x(&tx, p.X, gather ? 1 : p.rows, p.K) ||
-      !make_tmap_w(&tw, p.W, (int64_t)p.E * p.N, row_bytes))
+  if (!make_tmap_x(&tx, p.X, 1, p.K) || !make_tmap_w(&tw, p.W, (int64_t)p.E * p.N, row_bytes))
     return Q4K_ERR_CUDA;
   const bool swiglu = p.act == Q4K_ACT_SWIGLU;
   if (swiglu && (p.N / 2) % (kGemmBN / 2)) return Q4K_ERR_UNSUPPORTED;
   p.n_tiles = swiglu ? (p.N / 2) / (kGemmBN / 2) : p.N / kGemmBN;
   p.m_tiles = (p.rows + kGemmBM - 1) / kGemmBM + std::min(p.E, p.rows);
-  if (gather) {
-    return swiglu ? launch_gemm_t<true, true, true>(tx, tw, p, s)
-                  : launch_gemm_t<true, true, false>(tx, tw, p, s);
-  }
-  return swiglu ? launch_gemm_t<true, false, true>(tx, tw, p, s)
-                : launch_gemm_t<true, false, false>(tx, tw, p, s);
+  return swiglu ? launch_gemm_t<true, true>(tx, tw, p, s) : launch_gemm_t<true, false>(tx, tw, p, s);
 }
 
 }  // namespace q4k

@@ -48,37 +48,45 @@ q4k_status launch_status(cudaError_t e) {
 // ---------------------------------------------------------------- GEMV ----
 
 struct GemvCfg {
-  int mt, warps, ksplit, kc;
+  int mt, warps, ksplit, kc, stages;
 };
 
-// Launch shape for `tokens` (<= 32) tokens against `rows_out` output rows per
+constexpr int kSms = 148;
+
+// Launch shape for `tokens` (<= 32) tokens against `rows_out` weight rows per
 // matrix and `nkb` super-blocks per row, with `groups` matrices (experts)
-// processed side by side. Depends only on (tokens class, rows, nkb, groups).
+// processed side by side. Depends only on (token class, rows, nkb, groups), so
+// the summation order of a token's result never depends on the batch. The K
+// split (cluster size) is the largest that keeps every CTA resident at once.
 GemvCfg pick_gemv(int tokens, int rows_out, int nkb, int groups) {
   GemvCfg c;
   c.mt = tokens <= 8 ? 1 : (tokens <= 16 ? 2 : 4);
-  c.warps = c.mt == 4 ? 8 : 4;
-  c.kc = c.mt == 1 ? 8 : (c.mt == 2 ? 4 : 2);
-  const int tile_rows = 16 * c.warps;
-  const int tiles = (rows_out + tile_rows - 1) / tile_rows;
-  const long target = 4L * 148;
-  long ks = (target + (long)tiles * groups - 1) / ((long)tiles * groups);
+  c.warps = 4;
+  // two CTAs per SM: ring 4 x 20 KB (3 x 20 KB at 32 tokens) + activations <= 32 KB
+  c.kc = c.mt == 1 ? 4 : (c.mt == 2 ? 2 : 1);
+  c.stages = c.mt == 4 ? 3 : 4;
+  const int per_sm = 2;  // shared-memory residency of one CTA
+  const long tiles = (rows_out + 32 * c.warps - 1) / (32 * c.warps);
+  const long slots = (long)kSms * per_sm;
+  long ks = slots / std::max(1L, tiles * groups);
   ks = std::max(1L, std::min<long>(ks, 8));
   ks = std::min<long>(ks, nkb);
   c.ksplit = (int)ks;
-  c.kc = std::min(c.kc, (nkb + c.ksplit - 1) / c.ksplit);
+  const int span = (nkb + c.ksplit - 1) / c.ksplit;
+  while (c.kc > 1 && c.kc / 2 >= span) c.kc /= 2;  // power of two, no larger than needed
   return c;
 }
 
 template <int MT, int WARPS, bool GROUPED, bool SWIGLU>
-q4k_status launch_gemv_t(const GemvParams& p, int tiles, int groups, cudaStream_t s) {
+q4k_status launch_gemv_t(const CUtensorMap& tmap, const GemvParams& p, int tiles, int groups,
+                         cudaStream_t s) {
   auto* k = gemv_kernel<MT, WARPS, GROUPED, SWIGLU>;
   static std::atomic<size_t> smem_set[kMaxDevices];  // one per instantiation
-  const size_t smem = gemv_smem_bytes<MT, WARPS>(p.kc);
+  const size_t smem = GemvSmem<MT, WARPS>::total(p.stages, p.kc);
   if (ensure_smem(k, smem, smem_set) != cudaSuccess) return Q4K_ERR_LAUNCH;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * p.ksplit), (unsigned)groups, 1);
-  cfg.blockDim = dim3(32 * WARPS, 1, 1);
+  cfg.blockDim = dim3(32 * (WARPS + 1), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -88,17 +96,22 @@ q4k_status launch_gemv_t(const GemvParams& p, int tiles, int groups, cudaStream_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return launch_status(cudaLaunchKernelEx(&cfg, k, p));
+  return launch_status(cudaLaunchKernelEx(&cfg, k, tmap, p));
 }
 
 template <bool GROUPED, bool SWIGLU>
 q4k_status launch_gemv(const GemvCfg& c, GemvParams p, int rows_out, int groups, cudaStream_t s) {
   p.ksplit = c.ksplit;
   p.kc = c.kc;
-  const int tiles = (rows_out + 16 * c.warps - 1) / (16 * c.warps);
-  if (c.mt == 1) return launch_gemv_t<1, 4, GROUPED, SWIGLU>(p, tiles, groups, s);
-  if (c.mt == 2) return launch_gemv_t<2, 4, GROUPED, SWIGLU>(p, tiles, groups, s);
-  return launch_gemv_t<4, 8, GROUPED, SWIGLU>(p, tiles, groups, s);
+  p.stages = c.stages;
+  CUtensorMap tmap;
+  const int64_t row_bytes = (int64_t)p.nkb * BLOCK_BYTES;
+  const int64_t total_rows = GROUPED ? (int64_t)p.E * p.N : p.N;
+  if (!make_tmap_w_rowgroup(&tmap, p.W, total_rows, row_bytes)) return Q4K_ERR_CUDA;
+  const int tiles = (rows_out + 32 * c.warps - 1) / (32 * c.warps);
+  if (c.mt == 1) return launch_gemv_t<1, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
+  if (c.mt == 2) return launch_gemv_t<2, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
+  return launch_gemv_t<4, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
 }
 
 }  // namespace
@@ -117,6 +130,7 @@ const char* q4k_status_string(int s) {
     case Q4K_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case Q4K_ERR_DEVICE_BOUNDS: return "device-side index out of range";
     case Q4K_ERR_CUDA: return "CUDA runtime error";
+    case Q4K_ERR_DEVICE_RANGE: return "value outside the fp16 range of the tensor-core grouped path";
     default: return "unknown status";
   }
 }

@@ -153,6 +153,10 @@ def build_workloads(torch, q, synth):
     W["moe_pre"] = {k: dev(mp[k]) for k in ("logits", "X", "W_gate_up", "W_down")}
     W["moe_dims"] = (md["E"], md["H"], md["F"])
     W["moe_pre_hot"] = [int(x) for x in mp["hot_ids"]]
+    # scratch for the GEMV activation pre-pass, allocated once (largest use: 32 tokens x 17408)
+    need = max(q.q4k_workspace_bytes(q.OP_GEMV, 32, 0, 17408),
+               q.q4k_workspace_bytes(q.OP_GROUPED, 32 * 8, 0, 2048))
+    W["ws"] = torch.empty(need, dtype=torch.uint8, device="cuda")
     return W
 
 
@@ -161,10 +165,12 @@ def moe_layer_gpu(q, tm, key, d, M, dims, topk=8):
     rows = M * topk
     logits, X = d["logits"][:M], d["X"][:M]
     r = tm.run(key + ":route", lambda: q.moe_route_permute(logits, topk))
+    ws = d.get("ws") if M <= 32 else None
     h = tm.run(key + ":gate_up", lambda: q.moe_q4k_grouped(d["W_gate_up"], E, 2 * F, H, X, r["expert_offsets"],
-                                                            rows, M, q.ACT_SWIGLU, row_gather=r["row_token"]))
+                                                            rows, M, q.ACT_SWIGLU, row_gather=r["row_token"],
+                                                            ws=ws))
     o = tm.run(key + ":down", lambda: q.moe_q4k_grouped(d["W_down"], E, H, F, h, r["expert_offsets"], rows, M,
-                                                         q.ACT_NONE))
+                                                         q.ACT_NONE, ws=ws))
     return tm.run(key + ":combine", lambda: q.moe_combine(o, r["inv_perm"], r["topk_w"], M, topk, H)), r
 
 
@@ -174,12 +180,13 @@ def run_step(q, tm, W):
         for p in ("gate_up", "down"):
             N, K = W["dec_shapes"][p]
             Wt, Xt = W["dec"][f"W_{p}"], W["dec"][f"X_{p}"][:M]
-            tm.run(f"gemv:{p}:M{M}", lambda: q.q4k_gemv(Wt, Xt, N, K))
+            tm.run(f"gemv:{p}:M{M}", lambda: q.q4k_gemv(Wt, Xt, N, K, ws=W["ws"]))
             launches += 1
     Wt, Xt, N, K = W["pre"]
     for M in (512, 4096):
         tm.run(f"gemm:M{M}", lambda: q.q4k_gemm(Wt, Xt[:M], N, K))
         launches += 1
+    W["moe_dec"]["ws"] = W["ws"]
     for M in (1, 8, 32):
         moe_layer_gpu(q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"])
         launches += 5
@@ -211,7 +218,7 @@ def e2e_gemv(torch, q, W, steps, warmup):
                 s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 s.record()
                 xd.copy_(xh, non_blocking=True)
-                q.q4k_gemv(W["dec"][f"W_{p}"], xd, N, K, Y=yd)
+                q.q4k_gemv(W["dec"][f"W_{p}"], xd, N, K, Y=yd, ws=W["ws"])
                 yh.copy_(yd, non_blocking=True)
                 e.record()
                 e.synchronize()
@@ -329,7 +336,8 @@ def only(args):
         dd = synth.dense_decode(1)
         Wt, Xt = dev(dd[f"W_{args.proj}"]), dev(dd[f"X_{args.proj}"][:M])
         N, K = dd[f"W_{args.proj}"].shape[0], dd[f"W_{args.proj}"].shape[1] * 256
-        fn = lambda: q.q4k_gemv(Wt, Xt, N, K)
+        ws = torch.empty(q.q4k_workspace_bytes(q.OP_GEMV, M, N, K), dtype=torch.uint8, device="cuda")
+        fn = lambda: q.q4k_gemv(Wt, Xt, N, K, ws=ws)
         units = N * (K // 256) * BLOCK / 1e9
         unit = "GB/s"
     elif args.only == "gemm":

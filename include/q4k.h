@@ -67,7 +67,7 @@ typedef enum {
 } q4k_status;
 
 enum { Q4K_ACT_NONE = 0, Q4K_ACT_SWIGLU = 1 };
-enum { Q4K_OP_GEMM = 1, Q4K_OP_ROUTE = 2, Q4K_OP_GROUPED = 3 };
+enum { Q4K_OP_GEMM = 1, Q4K_OP_ROUTE = 2, Q4K_OP_GROUPED = 3, Q4K_OP_GEMV = 4 };
 
 /* Dequantise `nblocks` consecutive Q4_K blocks (hipEngine 0.3.0 README,
  * "GGUF Support": the Q4_K quant reader).
@@ -82,10 +82,17 @@ q4k_status q4k_dequant(const void* W, int64_t nblocks, int out_bf16, void* out, 
  * the GEMV-decode half of the WMMA-prefill/GEMV-decode session profile).
  *   Y[m][n] = sum_k w[n][k] * X[m][k],  W [N][K/256] blocks, X bf16 [M][K],
  *   Y fp32 [M][N].  N % 16 == 0.  M == 0 or N == 0 is a no-op.
+ *   ws/ws_bytes: device scratch of q4k_workspace_bytes(Q4K_OP_GEMV, M, N, K,
+ *   0, 0) bytes; a pre-pass writes each token's activations there, per
+ *   256-wide block scaled by a power of two and rounded to fp16 (an
+ *   activation is represented to 11 significant bits relative to the largest
+ *   magnitude of its 256-block). The 4-bit weights and their six-bit scales
+ *   enter exactly; products accumulate in fp32. Calls sharing `ws` must be
+ *   ordered on one stream.
  * Row m of the result does not depend on the other rows of X (bit-identical
  * to the M == 1 call on that row). */
 q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
-                    void* stream);
+                    void* ws, size_t ws_bytes, void* stream);
 
 /* Prefill GEMM on tcgen05 tensor cores with the Q4_K weights dequantised
  * tile by tile into shared memory (hipEngine 0.3.0 README, "GGUF Support":
@@ -126,7 +133,7 @@ q4k_status moe_route_permute(const float* logits, int M, int E, int topk,
  *   rows       total rows = off[E] (host value; must match the device array).
  *   max_rows_hint  upper bound on any single expert's row count (for a
  *              top-k layer over M tokens: M). <= 32 selects the GEMV-style
- *              decode kernel (exact 4-bit weights, per-32 scales in fp32);
+ *              decode kernel (same arithmetic as q4k_gemv);
  *              larger selects the tcgen05 grouped GEMM, whose operands are
  *              fp16: weights RN_fp16 of the fp32 dequant, activations
  *              converted from bf16 (|values| must stay below 65504, else
@@ -134,7 +141,9 @@ q4k_status moe_route_permute(const float* logits, int M, int E, int topk,
  *   act == Q4K_ACT_NONE:   out fp32 [rows][N].
  *   act == Q4K_ACT_SWIGLU: out bf16 [rows][N/2], h = SiLU(g) * u with
  *              g = columns 0..N/2-1 (gate rows of W) and u = N/2..N-1 (up rows).
- *   ws: unused by the current kernels (pass NULL, 0).
+ *   ws/ws_bytes: device scratch of q4k_workspace_bytes(Q4K_OP_GROUPED, rows,
+ *              N, K, E, 0) bytes (used by the decode kernel; may be NULL when
+ *              max_rows_hint > 32).
  * N % 32 == 0 (SWIGLU: N/2 % 16 == 0), rows == 0 is a no-op. */
 q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uint16_t* A,
                            const int32_t* row_gather, const int32_t* expert_offsets,
@@ -151,7 +160,10 @@ q4k_status moe_combine(const float* O, const int32_t* inv_perm, const float* top
                        int M, int topk, int H, float* Y, void* stream);
 
 /* Bytes of device workspace an entry point needs for these sizes
- * (Q4K_OP_ROUTE: moe_route_permute; others return 0). */
+ * (Q4K_OP_ROUTE: moe_route_permute with M tokens and E experts;
+ *  Q4K_OP_GEMV: q4k_gemv with M tokens and K inputs;
+ *  Q4K_OP_GROUPED: moe_q4k_grouped with M = rows and K inputs;
+ *  Q4K_OP_GEMM: 0). */
 size_t q4k_workspace_bytes(int op, int M, int N, int K, int E, int topk);
 
 /* Synchronises `stream`, returns the device status word (Q4K_OK if no

@@ -16,11 +16,11 @@ import torch
 __all__ = [
     "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemm", "moe_route_permute",
     "moe_q4k_grouped", "moe_combine", "q4k_workspace_bytes", "q4k_last_device_status",
-    "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "EXPORTS",
+    "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "OP_GEMV", "EXPORTS",
 ]
 
 ACT_NONE, ACT_SWIGLU = 0, 1
-OP_GEMM, OP_ROUTE, OP_GROUPED = 1, 2, 3
+OP_GEMM, OP_ROUTE, OP_GROUPED, OP_GEMV = 1, 2, 3, 4
 BLOCK_BYTES = 144
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libq4k.so")
 
@@ -28,7 +28,7 @@ _p, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size
 # name -> (restype, argtypes); mirrors include/q4k.h
 EXPORTS = {
     "q4k_dequant": (_i, [_p, _i64, _i, _p, _p]),
-    "q4k_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p]),
+    "q4k_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "q4k_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "moe_route_permute": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_q4k_grouped": (_i, [_p, _i, _i, _i, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
@@ -99,12 +99,20 @@ def q4k_dequant(W, out_bf16: bool = False, out=None, stream=None):
     return out
 
 
-def q4k_gemv(W, X, N: int, K: int, Y=None, stream=None):
+def _scratch(nbytes: int, device, ws=None):
+    if ws is not None:
+        return ws
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def q4k_gemv(W, X, N: int, K: int, Y=None, ws=None, stream=None):
     """Y[M][N] = X[M][K] @ W^T for 1 <= M <= 32 (W: Q4_K [N][K/256][144])."""
     M = X.shape[0]
     if Y is None:
         Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
-    _check("q4k_gemv", lib().q4k_gemv(_ptr(W), _ptr(_bits16(X)), _ptr(Y), M, N, K, _stream(stream)))
+    ws = _scratch(q4k_workspace_bytes(OP_GEMV, M, N, K), X.device, ws)
+    _check("q4k_gemv", lib().q4k_gemv(_ptr(W), _ptr(_bits16(X)), _ptr(Y), M, N, K, _ptr(ws), ws.numel(),
+                                      _stream(stream)))
     return Y
 
 
@@ -148,16 +156,19 @@ def moe_route_permute(logits, topk: int, out=None, ws=None, stream=None):
 
 
 def moe_q4k_grouped(W_experts, E: int, N: int, K: int, A, expert_offsets, rows: int,
-                    max_rows_hint: int, act: int = ACT_NONE, row_gather=None, out=None, stream=None):
+                    max_rows_hint: int, act: int = ACT_NONE, row_gather=None, out=None, ws=None,
+                    stream=None):
     """Grouped expert matmul over rows sorted by expert (see include/q4k.h)."""
     if out is None:
         if act == ACT_SWIGLU:
             out = torch.empty(rows, N // 2, dtype=torch.bfloat16, device=A.device)
         else:
             out = torch.empty(rows, N, dtype=torch.float32, device=A.device)
+    if ws is None and 0 < max_rows_hint <= 32:  # only the decode kernel uses scratch
+        ws = _scratch(q4k_workspace_bytes(OP_GROUPED, rows, N, K, E), A.device)
     st = lib().moe_q4k_grouped(_ptr(W_experts), E, N, K, _ptr(_bits16(A)), _ptr(row_gather),
-                               _ptr(expert_offsets), rows, max_rows_hint, act, _ptr(out), None, 0,
-                               _stream(stream))
+                               _ptr(expert_offsets), rows, max_rows_hint, act, _ptr(out), _ptr(ws),
+                               0 if ws is None else ws.numel(), _stream(stream))
     _check("moe_q4k_grouped", st)
     return out
 

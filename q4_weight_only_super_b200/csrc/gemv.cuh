@@ -5,26 +5,39 @@
 // table: "GEMV ... GB/s"). The weight stream from HBM is the roofline.
 //
 // Design (sm_100a):
-//  * A producer warp streams the CTA's weight rows, one super-block column
-//    (16 rows x 144 bytes per row group) per stage, into an S-deep shared
-//    memory ring with TMA (cp.async.bulk.tensor) and mbarrier completion, so
-//    many kilobytes per SM are in flight regardless of the compute loop.
-//  * Consumer warps own 16 weight rows each. Weights are the 16-row A operand
-//    of mma.sync m16n8k16 (bf16 in, fp32 accumulate); tokens are the 8-wide B
-//    operand (MT fragments of 8 tokens).
-//  * A nibble q ORed into the bf16 pattern 0x4300 is exactly 128+q, so two
-//    weights become one bf16x2 register with a single mask/or. The bias is
-//    removed per sub-block: with C = sum (128+q)*x and Sx = sum x,
-//      sum_i w_i x_i = (d*sc) * C - (128*d*sc + dmin*m) * Sx,
-//    applied with packed fp32x2 FMAs (one per pair of tokens).
+//  * A pre-pass (gemv_prep_kernel) turns each activation row, one 256-wide
+//    super-block column at a time, into a 576-byte record: the 256 values
+//    scaled by a power of two 2^k (chosen so the column's largest magnitude
+//    lands in [2^14, 2^15): exact, and fp16 can neither overflow nor lose the
+//    small values), rounded to fp16, stored in the order the MMA fragments
+//    read them; the eight 32-wide sub-block sums of the scaled values (times
+//    2^-6) as fp16 hi + lo pairs; and 2^-k. It runs once per call, so every
+//    CTA only copies prepared records.
+//  * In the GEMV a producer warp streams the CTA's weight rows (one
+//    super-block column per stage) into a shared-memory ring with TMA, a
+//    second producer warp copies the matching activation records with 1-D
+//    bulk copies; mbarriers track both. The GEMV is launched as a programmatic
+//    dependent of the pre-pass, so its weight stream starts while the pre-pass
+//    runs and only the activation copies wait for it.
+//  * Consumer warps own 32 weight rows each (two 16-row tiles, so every
+//    activation fragment feeds two MMAs). The A operand is fp16 q*sc, exact
+//    (q*sc <= 945): a nibble ORed into 0x6400 is 1024+q (low nibble) or
+//    1024+16q (high nibble), and one fp16x2 FMA with (sc or sc/16) and
+//    -1024*that removes the bias exactly. So the mma.sync m16n8k16 accumulator
+//    (fp32) runs over the whole super-block: C = sum_k sc*q*x'.
+//  * The min term, dmin * sum_j m_j * X_j over the eight sub-blocks, is one
+//    more MMA per tile: A = m_j (fp16, exact), B = the sub-block sums
+//    (hi + lo, two MMAs), k = sub-block index.
+//  * Per super-block the result is y += d*2^-k*C - 64*dmin*2^-k*Cm.
 //  * The k order inside a sub-block is free for a dot product, so each
-//    thread takes the nibbles in the order the mask produces them, and the
-//    activations staged in shared memory are stored in that same order.
-//  * A CTA owns 16*WARPS weight rows and a contiguous range of super-blocks;
+//    thread takes the nibbles in the order the masks produce them, and the
+//    pre-pass stores the activations in that same order.
+//  * A CTA owns 32*WARPS weight rows and a contiguous range of super-blocks;
 //    a thread-block cluster of KSPLIT CTAs covers the whole K range and its
 //    partial sums are reduced in rank order through distributed shared memory
-//    (deterministic, no atomics). The decomposition depends only on (N, K), so
-//    a token's result never depends on the other tokens in the batch.
+//    (deterministic, no atomics). The decomposition depends only on (N, K), and
+//    the pre-pass record of a row depends only on that row, so a token's
+//    result never depends on the other tokens in the batch.
 #pragma once
 #include <cooperative_groups.h>
 
@@ -35,58 +48,115 @@ namespace q4k {
 
 namespace cg = cooperative_groups;
 
-constexpr uint32_t kBf16Bias2 = 0x43004300u;  // bf16x2 (128.0, 128.0)
+// Prepared activation record of one (row, super-block): bytes [0,512) fp16 values
+// in fragment order [sub-block 8][quarter 4][8], [512,528) fp16 sub-block sums
+// (hi), [528,544) (lo), [544,548) fp32 2^-k, rest padding. 576 = 64 mod 128
+// keeps the per-thread 16-byte fragment reads bank-conflict-free.
+constexpr int kXRec = 576;
+constexpr int kXPadRows = 32;  // zero records appended after the real rows
 
-__device__ __forceinline__ uint32_t nib2(uint32_t word, int shift) {
-  return ((word >> shift) & 0x000F000Fu) | kBf16Bias2;
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1, bool zero_c) {
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1, bool zero_c) {
   if (zero_c) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%10,%10,%10,%10};"
         : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
   } else {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   }
 }
 
-// acc = fma(s, c, acc) on a pair of fp32 values with one packed instruction.
-__device__ __forceinline__ void fma2(float& acc0, float& acc1, float s, float c0, float c1) {
-  uint64_t a = (uint64_t)__float_as_uint(acc0) | ((uint64_t)__float_as_uint(acc1) << 32);
-  const uint64_t sv = (uint64_t)__float_as_uint(s) | ((uint64_t)__float_as_uint(s) << 32);
-  const uint64_t cv = (uint64_t)__float_as_uint(c0) | ((uint64_t)__float_as_uint(c1) << 32);
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(sv), "l"(cv));
-  acc0 = __uint_as_float((uint32_t)a);
-  acc1 = __uint_as_float((uint32_t)(a >> 32));
+__device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
+
+// fp16x2 (1024 + b_lo, 1024 + b_hi) from bytes `lo` and `hi` (0..3) of `word`
+// (each <= 63, so it fits the 10-bit mantissa of 1024).
+__device__ __forceinline__ uint32_t bytes_1024(uint32_t word, uint32_t lo, uint32_t hi) {
+  return __byte_perm(word, 0x64u, (4u << 12) | (hi << 8) | (4u << 4) | lo);
 }
 
-__device__ __forceinline__ void consumer_sync(int nthreads) {
-  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+// ------------------------------------------------------------------ pre-pass ---
+
+// One warp per (row, super-block) record; rows >= `rows` (padding) become zeros.
+__global__ void __launch_bounds__(256) gemv_prep_kernel(const uint16_t* __restrict__ X,
+                                                        const int32_t* __restrict__ gather, int rows,
+                                                        int rows_pad, int K, int nkb,
+                                                        uint8_t* __restrict__ ws) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= (int64_t)rows_pad * nkb) return;  // uniform per warp
+  const int kb = (int)(w / rows_pad), r = (int)(w % rows_pad);
+  uint8_t* rec = ws + w * kXRec;  // record index kb * rows_pad + r
+  const int sb = lane >> 2, tq = lane & 3;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (r < rows) {
+    const int64_t src = gather ? gather[r] : r;
+    v = ldg_u4(X + src * K + (int64_t)kb * QK + sb * 32 + tq * 8);
+  }
+  const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+  float x[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    x[2 * e] = bf16_bits_to_float(wv[e] & 0xFFFFu);
+    x[2 * e + 1] = bf16_bits_to_float(wv[e] >> 16);
+  }
+  uint32_t amax = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) amax = max(amax, __float_as_uint(x[e]) & 0x7FFFFFFFu);
+  amax = __reduce_max_sync(0xffffffffu, amax);  // bit order = magnitude order for |x|
+  int k = 0;
+  if (amax != 0) {
+    const int E = max(1, (int)(amax >> 23));  // biased exponent of the largest |x|
+    k = min(126, max(-126, 141 - E));          // largest |x| * 2^k in [2^14, 2^15)
+  }
+  const float f = __uint_as_float((uint32_t)(127 + k) << 23);  // 2^k
+  float xs[8];
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    xs[e] = x[e] * f;  // exact
+    sum += xs[e];
+  }
+  uint4 o;  // fragment order (e0,e2),(e1,e3),(e4,e6),(e5,e7)
+  o.x = h2_bits(__floats2half2_rn(xs[0], xs[2]));
+  o.y = h2_bits(__floats2half2_rn(xs[1], xs[3]));
+  o.z = h2_bits(__floats2half2_rn(xs[4], xs[6]));
+  o.w = h2_bits(__floats2half2_rn(xs[5], xs[7]));
+  *reinterpret_cast<uint4*>(rec + (sb * 4 + tq) * 16) = o;
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  const float s2 = sum * 0.015625f;  // 2^-6: |s2| < 2^14
+  const __half hi = __float2half_rn(s2);
+  const __half lo = __float2half_rn(s2 - __half2float(hi));
+  if (tq == 0) {
+    reinterpret_cast<__half*>(rec + 512)[sb] = hi;
+    reinterpret_cast<__half*>(rec + 528)[sb] = lo;
+  }
+  if (lane == 0) *reinterpret_cast<float*>(rec + 544) = __uint_as_float((uint32_t)(127 - k) << 23);
 }
+
+// ---------------------------------------------------------------------- GEMV ---
 
 struct GemvParams {
   const uint8_t* W;          // dense: [N][nkb][144]; grouped: [E][N][nkb][144]
-  const uint16_t* X;         // bf16 activations
+  const uint8_t* xprep;      // prepared records [nkb][rows_pad][576]
   void* out;                 // fp32 [rows][N] or bf16 [rows][N/2] (SWIGLU)
   const int32_t* offsets;    // grouped: [E+1] rows per expert (device); dense: nullptr
-  const int32_t* gather;     // grouped: optional sorted row -> X row
   int M;                     // dense: tokens; grouped: unused
   int N;                     // weight rows per matrix
-  int K;
   int nkb;                   // K / 256
   int E;                     // grouped: experts
-  int64_t expert_stride;     // bytes per expert matrix
+  int rows_pad;              // records per super-block column
   int ksplit;                // cluster size along K
-  int kc;                    // super-blocks of activations staged per chunk (power of 2)
-  int stages;                // weight ring depth
+  int wstages;               // weight ring depth
+  int xstages;               // activation ring depth
 };
 
 // Each consumer warp owns 32 weight rows (two 16-row MMA tiles). A stage of the
@@ -97,25 +167,21 @@ constexpr int kGemvPitch = 160;
 constexpr int kGemvWarpTile = 32 * kGemvPitch;  // 5120 B
 
 // Shared memory layout (dynamic):
-//   ring [stages][WARPS][32 rows][160 B]              weight tiles (TMA destination)
-//   xs   [8*MT tokens][kc*8 sub-blocks][4][8] bf16    permuted activations of one chunk
-//   xsum [kc*8][8*MT] fp32                            per sub-block sum of x
-//   red  [32*WARPS rows][8*MT] fp32                   per-CTA partial result
-//   bars [2*stages] mbarriers, abort flag
+//   wring [wstages][WARPS][32 rows][160 B]   weight tiles (TMA destination)
+//   xring [xstages][8*MT tokens][576 B]      activation records (bulk-copy destination)
+//   red   [32*WARPS rows][8*MT] fp32         per-CTA partial result
+//   bars  wfull, wempty [wstages], xfull, xempty [xstages]; abort flag
 template <int MT, int WARPS>
 struct GemvSmem {
-  static constexpr size_t ring_stage = (size_t)WARPS * kGemvWarpTile;
-  static __host__ __device__ size_t xs_off(int stages) { return (size_t)stages * ring_stage; }
-  static __host__ __device__ size_t xsum_off(int stages, int kc) {
-    return xs_off(stages) + (size_t)8 * MT * kc * 8 * 32 * 2;
+  static constexpr int TOK = 8 * MT;
+  static constexpr size_t wstage = (size_t)WARPS * kGemvWarpTile;
+  static constexpr size_t xstage = (size_t)TOK * kXRec;
+  static __host__ __device__ size_t xring_off(int ws) { return (size_t)ws * wstage; }
+  static __host__ __device__ size_t red_off(int ws, int xsn) { return xring_off(ws) + (size_t)xsn * xstage; }
+  static __host__ __device__ size_t bar_off(int ws, int xsn) {
+    return red_off(ws, xsn) + (size_t)32 * WARPS * TOK * 4;
   }
-  static __host__ __device__ size_t red_off(int stages, int kc) {
-    return xsum_off(stages, kc) + (size_t)kc * 8 * 8 * MT * 4;
-  }
-  static __host__ __device__ size_t bar_off(int stages, int kc) {
-    return red_off(stages, kc) + (size_t)32 * WARPS * 8 * MT * 4;
-  }
-  static __host__ __device__ size_t total(int stages, int kc) { return bar_off(stages, kc) + 16 * stages + 16; }
+  static __host__ __device__ size_t total(int ws, int xsn) { return bar_off(ws, xsn) + 16 * (ws + xsn) + 16; }
 };
 
 // The eight six-bit scales and mins of a block, four per word as bytes:
@@ -128,25 +194,28 @@ __device__ __forceinline__ void unpack_scales(uint32_t s0, uint32_t s1, uint32_t
   mn[1] = ((s2 >> 4) & 0x0F0F0F0Fu) | ((s1 >> 2) & 0x30303030u);
 }
 
-// Byte b of `word` as the float 2^23 + byte (exact), by one byte permute.
-__device__ __forceinline__ float byte_magic(uint32_t word, int b) {
-  return __uint_as_float(__byte_perm(word, 0x4B000000u, 0x7650u | (uint32_t)b));
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
+// Roles: warps 0..WARPS-1 consume (32 weight rows each); warp WARPS issues the
+// weight TMA; warp WARPS+1 copies the activation records.
 // GROUPED: blockIdx.y enumerates non-empty experts (the y-th expert with a
-// non-zero row count); SWIGLU: the CTA's first WARPS/2 warps hold gate rows and
-// the last WARPS/2 the matching up rows (at +N/2).
+// non-zero row count); SWIGLU: the first WARPS/2 consumer warps hold gate rows
+// and the last WARPS/2 the matching up rows (at +N/2).
 template <int MT, int WARPS, bool GROUPED, bool SWIGLU>
-__global__ void __launch_bounds__(32 * (WARPS + 1)) gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                                                                GemvParams p) {
+__global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                                                                   GemvParams p) {
   using L = GemvSmem<MT, WARPS>;
   constexpr int TOK = 8 * MT;
-  constexpr int NCONS = 32 * WARPS;
   constexpr int ROWS = 32 * WARPS;  // weight rows per CTA
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int S = p.stages;
+  const int SW = p.wstages, SX = p.xstages;
 
   const int rank = (int)(blockIdx.x % (unsigned)p.ksplit);
   const int tile = (int)(blockIdx.x / (unsigned)p.ksplit);
@@ -183,75 +252,76 @@ __global__ void __launch_bounds__(32 * (WARPS + 1)) gemv_kernel(const __grid_con
     }
   }
 
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L::xs_off(S));
-  float* xsum = reinterpret_cast<float*>(smem + L::xsum_off(S, p.kc));
-  float* red = reinterpret_cast<float*>(smem + L::red_off(S, p.kc));
-  const uint32_t bar0 = smem_u32(smem + L::bar_off(S, p.kc));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::bar_off(S, p.kc) + 16 * S);
-  auto bar_full = [&](int s) { return bar0 + 8u * s; };
-  auto bar_empty = [&](int s) { return bar0 + 8u * (S + s); };
-  const int nsb = p.kc * 8;  // sub-blocks per staged chunk
-
-  // First weight row (within the [E*N] row space) of warp w's 32 rows, and
-  // whether those rows exist (N is a multiple of 16, so a warp's second
-  // 16-row tile may be past the end while its first is not).
-  auto warp_row = [&](int w) -> int {
-    int r;
-    if (SWIGLU) {
-      r = (w < WARPS / 2 ? 0 : p.N / 2) + tile * (ROWS / 2) + 32 * (w % (WARPS / 2));
-    } else {
-      r = tile * ROWS + 32 * w;
-    }
-    return expert * p.N + r;
-  };
-  auto rows_left = [&](int w) -> int {  // rows of warp w's 32 that exist
-    const int lim = SWIGLU ? p.N / 2 : p.N;
-    const int r0 = SWIGLU ? tile * (ROWS / 2) + 32 * (w % (WARPS / 2)) : tile * ROWS + 32 * w;
-    return max(0, min(32, lim - r0));
-  };
+  uint8_t* xring = smem + L::xring_off(SW);
+  float* red = reinterpret_cast<float*>(smem + L::red_off(SW, SX));
+  const uint32_t bar0 = smem_u32(smem + L::bar_off(SW, SX));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::bar_off(SW, SX) + 16 * (SW + SX));
+  auto wfull = [&](int s) { return bar0 + 8u * s; };
+  auto wempty = [&](int s) { return bar0 + 8u * (SW + s); };
+  auto xfull = [&](int s) { return bar0 + 8u * (2 * SW + s); };
+  auto xempty = [&](int s) { return bar0 + 8u * (2 * SW + SX + s); };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), WARPS);
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(wfull(s), 1);
+      mbar_init(wempty(s), WARPS);
+    }
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(xfull(s), 1);
+      mbar_init(xempty(s), WARPS);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // Token rows past `count` stay zero for the whole kernel.
-  for (int it = threadIdx.x; it < (TOK - count) * nsb * 4; it += blockDim.x) {
-    const int i = count + it / (nsb * 4), rest = it % (nsb * 4);
-    *reinterpret_cast<uint4*>(xs + ((size_t)i * nsb * 4 + rest) * 8) = make_uint4(0u, 0u, 0u, 0u);
-  }
-  for (int it = threadIdx.x; it < nsb * TOK; it += blockDim.x)
-    if (it % TOK >= count) xsum[it] = 0.f;
   __syncthreads();
 
   if (warp == WARPS) {
-    // ---------------- producer: weight tiles by TMA ----------------
+    // ---------------- weight producer: TMA ----------------
     if (lane == 0) {
+      const int lim = SWIGLU ? p.N / 2 : p.N;
       int issued = 0;
       for (int ks = 0; ks < nk; ++ks) {
-        const int s = ks % S, u = ks / S;
-        if (u >= 1) mbar_wait(bar_empty(s), (u - 1) & 1, abort_flag);
+        const int s = ks % SW, u = ks / SW;
+        if (u >= 1) mbar_wait(wempty(s), (u - 1) & 1, abort_flag);
         if (*abort_flag) break;
-        mbar_arrive_expect_tx(bar_full(s), (uint32_t)(WARPS * kGemvWarpTile));
-        const uint32_t dst = smem_u32(smem) + (uint32_t)(s * L::ring_stage);
+        mbar_arrive_expect_tx(wfull(s), (uint32_t)(WARPS * kGemvWarpTile));
+        const uint32_t dst = smem_u32(smem) + (uint32_t)(s * L::wstage);
         const int x = (kb0 + ks) * BLOCK_BYTES;
 #pragma unroll
-        for (int w = 0; w < WARPS; ++w)
-          tma_load_2d(dst + w * kGemvWarpTile, &tmap_w, x, warp_row(w), bar_full(s));
+        for (int w = 0; w < WARPS; ++w) {
+          int r0 = SWIGLU ? tile * (ROWS / 2) + 32 * (w % (WARPS / 2)) : tile * ROWS + 32 * w;
+          r0 = min(r0, lim);  // rows past the end read zeros (or are ignored)
+          const int row = expert * p.N + (SWIGLU && w >= WARPS / 2 ? p.N / 2 : 0) + r0;
+          tma_load_2d(dst + w * kGemvWarpTile, &tmap_w, x, row, wfull(s));
+        }
         ++issued;
       }
       // Every issued stage must land before the CTA exits (normally the
       // consumers have already waited for all of them).
-      for (int ks = (issued > S ? issued - S : 0); ks < issued; ++ks)
-        mbar_wait(bar_full(ks % S), (ks / S) & 1, abort_flag);
+      for (int ks = (issued > SW ? issued - SW : 0); ks < issued; ++ks)
+        mbar_wait(wfull(ks % SW), (ks / SW) & 1, abort_flag);
+    }
+  } else if (warp == WARPS + 1) {
+    // ---------------- activation producer: bulk copies of prepared records ----------------
+    if (lane == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // the pre-pass has finished
+      int issued = 0;
+      for (int ks = 0; ks < nk; ++ks) {
+        const int s = ks % SX, u = ks / SX;
+        if (u >= 1) mbar_wait(xempty(s), (u - 1) & 1, abort_flag);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(xfull(s), (uint32_t)L::xstage);
+        const uint8_t* src = p.xprep + ((int64_t)(kb0 + ks) * p.rows_pad + row_base) * kXRec;
+        bulk_copy_g2s(smem_u32(xring) + (uint32_t)(s * L::xstage), src, (uint32_t)L::xstage, xfull(s));
+        ++issued;
+      }
+      for (int ks = (issued > SX ? issued - SX : 0); ks < issued; ++ks)
+        mbar_wait(xfull(ks % SX), (ks / SX) & 1, abort_flag);
     }
   } else {
     // ---------------- consumers ----------------
-    const int nrows = rows_left(warp);
-    const bool valid = nrows > 0;
+    const int r0 = SWIGLU ? tile * (ROWS / 2) + 32 * (warp % (WARPS / 2)) : tile * ROWS + 32 * warp;
+    const bool valid = r0 < (SWIGLU ? p.N / 2 : p.N);
     float acc[2][MT][4];
 #pragma unroll
     for (int r = 0; r < 2; ++r)
@@ -259,137 +329,115 @@ __global__ void __launch_bounds__(32 * (WARPS + 1)) gemv_kernel(const __grid_con
       for (int f = 0; f < MT; ++f)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[r][f][e] = 0.f;
+    const __half2 neg1024 = __float2half2_rn(-1024.f);
+    const __half2 sixteenth = __float2half2_rn(0.0625f);
+    const __half2 neg64 = __float2half2_rn(-64.f);
 
-    for (int cb = kb0; cb < kb1;) {
-      // chunk of kcn super-blocks: a power of two, at most kc
-      int kcn = p.kc;
-      while (kcn > kb1 - cb) kcn >>= 1;
-      int lg = 5;  // log2 of the staging items per token (32 per super-block)
-      while ((1 << lg) < 32 * kcn) ++lg;
-      consumer_sync(NCONS);  // previous chunk fully consumed
-      // Stage activations of super-blocks [cb, cb+kcn) for the real tokens: each run
-      // of 8 consecutive k is stored permuted as (e0,e2),(e1,e3),(e4,e6),(e5,e7) to
-      // match the A-fragment nibble order, plus the fp32 sum of every 32-wide
-      // sub-block. Item = (token, sub-block, quarter of 8 k); a warp's 32 lanes take
-      // 32 consecutive items of one token, so a sub-block's quarters are adjacent.
-      auto row_of = [&](int i) -> const uint16_t* {
-        int64_t xrow = i;
-        if (GROUPED) xrow = p.gather ? p.gather[row_base + i] : (row_base + i);
-        return p.X + xrow * p.K + (int64_t)cb * QK;
-      };
-      auto put = [&](int it, const uint4 v) {
-        const int i = it >> lg, q = it & ((1 << lg) - 1);
-        const int sidx = q >> 2, tq = q & 3;
-        uint4 o;
-        o.x = __byte_perm(v.x, v.y, 0x5410);  // (e0, e2)
-        o.y = __byte_perm(v.x, v.y, 0x7632);  // (e1, e3)
-        o.z = __byte_perm(v.z, v.w, 0x5410);  // (e4, e6)
-        o.w = __byte_perm(v.z, v.w, 0x7632);  // (e5, e7)
-        *reinterpret_cast<uint4*>(xs + (((size_t)i * nsb + sidx) * 4 + tq) * 8) = o;
-        float sum = 0.f;
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    for (int ks = 0; ks < nk; ++ks) {
+      const int sw = ks % SW, sx = ks % SX;
+      mbar_wait(wfull(sw), (ks / SW) & 1, abort_flag);
+      const uint8_t* wt = smem + sw * L::wstage + warp * kGemvWarpTile;
+      // rows g, g+8 (tile 0) and g+16, g+24 (tile 1) of this warp's 32
+      uint32_t hdx[4];
+      uint32_t scw[4][2], mnw[4][2];
+      uint2 qv[4][4];  // [row][chunk]
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          sum += bf16_bits_to_float(w4[e] & 0xFFFFu);
-          sum += bf16_bits_to_float(w4[e] >> 16);
-        }
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (tq == 0) xsum[(size_t)sidx * TOK + i] = sum;
-      };
-      const int total = count << lg;  // a multiple of 32: warps are fully in or out
-      int it = threadIdx.x;
-      for (; it + NCONS < total; it += 2 * NCONS) {  // two independent loads in flight
-        const int q0 = it & ((1 << lg) - 1), q1 = (it + NCONS) & ((1 << lg) - 1);
-        const uint4 v0 = ldg_u4(row_of(it >> lg) + (q0 >> 2) * 32 + (q0 & 3) * 8);
-        const uint4 v1 = ldg_u4(row_of((it + NCONS) >> lg) + (q1 >> 2) * 32 + (q1 & 3) * 8);
-        put(it, v0);
-        put(it + NCONS, v1);
+      for (int r = 0; r < 4; ++r) {
+        const uint8_t* rp = wt + (g + 8 * r) * kGemvPitch;
+        const uint4 hd = *reinterpret_cast<const uint4*>(rp);
+        hdx[r] = hd.x;
+        unpack_scales(hd.y, hd.z, hd.w, scw[r], mnw[r]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qv[r][c] = *reinterpret_cast<const uint2*>(rp + 16 + 32 * c + 8 * t);
       }
-      if (it < total) {
-        const int q0 = it & ((1 << lg) - 1);
-        put(it, ldg_u4(row_of(it >> lg) + (q0 >> 2) * 32 + (q0 & 3) * 8));
-      }
-      consumer_sync(NCONS);
-
-      for (int kb = cb; kb < cb + kcn; ++kb) {
-        const int ks = kb - kb0, s = ks % S;
-        mbar_wait(bar_full(s), (ks / S) & 1, abort_flag);
-        const uint8_t* wt = smem + s * L::ring_stage + warp * kGemvWarpTile;
-        // rows g, g+8 (tile 0) and g+16, g+24 (tile 1) of this warp's 32
-        uint4 hd[4];
-        uint2 qv[4][4];  // [row][chunk]
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const uint8_t* rp = wt + (g + 8 * r) * kGemvPitch;
-          hd[r] = *reinterpret_cast<const uint4*>(rp);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) qv[r][c] = *reinterpret_cast<const uint2*>(rp + 16 + 32 * c + 8 * t);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty(s));  // the tile is in registers: release the slot
-        if (!valid) continue;
-
-        // Scales of the four rows: a_j = d*sc_j (exact), b_j = 128*a_j + dmin*m_j.
-        uint32_t scw[4][2], mnw[4][2];
-        float dd[4], dn[4], cd[4], cn[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          unpack_scales(hd[r].y, hd[r].z, hd[r].w, scw[r], mnw[r]);
-          dd[r] = half_bits_to_float(hd[r].x);
-          dn[r] = half_bits_to_float(hd[r].x >> 16);
-          cd[r] = -8388608.f * dd[r];  // -2^23 d, exact
-          cn[r] = -8388608.f * dn[r];
-        }
-        const int sb_base = (kb - cb) * 8;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(wempty(sw));  // the weight tile is in registers: release it
+      mbar_wait(xfull(sx), (ks / SX) & 1, abort_flag);
+      const uint8_t* xb = xring + (size_t)sx * L::xstage;
+      if (valid) {
+        float C[2][MT][4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          uint32_t qs8[4][2];  // words shifted by 8: bytes 1,3 in the positions of bytes 0,2
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            qs8[r][0] = qv[r][c].x >> 8;
+            qs8[r][1] = qv[r][c].y >> 8;
+          }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int j = 2 * c + h;
-            float a[4], b[4];
+            const int j = 2 * c + h;  // sub-block
+            const uint32_t msk = h ? 0x00F000F0u : 0x000F000Fu;
+            // per row: multiplier (sc, or sc/16 for high nibbles) and bias -1024 * multiplier
+            __half2 mul[4], cst[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-              a[r] = fmaf(byte_magic(scw[r][j >> 2], j & 3), dd[r], cd[r]);  // d*sc, exact
-              const float dm = fmaf(byte_magic(mnw[r][j >> 2], j & 3), dn[r], cn[r]);  // dmin*m, exact
-              b[r] = fmaf(128.f, a[r], dm);
+              const __half2 s1024 = bits_h2(bytes_1024(scw[r][j >> 2], j & 3, j & 3));
+              mul[r] = h ? __hfma2(s1024, sixteenth, neg64) : __hadd2(s1024, neg1024);
+              cst[r] = __hmul2(mul[r], neg1024);
             }
-            // A fragments of sub-block j for its two k-steps, both 16-row tiles.
-            const int sh = 4 * h;
-            uint32_t A[2][2][4];  // [tile][k-step][reg]
+            uint32_t A[2][2][4];  // [tile][k-step][reg], fp16 q*sc
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
-              const uint2 lo = qv[2 * tt][c], hi = qv[2 * tt + 1][c];
-              A[tt][0][0] = nib2(lo.x, sh);
-              A[tt][0][1] = nib2(hi.x, sh);
-              A[tt][0][2] = nib2(lo.x, sh + 8);
-              A[tt][0][3] = nib2(hi.x, sh + 8);
-              A[tt][1][0] = nib2(lo.y, sh);
-              A[tt][1][1] = nib2(hi.y, sh);
-              A[tt][1][2] = nib2(lo.y, sh + 8);
-              A[tt][1][3] = nib2(hi.y, sh + 8);
+              const int ra = 2 * tt, rb = 2 * tt + 1;  // rows g(+16), g+8(+16)
+#pragma unroll
+              for (int st = 0; st < 2; ++st) {
+                const uint32_t wa = st ? qv[ra][c].y : qv[ra][c].x, wb = st ? qv[rb][c].y : qv[rb][c].x;
+                const uint32_t sa = qs8[ra][st], sbw = qs8[rb][st];
+                A[tt][st][0] = h2_bits(__hfma2(bits_h2((wa & msk) | 0x64006400u), mul[ra], cst[ra]));
+                A[tt][st][1] = h2_bits(__hfma2(bits_h2((wb & msk) | 0x64006400u), mul[rb], cst[rb]));
+                A[tt][st][2] = h2_bits(__hfma2(bits_h2((sa & msk) | 0x64006400u), mul[ra], cst[ra]));
+                A[tt][st][3] = h2_bits(__hfma2(bits_h2((sbw & msk) | 0x64006400u), mul[rb], cst[rb]));
+              }
             }
-            const int sbi = sb_base + j;
 #pragma unroll
             for (int f = 0; f < MT; ++f) {
-              const uint4 bx = *reinterpret_cast<const uint4*>(
-                  xs + (((size_t)(8 * f + g) * nsb + sbi) * 4 + t) * 8);
-              const float2 sx = *reinterpret_cast<const float2*>(xsum + (size_t)sbi * TOK + 8 * f + 2 * t);
+              const uint4 bx = *reinterpret_cast<const uint4*>(xb + (8 * f + g) * kXRec + (j * 4 + t) * 16);
 #pragma unroll
               for (int tt = 0; tt < 2; ++tt) {
-                float cc[4];
-                mma_bf16_16816(cc, A[tt][0], bx.x, bx.y, true);
-                mma_bf16_16816(cc, A[tt][1], bx.z, bx.w, false);
-                fma2(acc[tt][f][0], acc[tt][f][1], a[2 * tt], cc[0], cc[1]);
-                fma2(acc[tt][f][0], acc[tt][f][1], -b[2 * tt], sx.x, sx.y);
-                fma2(acc[tt][f][2], acc[tt][f][3], a[2 * tt + 1], cc[2], cc[3]);
-                fma2(acc[tt][f][2], acc[tt][f][3], -b[2 * tt + 1], sx.x, sx.y);
+                mma_f16_16816(C[tt][f], A[tt][0][0], A[tt][0][1], A[tt][0][2], A[tt][0][3], bx.x, bx.y,
+                              j == 0);
+                mma_f16_16816(C[tt][f], A[tt][1][0], A[tt][1][1], A[tt][1][2], A[tt][1][3], bx.z, bx.w,
+                              false);
               }
             }
           }
         }
+        // min term: Cm = sum_j m_j * X_j (k = sub-block index; k >= 8 is zero)
+        uint32_t am[4];
+        const uint32_t mb = 2u * (t & 1);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          am[r] = h2_bits(__hadd2(bits_h2(bytes_1024((t >> 1) ? mnw[r][1] : mnw[r][0], mb, mb + 1)),
+                                  neg1024));
+        float dd[4], dn[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          dd[r] = half_bits_to_float(hdx[r]);
+          dn[r] = 64.f * half_bits_to_float(hdx[r] >> 16);
+        }
+#pragma unroll
+        for (int f = 0; f < MT; ++f) {
+          const uint8_t* rg = xb + (8 * f + g) * kXRec;
+          const uint32_t bh = *reinterpret_cast<const uint32_t*>(rg + 512 + 4 * t);
+          const uint32_t bl = *reinterpret_cast<const uint32_t*>(rg + 528 + 4 * t);
+          const float s0 = *reinterpret_cast<const float*>(xb + (8 * f + 2 * t) * kXRec + 544);
+          const float s1 = *reinterpret_cast<const float*>(xb + (8 * f + 2 * t + 1) * kXRec + 544);
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt) {
+            float Cm[4];
+            mma_f16_16816(Cm, am[2 * tt], am[2 * tt + 1], 0u, 0u, bh, 0u, true);
+            mma_f16_16816(Cm, am[2 * tt], am[2 * tt + 1], 0u, 0u, bl, 0u, false);
+            const float dA = dd[2 * tt], dB = dd[2 * tt + 1], mA = dn[2 * tt], mB = dn[2 * tt + 1];
+            acc[tt][f][0] = fmaf(-mA * s0, Cm[0], fmaf(dA * s0, C[tt][f][0], acc[tt][f][0]));
+            acc[tt][f][1] = fmaf(-mA * s1, Cm[1], fmaf(dA * s1, C[tt][f][1], acc[tt][f][1]));
+            acc[tt][f][2] = fmaf(-mB * s0, Cm[2], fmaf(dB * s0, C[tt][f][2], acc[tt][f][2]));
+            acc[tt][f][3] = fmaf(-mB * s1, Cm[3], fmaf(dB * s1, C[tt][f][3], acc[tt][f][3]));
+          }
+        }
       }
-      cb += kcn;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xempty(sx));
     }
 
     // ---- CTA partial -> shared memory: red[local row][token] ----
@@ -453,6 +501,11 @@ inline bool make_tmap_w_rowgroup(CUtensorMap* m, const void* base, int64_t rows,
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Bytes of prepared-activation workspace for `rows` activation rows of K inputs.
+inline size_t gemv_ws_bytes(int64_t rows, int K) {
+  return (size_t)(K / QK) * (size_t)(rows + kXPadRows) * kXRec;
 }
 
 }  // namespace q4k

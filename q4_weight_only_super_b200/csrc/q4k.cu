@@ -35,6 +35,9 @@ cudaError_t ensure_smem(F* func, size_t bytes, std::atomic<size_t> (&set_to)[kMa
   if (bytes <= 48 * 1024 || set_to[dev].load() >= bytes) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(func),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess)  // prefer the largest shared-memory carveout (two CTAs per SM)
+    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(func),
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e == cudaSuccess) set_to[dev].store(bytes);
   return e;
 }
@@ -48,7 +51,7 @@ q4k_status launch_status(cudaError_t e) {
 // ---------------------------------------------------------------- GEMV ----
 
 struct GemvCfg {
-  int mt, warps, ksplit, kc, stages;
+  int mt, warps, ksplit, wstages, xstages;
 };
 
 constexpr int kSms = 148;
@@ -56,24 +59,21 @@ constexpr int kSms = 148;
 // Launch shape for `tokens` (<= 32) tokens against `rows_out` weight rows per
 // matrix and `nkb` super-blocks per row, with `groups` matrices (experts)
 // processed side by side. Depends only on (token class, rows, nkb, groups), so
-// the summation order of a token's result never depends on the batch. The K
-// split (cluster size) is the largest that keeps every CTA resident at once.
+// the summation order of a token's result never depends on the batch. Two
+// CTAs fit per SM; the K split (cluster size) is the largest that keeps every
+// CTA resident at once.
 GemvCfg pick_gemv(int tokens, int rows_out, int nkb, int groups) {
   GemvCfg c;
   c.mt = tokens <= 8 ? 1 : (tokens <= 16 ? 2 : 4);
   c.warps = 4;
-  // two CTAs per SM: ring 4 x 20 KB (3 x 20 KB at 32 tokens) + activations <= 32 KB
-  c.kc = c.mt == 1 ? 4 : (c.mt == 2 ? 2 : 1);
-  c.stages = c.mt == 4 ? 3 : 4;
-  const int per_sm = 2;  // shared-memory residency of one CTA
+  c.wstages = c.mt == 4 ? 3 : 4;
+  c.xstages = c.mt == 1 ? 3 : 2;
   const long tiles = (rows_out + 32 * c.warps - 1) / (32 * c.warps);
-  const long slots = (long)kSms * per_sm;
+  const long slots = (long)kSms * 2;
   long ks = slots / std::max(1L, tiles * groups);
   ks = std::max(1L, std::min<long>(ks, 8));
   ks = std::min<long>(ks, nkb);
   c.ksplit = (int)ks;
-  const int span = (nkb + c.ksplit - 1) / c.ksplit;
-  while (c.kc > 1 && c.kc / 2 >= span) c.kc /= 2;  // power of two, no larger than needed
   return c;
 }
 
@@ -82,32 +82,45 @@ q4k_status launch_gemv_t(const CUtensorMap& tmap, const GemvParams& p, int tiles
                          cudaStream_t s) {
   auto* k = gemv_kernel<MT, WARPS, GROUPED, SWIGLU>;
   static std::atomic<size_t> smem_set[kMaxDevices];  // one per instantiation
-  const size_t smem = GemvSmem<MT, WARPS>::total(p.stages, p.kc);
+  const size_t smem = GemvSmem<MT, WARPS>::total(p.wstages, p.xstages);
   if (ensure_smem(k, smem, smem_set) != cudaSuccess) return Q4K_ERR_LAUNCH;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * p.ksplit), (unsigned)groups, 1);
-  cfg.blockDim = dim3(32 * (WARPS + 1), 1, 1);
+  cfg.blockDim = dim3(32 * (WARPS + 2), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)p.ksplit;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the weight stream starts while the activation
+  // pre-pass still runs; the kernel waits for it before reading its records
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return launch_status(cudaLaunchKernelEx(&cfg, k, tmap, p));
 }
 
+// Activation pre-pass (rows of X, gathered when `gather` is set) then the GEMV.
 template <bool GROUPED, bool SWIGLU>
-q4k_status launch_gemv(const GemvCfg& c, GemvParams p, int rows_out, int groups, cudaStream_t s) {
+q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const int32_t* gather,
+                       int rows, int K, void* ws, int rows_out, int groups, cudaStream_t s) {
   p.ksplit = c.ksplit;
-  p.kc = c.kc;
-  p.stages = c.stages;
+  p.wstages = c.wstages;
+  p.xstages = c.xstages;
+  p.rows_pad = rows + kXPadRows;
+  p.xprep = static_cast<const uint8_t*>(ws);
   CUtensorMap tmap;
   const int64_t row_bytes = (int64_t)p.nkb * BLOCK_BYTES;
   const int64_t total_rows = GROUPED ? (int64_t)p.E * p.N : p.N;
   if (!make_tmap_w_rowgroup(&tmap, p.W, total_rows, row_bytes)) return Q4K_ERR_CUDA;
+  const int64_t recs = (int64_t)p.rows_pad * p.nkb;
+  gemv_prep_kernel<<<(unsigned)((recs + 7) / 8), 256, 0, s>>>(X, gather, rows, p.rows_pad, K, p.nkb,
+                                                               static_cast<uint8_t*>(ws));
+  const q4k_status st = launch_status(cudaGetLastError());
+  if (st != Q4K_OK) return st;
   const int tiles = (rows_out + 32 * c.warps - 1) / (32 * c.warps);
   if (c.mt == 1) return launch_gemv_t<1, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
   if (c.mt == 2) return launch_gemv_t<2, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
@@ -151,22 +164,22 @@ q4k_status q4k_dequant(const void* W, int64_t nblocks, int out_bf16, void* out, 
   return launch_status(cudaGetLastError());
 }
 
-q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* stream) {
+q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws,
+                    size_t ws_bytes, void* stream) {
   if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
   if (M == 0 || N == 0) return Q4K_OK;
-  if (!W || !X || !Y) return Q4K_ERR_NULL;
-  if (!aligned16(W) || !aligned16(X) || !aligned16(Y)) return Q4K_ERR_ALIGN;
+  if (!W || !X || !Y || !ws) return Q4K_ERR_NULL;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(Y) || !aligned16(ws)) return Q4K_ERR_ALIGN;
   if (M > 32 || N % 16) return Q4K_ERR_UNSUPPORTED;
+  if (ws_bytes < gemv_ws_bytes(M, K)) return Q4K_ERR_WORKSPACE;
   GemvParams p = {};
   p.W = static_cast<const uint8_t*>(W);
-  p.X = X;
   p.out = Y;
   p.M = M;
   p.N = N;
-  p.K = K;
   p.nkb = K / QK;
   const GemvCfg c = pick_gemv(M, N, p.nkb, 1);
-  return launch_gemv<false, false>(c, p, N, 1, static_cast<cudaStream_t>(stream));
+  return launch_gemv<false, false>(c, p, X, nullptr, M, K, ws, N, 1, static_cast<cudaStream_t>(stream));
 }
 
 q4k_status q4k_gemm(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws,
@@ -190,12 +203,15 @@ q4k_status q4k_gemm(const void* W, const uint16_t* X, float* Y, int M, int N, in
 
 size_t q4k_workspace_bytes(int op, int M, int N, int K, int E, int topk) {
   (void)N;
-  (void)K;
   (void)topk;
   if (op == Q4K_OP_ROUTE) {
     if (M <= 0 || E <= 0) return 0;
     const size_t tiles = (size_t)(M + kRouteTokPerCta - 1) / kRouteTokPerCta;
     return tiles * (size_t)E * sizeof(int32_t);
+  }
+  if (op == Q4K_OP_GEMV || op == Q4K_OP_GROUPED) {
+    if (M <= 0 || K <= 0 || K % QK) return 0;
+    return gemv_ws_bytes(M, K);
   }
   return 0;
 }
@@ -234,8 +250,6 @@ q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uin
                            const int32_t* row_gather, const int32_t* expert_offsets, int rows,
                            int max_rows_hint, int act, void* out, void* ws, size_t ws_bytes,
                            void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   if (E <= 0 || N <= 0 || K <= 0 || K % QK || rows < 0 || max_rows_hint < 0) return Q4K_ERR_SHAPE;
   if (act != Q4K_ACT_NONE && act != Q4K_ACT_SWIGLU) return Q4K_ERR_UNSUPPORTED;
   if (rows == 0) return Q4K_OK;
@@ -248,23 +262,23 @@ q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uin
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int hint = std::min(max_rows_hint == 0 ? rows : max_rows_hint, rows);
   if (hint <= 32) {
+    if (!ws) return Q4K_ERR_NULL;
+    if (!aligned16(ws)) return Q4K_ERR_ALIGN;
+    if (ws_bytes < gemv_ws_bytes(rows, K)) return Q4K_ERR_WORKSPACE;
     GemvParams p = {};
     p.W = static_cast<const uint8_t*>(W_experts);
-    p.X = A;
     p.out = out;
     p.offsets = expert_offsets;
-    p.gather = row_gather;
     p.N = N;
-    p.K = K;
     p.nkb = nkb;
     p.E = E;
-    p.expert_stride = (int64_t)N * nkb * BLOCK_BYTES;
     const int groups = std::min(E, rows);
     // The same launch shape (hence the same K partition and summation order) for
     // the fp32 and the SwiGLU outputs: a SwiGLU CTA covers as many weight rows.
     const GemvCfg c = pick_gemv(hint, N, nkb, groups);
-    if (act == Q4K_ACT_SWIGLU) return launch_gemv<true, true>(c, p, N, groups, s);
-    return launch_gemv<true, false>(c, p, N, groups, s);
+    if (act == Q4K_ACT_SWIGLU)
+      return launch_gemv<true, true>(c, p, A, row_gather, rows, K, ws, N, groups, s);
+    return launch_gemv<true, false>(c, p, A, row_gather, rows, K, ws, N, groups, s);
   }
   if (N % kGemmBN) return Q4K_ERR_UNSUPPORTED;
   GemmParams p = {};

@@ -44,16 +44,20 @@ def test_status_strings(L):
 
 def test_argument_errors_return_before_launch(L):
     fake = 4096  # never dereferenced: every call below fails validation first
+    big = 1 << 30
     # K not a multiple of 256
-    assert L.q4k_gemv(fake, fake, fake, 1, 16, 100, None) == 3
-    # null pointers
-    assert L.q4k_gemv(None, fake, fake, 1, 16, 256, None) == 1
+    assert L.q4k_gemv(fake, fake, fake, 1, 16, 100, fake, big, None) == 3
+    # null pointers (weights, workspace)
+    assert L.q4k_gemv(None, fake, fake, 1, 16, 256, fake, big, None) == 1
+    assert L.q4k_gemv(fake, fake, fake, 1, 16, 256, None, big, None) == 1
     # misaligned pointer
-    assert L.q4k_gemv(fake + 4, fake, fake, 1, 16, 256, None) == 2
+    assert L.q4k_gemv(fake + 4, fake, fake, 1, 16, 256, fake, big, None) == 2
     # M > 32 is not a GEMV shape
-    assert L.q4k_gemv(fake, fake, fake, 33, 16, 256, None) == 4
+    assert L.q4k_gemv(fake, fake, fake, 33, 16, 256, fake, big, None) == 4
     # N not a multiple of 16
-    assert L.q4k_gemv(fake, fake, fake, 1, 24, 256, None) == 4
+    assert L.q4k_gemv(fake, fake, fake, 1, 24, 256, fake, big, None) == 4
+    # workspace too small
+    assert L.q4k_gemv(fake, fake, fake, 1, 16, 256, fake, 64, None) == 5
     # GEMM N not a multiple of 256
     assert L.q4k_gemm(fake, fake, fake, 4, 128, 256, None, 0, None) == 4
     # routing: too many experts / top-k
@@ -68,7 +72,7 @@ def test_argument_errors_return_before_launch(L):
     assert L.moe_q4k_grouped(fake, 4, 64, 256, fake, None, fake, 8, 8, 7, fake, None, 0, None) == 4
     assert L.moe_combine(fake, fake, fake, 2, 2, 6, fake, None) == 4
     # empty problems are no-ops
-    assert L.q4k_gemv(None, None, None, 0, 16, 256, None) == 0
+    assert L.q4k_gemv(None, None, None, 0, 16, 256, None, 0, None) == 0
     assert L.moe_combine(None, None, None, 0, 2, 8, None, None) == 0
 
 
@@ -76,3 +80,6 @@ def test_workspace_size(L):
     assert L.q4k_workspace_bytes(2, 4096, 0, 0, 128, 8) == 128 * 128 * 4
     assert L.q4k_workspace_bytes(2, 1, 0, 0, 128, 8) == 128 * 4
     assert L.q4k_workspace_bytes(1, 4096, 17408, 5120, 0, 0) == 0
+    # GEMV: (K/256) blocks x (M + 32 padding rows) x 576-byte records
+    assert L.q4k_workspace_bytes(4, 1, 34816, 5120, 0, 0) == 20 * 33 * 576
+    assert L.q4k_workspace_bytes(3, 256, 1536, 2048, 128, 8) == 8 * 288 * 576

@@ -67,7 +67,7 @@ GemvCfg pick_gemv(int tokens, int rows_out, int nkb, int groups) {
   c.mt = tokens <= 8 ? 1 : (tokens <= 16 ? 2 : 4);
   c.warps = 4;
   c.wstages = c.mt == 4 ? 3 : 4;
-  c.xstages = c.mt == 1 ? 3 : 2;
+  c.xstages = c.mt == 1 ? 6 : (c.mt == 2 ? 3 : 2);
   const long tiles = (rows_out + 32 * c.warps - 1) / (32 * c.warps);
   const long slots = (long)kSms * 2;
   long ks = slots / std::max(1L, tiles * groups);

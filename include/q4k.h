@@ -62,8 +62,10 @@ typedef enum {
   Q4K_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up                */
   Q4K_ERR_DEVICE_BOUNDS = 8,  /* a device-side index check failed                  */
   Q4K_ERR_CUDA = 9,           /* a CUDA runtime call returned an error             */
-  Q4K_ERR_DEVICE_RANGE = 10   /* a value does not fit the fp16 operands of the
+  Q4K_ERR_DEVICE_RANGE = 10,  /* a value does not fit the fp16 operands of the
                                  tensor-core grouped path (|x| or |w| > 65504)     */
+  Q4K_ERR_TOO_LARGE = 11      /* the problem needs more than the fixed scratch of
+                                 the no-allocation entry point                     */
 } q4k_status;
 
 enum { Q4K_ACT_NONE = 0, Q4K_ACT_SWIGLU = 1 };
@@ -123,6 +125,30 @@ q4k_status moe_route_permute(const float* logits, int M, int E, int topk,
                              int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
                              int32_t* perm, int32_t* inv_perm, int32_t* row_token,
                              void* ws, size_t ws_bytes, void* stream);
+
+/* moe_route_permute without a workspace argument: for callers that cannot
+ * allocate device memory at call time -- a runtime whose device memory is
+ * owned and budgeted by a host framework that exposes no allocator to this
+ * library, or a serving loop that forbids cudaMalloc after start-up because
+ * it can synchronise the device and stall other streams. There is no
+ * counterpart of this entry point in the paper; it exists only for such callers.
+ * Same arguments, results and errors as moe_route_permute, except:
+ *  - The per-tile expert histograms live in one fixed device array inside
+ *    this library, 65536 int32 (256 KiB), which every GPU that loads the
+ *    library keeps until process exit. Problems needing more, i.e.
+ *    ceil(M / 32) * E > 65536, return Q4K_ERR_TOO_LARGE and launch nothing.
+ *  - The first call on a device looks up that array's device address (a
+ *    cudaGetSymbolAddress with the device current); make that first call
+ *    before any stream capture on that device.
+ *  - Every call, on any stream, uses the same array and it keeps the last
+ *    call's contents (each call overwrites every entry it reads, so nothing
+ *    needs clearing). Calls that may overlap on the GPU race: order them on
+ *    one stream, or with events.
+ *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+q4k_status moe_route_permute_noalloc(const float* logits, int M, int E, int topk,
+                                     int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                                     int32_t* perm, int32_t* inv_perm, int32_t* row_token,
+                                     void* stream);
 
 /* Grouped expert matmul over rows sorted by expert (hipster README, claims
  * table: "MoE grouped GEMM"; hipEngine 0.3.0 README, moe kernels).

@@ -15,6 +15,7 @@ import torch
 
 __all__ = [
     "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemm", "moe_route_permute",
+    "moe_route_permute_noalloc",
     "moe_q4k_grouped", "moe_combine", "q4k_workspace_bytes", "q4k_last_device_status",
     "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "OP_GEMV", "EXPORTS",
 ]
@@ -31,6 +32,7 @@ EXPORTS = {
     "q4k_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "q4k_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "moe_route_permute": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "moe_route_permute_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
     "moe_q4k_grouped": (_i, [_p, _i, _i, _i, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
     "moe_combine": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
     "q4k_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -152,6 +154,28 @@ def moe_route_permute(logits, topk: int, out=None, ws=None, stream=None):
         _ptr(out["expert_offsets"]), _ptr(out["perm"]), _ptr(out["inv_perm"]),
         _ptr(out["row_token"]), _ptr(ws), ws.numel(), _stream(stream))
     _check("moe_route_permute", st)
+    return out
+
+
+def moe_route_permute_noalloc(logits, topk: int, out=None, stream=None):
+    """moe_route_permute with the library's fixed scratch instead of a workspace
+    (for callers that cannot allocate device memory at call time; see q4k.h)."""
+    M, E = logits.shape
+    dev = logits.device
+    if out is None:
+        out = dict(
+            topk_ids=torch.empty(M, topk, dtype=torch.int32, device=dev),
+            topk_w=torch.empty(M, topk, dtype=torch.float32, device=dev),
+            expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            perm=torch.empty(M * topk, dtype=torch.int32, device=dev),
+            inv_perm=torch.empty(M * topk, dtype=torch.int32, device=dev),
+            row_token=torch.empty(M * topk, dtype=torch.int32, device=dev),
+        )
+    st = lib().moe_route_permute_noalloc(
+        _ptr(logits), M, E, topk, _ptr(out["topk_ids"]), _ptr(out["topk_w"]),
+        _ptr(out["expert_offsets"]), _ptr(out["perm"]), _ptr(out["inv_perm"]),
+        _ptr(out["row_token"]), _stream(stream))
+    _check("moe_route_permute_noalloc", st)
     return out
 
 

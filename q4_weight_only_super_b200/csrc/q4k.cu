@@ -127,6 +127,32 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
   return launch_gemv_t<4, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
 }
 
+// Fixed scratch of moe_route_permute_noalloc: one array per device that loads
+// this library, alive until process exit. Host code must not pass the symbol
+// itself to a kernel (on the host it names a host-side stand-in, not device
+// memory): its device address is looked up once per device, with that device
+// current, and cached.
+constexpr size_t kNoAllocRouteInts = 65536;  // 256 KiB
+static __device__ __align__(256) int32_t g_noalloc_route_scratch[kNoAllocRouteInts];
+std::atomic<int32_t*> g_noalloc_route_ptr[kMaxDevices];
+
+q4k_status noalloc_route_scratch(int32_t** out) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return Q4K_ERR_CUDA;
+  int32_t* p = g_noalloc_route_ptr[dev].load();
+  if (!p) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_route_scratch) != cudaSuccess || !addr) {
+      cudaGetLastError();
+      return Q4K_ERR_CUDA;
+    }
+    p = static_cast<int32_t*>(addr);
+    g_noalloc_route_ptr[dev].store(p);
+  }
+  *out = p;
+  return Q4K_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -144,6 +170,7 @@ const char* q4k_status_string(int s) {
     case Q4K_ERR_DEVICE_BOUNDS: return "device-side index out of range";
     case Q4K_ERR_CUDA: return "CUDA runtime error";
     case Q4K_ERR_DEVICE_RANGE: return "value outside the fp16 range of the tensor-core grouped path";
+    case Q4K_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }
@@ -238,6 +265,40 @@ q4k_status moe_route_permute(const float* logits, int M, int E, int topk, int32_
   if (ws_bytes < q4k_workspace_bytes(Q4K_OP_ROUTE, M, 0, 0, E, topk)) return Q4K_ERR_WORKSPACE;
   const int tiles = (M + kRouteTokPerCta - 1) / kRouteTokPerCta;
   int32_t* counts = static_cast<int32_t*>(ws);
+  route_kernel<<<tiles, 32 * kRouteWarps, 0, s>>>(logits, M, E, topk, topk_ids, topk_w, counts);
+  q4k_status st = launch_status(cudaGetLastError());
+  if (st != Q4K_OK) return st;
+  permute_kernel<<<tiles, 256, 0, s>>>(topk_ids, counts, M, E, topk, tiles, expert_offsets, perm,
+                                       inv_perm, row_token);
+  return launch_status(cudaGetLastError());
+}
+
+// The no-allocation variant: same checks and kernels as moe_route_permute, with
+// the per-tile histograms in the library's fixed device array.
+q4k_status moe_route_permute_noalloc(const float* logits, int M, int E, int topk, int32_t* topk_ids,
+                                     float* topk_w, int32_t* expert_offsets, int32_t* perm,
+                                     int32_t* inv_perm, int32_t* row_token, void* stream) {
+  if (M < 0 || E <= 0 || topk <= 0) return Q4K_ERR_SHAPE;
+  if (E > kMaxE || topk > kMaxTopk || topk > E) return Q4K_ERR_UNSUPPORTED;
+  if ((int64_t)M * topk > 0x7fffffffLL) return Q4K_ERR_UNSUPPORTED;
+  if (!expert_offsets) return Q4K_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    return cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), s) == cudaSuccess
+               ? Q4K_OK : Q4K_ERR_CUDA;
+  }
+  if (!logits || !topk_ids || !topk_w || !perm || !inv_perm || !row_token) return Q4K_ERR_NULL;
+  if (!aligned16(logits) || !aligned16(topk_ids) || !aligned16(topk_w) ||
+      !aligned16(expert_offsets) || !aligned16(perm) || !aligned16(inv_perm) ||
+      !aligned16(row_token))
+    return Q4K_ERR_ALIGN;
+  const int tiles = (M + kRouteTokPerCta - 1) / kRouteTokPerCta;
+  if ((size_t)tiles * (size_t)E > kNoAllocRouteInts) return Q4K_ERR_TOO_LARGE;
+  int32_t* counts = nullptr;
+  const q4k_status sst = noalloc_route_scratch(&counts);
+  if (sst != Q4K_OK) return sst;
+  // route_kernel writes every histogram entry permute_kernel reads, so the
+  // array's previous contents never matter and nothing is cleared.
   route_kernel<<<tiles, 32 * kRouteWarps, 0, s>>>(logits, M, E, topk, topk_ids, topk_w, counts);
   q4k_status st = launch_status(cudaGetLastError());
   if (st != Q4K_OK) return st;

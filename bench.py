@@ -314,6 +314,33 @@ def cpu_oracle_gemv_sample(seconds_target=10.0):
             "sample": f"{done} x (512 rows x 5120 Q4_K gate+up GEMV, M=1, dequant+fp64 matmul) in {dt:.1f} s"}
 
 
+# ------------------------------------------------------------ read roof ---
+
+def roof(torch, tm):
+    """Read and copy bandwidth of plain streaming kernels (torch's own) at the
+    GEMV's transfer size (100 MB) and at 1 GB, after a sustained warm-up: the
+    ceiling a single launch of that size can reach on this GPU."""
+    out = {}
+    for nbytes in (100270080, 1 << 30):
+        a = torch.ones(nbytes // 4, dtype=torch.int32, device="cuda")
+        b = torch.empty_like(a)
+        a = a.view(torch.float32).fill_(1.0)
+        b = b.view(torch.float32)
+        for _ in range(50):
+            a.amax()
+        for name, fn, moved in (("read_amax", lambda: a.amax(), nbytes), ("copy", lambda: b.copy_(a), 2 * nbytes)):
+            tm.times.clear()
+            for _ in range(20):
+                tm.run(name, fn)
+            tm.collect()
+            t = min(tm.times[name])
+            out[f"{name}_{nbytes}B_GBps"] = round(moved / t / 1e9, 1)
+            out[f"{name}_{nbytes}B_us"] = round(t * 1e6, 2)
+        del a, b
+    print(json.dumps({"only": "roof", **out}))
+    return 0
+
+
 # ------------------------------------------------------------ single kernel ---
 
 def only(args):
@@ -331,6 +358,8 @@ def only(args):
         return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
 
     tm = Timer(torch)
+    if args.only == "roof":
+        return roof(torch, tm)
     if args.only == "gemv":
         M = args.m or 1
         dd = synth.dense_decode(1)
@@ -384,7 +413,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default=None, choices=["gemv", "gemm", "moe_dec", "moe_pre"],
+    ap.add_argument("--only", default=None, choices=["gemv", "gemm", "moe_dec", "moe_pre", "roof"],
                     help="run one kernel family a few times (for profiler captures), print times")
     ap.add_argument("--m", type=int, default=None, help="tokens for --only")
     ap.add_argument("--proj", default="gate_up", choices=["gate_up", "down"], help="GEMV matrix for --only")

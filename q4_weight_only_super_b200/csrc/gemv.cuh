@@ -19,8 +19,8 @@
 //    bulk copies; mbarriers track both. The GEMV is launched as a programmatic
 //    dependent of the pre-pass, so its weight stream starts while the pre-pass
 //    runs and only the activation copies wait for it.
-//  * Consumer warps own 32 weight rows each (two 16-row tiles, so every
-//    activation fragment feeds two MMAs). The A operand is fp16 q*sc, exact
+//  * Consumer warps own 16 or 32 weight rows each (one or two 16-row MMA
+//    tiles; with two, every activation fragment feeds two MMAs). The A operand is fp16 q*sc, exact
 //    (q*sc <= 945): a nibble ORed into 0x6400 is 1024+q (low nibble) or
 //    1024+16q (high nibble), and one fp16x2 FMA with (sc or sc/16) and
 //    -1024*that removes the bias exactly. So the mma.sync m16n8k16 accumulator
@@ -32,7 +32,7 @@
 //  * The k order inside a sub-block is free for a dot product, so each
 //    thread takes the nibbles in the order the masks produce them, and the
 //    pre-pass stores the activations in that same order.
-//  * A CTA owns 32*WARPS weight rows and a contiguous range of super-blocks;
+//  * A CTA owns 16*TILES*WARPS weight rows and a contiguous range of super-blocks;
 //    a thread-block cluster of KSPLIT CTAs covers the whole K range and its
 //    partial sums are reduced in rank order through distributed shared memory
 //    (deterministic, no atomics). The decomposition depends only on (N, K), and
@@ -70,6 +70,13 @@ __device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   }
+}
+
+// (a & b) | c in one logic instruction.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
@@ -159,27 +166,27 @@ struct GemvParams {
   int xstages;               // activation ring depth
 };
 
-// Each consumer warp owns 32 weight rows (two 16-row MMA tiles). A stage of the
-// weight ring holds, per warp, 32 rows x 160 bytes: one 144-byte super-block plus
-// the first 16 bytes of the next (read and ignored) -- the 160-byte pitch makes the
-// per-thread 8-byte quant reads bank-conflict-free.
+// Each consumer warp owns 16*TILES weight rows (TILES 16-row MMA tiles). A stage
+// of the weight ring holds, per warp, those rows x 160 bytes: one 144-byte
+// super-block plus the first 16 bytes of the next (read and ignored) -- the
+// 160-byte pitch makes the per-thread 8-byte quant reads bank-conflict-free.
 constexpr int kGemvPitch = 160;
-constexpr int kGemvWarpTile = 32 * kGemvPitch;  // 5120 B
 
 // Shared memory layout (dynamic):
-//   wring [wstages][WARPS][32 rows][160 B]   weight tiles (TMA destination)
-//   xring [xstages][8*MT tokens][576 B]      activation records (bulk-copy destination)
-//   red   [32*WARPS rows][8*MT] fp32         per-CTA partial result
+//   wring [wstages][WARPS][16*TILES rows][160 B]   weight tiles (TMA destination)
+//   xring [xstages][8*MT tokens][576 B]            activation records (bulk-copy destination)
+//   red   [16*TILES*WARPS rows][8*MT] fp32         per-CTA partial result
 //   bars  wfull, wempty [wstages], xfull, xempty [xstages]; abort flag
-template <int MT, int WARPS>
+template <int MT, int WARPS, int TILES>
 struct GemvSmem {
   static constexpr int TOK = 8 * MT;
-  static constexpr size_t wstage = (size_t)WARPS * kGemvWarpTile;
+  static constexpr int warp_tile = 16 * TILES * kGemvPitch;
+  static constexpr size_t wstage = (size_t)WARPS * warp_tile;
   static constexpr size_t xstage = (size_t)TOK * kXRec;
   static __host__ __device__ size_t xring_off(int ws) { return (size_t)ws * wstage; }
   static __host__ __device__ size_t red_off(int ws, int xsn) { return xring_off(ws) + (size_t)xsn * xstage; }
   static __host__ __device__ size_t bar_off(int ws, int xsn) {
-    return red_off(ws, xsn) + (size_t)32 * WARPS * TOK * 4;
+    return red_off(ws, xsn) + (size_t)16 * TILES * WARPS * TOK * 4;
   }
   static __host__ __device__ size_t total(int ws, int xsn) { return bar_off(ws, xsn) + 16 * (ws + xsn) + 16; }
 };
@@ -201,17 +208,18 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
       : "memory");
 }
 
-// Roles: warps 0..WARPS-1 consume (32 weight rows each); warp WARPS issues the
-// weight TMA; warp WARPS+1 copies the activation records.
+// Roles: warps 0..WARPS-1 consume (16*TILES weight rows each); warp WARPS issues
+// the weight TMA; warp WARPS+1 copies the activation records.
 // GROUPED: blockIdx.y enumerates non-empty experts (the y-th expert with a
 // non-zero row count); SWIGLU: the first WARPS/2 consumer warps hold gate rows
 // and the last WARPS/2 the matching up rows (at +N/2).
-template <int MT, int WARPS, bool GROUPED, bool SWIGLU>
+template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU>
 __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                                    GemvParams p) {
-  using L = GemvSmem<MT, WARPS>;
+  using L = GemvSmem<MT, WARPS, TILES>;
   constexpr int TOK = 8 * MT;
-  constexpr int ROWS = 32 * WARPS;  // weight rows per CTA
+  constexpr int WROWS = 16 * TILES;    // weight rows per consumer warp
+  constexpr int ROWS = WROWS * WARPS;  // weight rows per CTA
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -280,21 +288,26 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     if (lane == 0) {
       const int lim = SWIGLU ? p.N / 2 : p.N;
       int issued = 0;
+      int s = 0;
+      uint32_t ph = 0;  // stage index and the parity of its current use (no divisions)
       for (int ks = 0; ks < nk; ++ks) {
-        const int s = ks % SW, u = ks / SW;
-        if (u >= 1) mbar_wait(wempty(s), (u - 1) & 1, abort_flag);
+        if (ks >= SW) mbar_wait(wempty(s), ph ^ 1u, abort_flag);
         if (*abort_flag) break;
-        mbar_arrive_expect_tx(wfull(s), (uint32_t)(WARPS * kGemvWarpTile));
+        mbar_arrive_expect_tx(wfull(s), (uint32_t)(WARPS * L::warp_tile));
         const uint32_t dst = smem_u32(smem) + (uint32_t)(s * L::wstage);
         const int x = (kb0 + ks) * BLOCK_BYTES;
 #pragma unroll
         for (int w = 0; w < WARPS; ++w) {
-          int r0 = SWIGLU ? tile * (ROWS / 2) + 32 * (w % (WARPS / 2)) : tile * ROWS + 32 * w;
+          int r0 = SWIGLU ? tile * (ROWS / 2) + WROWS * (w % (WARPS / 2)) : tile * ROWS + WROWS * w;
           r0 = min(r0, lim);  // rows past the end read zeros (or are ignored)
           const int row = expert * p.N + (SWIGLU && w >= WARPS / 2 ? p.N / 2 : 0) + r0;
-          tma_load_2d(dst + w * kGemvWarpTile, &tmap_w, x, row, wfull(s));
+          tma_load_2d(dst + w * L::warp_tile, &tmap_w, x, row, wfull(s));
         }
         ++issued;
+        if (++s == SW) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       // Every issued stage must land before the CTA exits (normally the
       // consumers have already waited for all of them).
@@ -306,25 +319,30 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     if (lane == 0) {
       asm volatile("griddepcontrol.wait;" ::: "memory");  // the pre-pass has finished
       int issued = 0;
+      int s = 0;
+      uint32_t ph = 0;
       for (int ks = 0; ks < nk; ++ks) {
-        const int s = ks % SX, u = ks / SX;
-        if (u >= 1) mbar_wait(xempty(s), (u - 1) & 1, abort_flag);
+        if (ks >= SX) mbar_wait(xempty(s), ph ^ 1u, abort_flag);
         if (*abort_flag) break;
         mbar_arrive_expect_tx(xfull(s), (uint32_t)L::xstage);
         const uint8_t* src = p.xprep + ((int64_t)(kb0 + ks) * p.rows_pad + row_base) * kXRec;
         bulk_copy_g2s(smem_u32(xring) + (uint32_t)(s * L::xstage), src, (uint32_t)L::xstage, xfull(s));
         ++issued;
+        if (++s == SX) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       for (int ks = (issued > SX ? issued - SX : 0); ks < issued; ++ks)
         mbar_wait(xfull(ks % SX), (ks / SX) & 1, abort_flag);
     }
   } else {
     // ---------------- consumers ----------------
-    const int r0 = SWIGLU ? tile * (ROWS / 2) + 32 * (warp % (WARPS / 2)) : tile * ROWS + 32 * warp;
+    const int r0 = SWIGLU ? tile * (ROWS / 2) + WROWS * (warp % (WARPS / 2)) : tile * ROWS + WROWS * warp;
     const bool valid = r0 < (SWIGLU ? p.N / 2 : p.N);
-    float acc[2][MT][4];
+    float acc[TILES][MT][4];
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int r = 0; r < TILES; ++r)
 #pragma unroll
       for (int f = 0; f < MT; ++f)
 #pragma unroll
@@ -333,16 +351,18 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     const __half2 sixteenth = __float2half2_rn(0.0625f);
     const __half2 neg64 = __float2half2_rn(-64.f);
 
+    int sw = 0, sx = 0;
+    uint32_t pw = 0, px = 0;  // ring stage indices and phase parities (no divisions)
     for (int ks = 0; ks < nk; ++ks) {
-      const int sw = ks % SW, sx = ks % SX;
-      mbar_wait(wfull(sw), (ks / SW) & 1, abort_flag);
-      const uint8_t* wt = smem + sw * L::wstage + warp * kGemvWarpTile;
-      // rows g, g+8 (tile 0) and g+16, g+24 (tile 1) of this warp's 32
-      uint32_t hdx[4];
-      uint32_t scw[4][2], mnw[4][2];
-      uint2 qv[4][4];  // [row][chunk]
+      mbar_wait(wfull(sw), pw, abort_flag);
+      const uint8_t* wt = smem + sw * L::wstage + warp * L::warp_tile;
+      // rows g, g+8 (tile 0), g+16, g+24 (tile 1), ... of this warp's rows
+      constexpr int R = 2 * TILES;
+      uint32_t hdx[R];
+      uint32_t scw[R][2], mnw[R][2];
+      uint2 qv[R][4];  // [row][chunk]
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
+      for (int r = 0; r < R; ++r) {
         const uint8_t* rp = wt + (g + 8 * r) * kGemvPitch;
         const uint4 hd = *reinterpret_cast<const uint4*>(rp);
         hdx[r] = hd.x;
@@ -352,15 +372,19 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(wempty(sw));  // the weight tile is in registers: release it
-      mbar_wait(xfull(sx), (ks / SX) & 1, abort_flag);
+      if (++sw == SW) {
+        sw = 0;
+        pw ^= 1u;
+      }
+      mbar_wait(xfull(sx), px, abort_flag);
       const uint8_t* xb = xring + (size_t)sx * L::xstage;
       if (valid) {
-        float C[2][MT][4];
+        float C[TILES][MT][4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t qs8[4][2];  // words shifted by 8: bytes 1,3 in the positions of bytes 0,2
+          uint32_t qs8[R][2];  // words shifted by 8: bytes 1,3 in the positions of bytes 0,2
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
+          for (int r = 0; r < R; ++r) {
             qs8[r][0] = qv[r][c].x >> 8;
             qs8[r][1] = qv[r][c].y >> 8;
           }
@@ -369,32 +393,32 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
             const int j = 2 * c + h;  // sub-block
             const uint32_t msk = h ? 0x00F000F0u : 0x000F000Fu;
             // per row: multiplier (sc, or sc/16 for high nibbles) and bias -1024 * multiplier
-            __half2 mul[4], cst[4];
+            __half2 mul[R], cst[R];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < R; ++r) {
               const __half2 s1024 = bits_h2(bytes_1024(scw[r][j >> 2], j & 3, j & 3));
               mul[r] = h ? __hfma2(s1024, sixteenth, neg64) : __hadd2(s1024, neg1024);
               cst[r] = __hmul2(mul[r], neg1024);
             }
-            uint32_t A[2][2][4];  // [tile][k-step][reg], fp16 q*sc
+            uint32_t A[TILES][2][4];  // [tile][k-step][reg], fp16 q*sc
 #pragma unroll
-            for (int tt = 0; tt < 2; ++tt) {
+            for (int tt = 0; tt < TILES; ++tt) {
               const int ra = 2 * tt, rb = 2 * tt + 1;  // rows g(+16), g+8(+16)
 #pragma unroll
               for (int st = 0; st < 2; ++st) {
                 const uint32_t wa = st ? qv[ra][c].y : qv[ra][c].x, wb = st ? qv[rb][c].y : qv[rb][c].x;
                 const uint32_t sa = qs8[ra][st], sbw = qs8[rb][st];
-                A[tt][st][0] = h2_bits(__hfma2(bits_h2((wa & msk) | 0x64006400u), mul[ra], cst[ra]));
-                A[tt][st][1] = h2_bits(__hfma2(bits_h2((wb & msk) | 0x64006400u), mul[rb], cst[rb]));
-                A[tt][st][2] = h2_bits(__hfma2(bits_h2((sa & msk) | 0x64006400u), mul[ra], cst[ra]));
-                A[tt][st][3] = h2_bits(__hfma2(bits_h2((sbw & msk) | 0x64006400u), mul[rb], cst[rb]));
+                A[tt][st][0] = h2_bits(__hfma2(bits_h2(and_or(wa, msk, 0x64006400u)), mul[ra], cst[ra]));
+                A[tt][st][1] = h2_bits(__hfma2(bits_h2(and_or(wb, msk, 0x64006400u)), mul[rb], cst[rb]));
+                A[tt][st][2] = h2_bits(__hfma2(bits_h2(and_or(sa, msk, 0x64006400u)), mul[ra], cst[ra]));
+                A[tt][st][3] = h2_bits(__hfma2(bits_h2(and_or(sbw, msk, 0x64006400u)), mul[rb], cst[rb]));
               }
             }
 #pragma unroll
             for (int f = 0; f < MT; ++f) {
               const uint4 bx = *reinterpret_cast<const uint4*>(xb + (8 * f + g) * kXRec + (j * 4 + t) * 16);
 #pragma unroll
-              for (int tt = 0; tt < 2; ++tt) {
+              for (int tt = 0; tt < TILES; ++tt) {
                 mma_f16_16816(C[tt][f], A[tt][0][0], A[tt][0][1], A[tt][0][2], A[tt][0][3], bx.x, bx.y,
                               j == 0);
                 mma_f16_16816(C[tt][f], A[tt][1][0], A[tt][1][1], A[tt][1][2], A[tt][1][3], bx.z, bx.w,
@@ -404,15 +428,15 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           }
         }
         // min term: Cm = sum_j m_j * X_j (k = sub-block index; k >= 8 is zero)
-        uint32_t am[4];
+        uint32_t am[R];
         const uint32_t mb = 2u * (t & 1);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < R; ++r)
           am[r] = h2_bits(__hadd2(bits_h2(bytes_1024((t >> 1) ? mnw[r][1] : mnw[r][0], mb, mb + 1)),
                                   neg1024));
-        float dd[4], dn[4];
+        float dd[R], dn[R];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < R; ++r) {
           dd[r] = half_bits_to_float(hdx[r]);
           dn[r] = 64.f * half_bits_to_float(hdx[r] >> 16);
         }
@@ -424,7 +448,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           const float s0 = *reinterpret_cast<const float*>(xb + (8 * f + 2 * t) * kXRec + 544);
           const float s1 = *reinterpret_cast<const float*>(xb + (8 * f + 2 * t + 1) * kXRec + 544);
 #pragma unroll
-          for (int tt = 0; tt < 2; ++tt) {
+          for (int tt = 0; tt < TILES; ++tt) {
             float Cm[4];
             mma_f16_16816(Cm, am[2 * tt], am[2 * tt + 1], 0u, 0u, bh, 0u, true);
             mma_f16_16816(Cm, am[2 * tt], am[2 * tt + 1], 0u, 0u, bl, 0u, false);
@@ -438,14 +462,18 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(xempty(sx));
+      if (++sx == SX) {
+        sx = 0;
+        px ^= 1u;
+      }
     }
 
     // ---- CTA partial -> shared memory: red[local row][token] ----
 #pragma unroll
-    for (int tt = 0; tt < 2; ++tt)
+    for (int tt = 0; tt < TILES; ++tt)
 #pragma unroll
       for (int f = 0; f < MT; ++f) {
-        const int lr = warp * 32 + tt * 16 + g;
+        const int lr = warp * WROWS + tt * 16 + g;
         red[(size_t)lr * TOK + 8 * f + 2 * t] = acc[tt][f][0];
         red[(size_t)lr * TOK + 8 * f + 2 * t + 1] = acc[tt][f][1];
         red[(size_t)(lr + 8) * TOK + 8 * f + 2 * t] = acc[tt][f][2];
@@ -489,14 +517,15 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
   if (p.ksplit > 1) cluster.sync();  // keep every CTA's shared memory alive until rank 0 is done
 }
 
-// Raw Q4_K rows as bytes [rows][row_bytes], box 160 bytes x 32 rows (one super-block per
-// row plus 16 bytes of the next; past the end of a row the box reads zeros).
-inline bool make_tmap_w_rowgroup(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes) {
+// Raw Q4_K rows as bytes [rows][row_bytes], box 160 bytes x box_rows rows (one super-block
+// per row plus 16 bytes of the next; past the end of a row the box reads zeros).
+inline bool make_tmap_w_rowgroup(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes,
+                                 int box_rows) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  cuuint32_t box[2] = {(cuuint32_t)kGemvPitch, 32};
+  cuuint32_t box[2] = {(cuuint32_t)kGemvPitch, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,

@@ -51,7 +51,7 @@ q4k_status launch_status(cudaError_t e) {
 // ---------------------------------------------------------------- GEMV ----
 
 struct GemvCfg {
-  int mt, warps, ksplit, wstages, xstages;
+  int mt, warps, tiles, ksplit, wstages, xstages;
 };
 
 constexpr int kSms = 148;
@@ -65,10 +65,14 @@ constexpr int kSms = 148;
 GemvCfg pick_gemv(int tokens, int rows_out, int nkb, int groups) {
   GemvCfg c;
   c.mt = tokens <= 8 ? 1 : (tokens <= 16 ? 2 : 4);
-  c.warps = 4;
+  // 128 weight rows per CTA: 8 warps x one 16-row tile up to 16 tokens (more warps
+  // to hide latency), 4 warps x two tiles at 32 tokens (each activation fragment
+  // feeds two MMAs)
+  c.tiles = c.mt == 4 ? 2 : 1;
+  c.warps = c.mt == 4 ? 4 : 8;
   c.wstages = c.mt == 4 ? 3 : 4;
   c.xstages = c.mt == 1 ? 6 : (c.mt == 2 ? 3 : 2);
-  const long tiles = (rows_out + 32 * c.warps - 1) / (32 * c.warps);
+  const long tiles = (rows_out + 128 - 1) / 128;
   const long slots = (long)kSms * 2;
   long ks = slots / std::max(1L, tiles * groups);
   ks = std::max(1L, std::min<long>(ks, 8));
@@ -77,12 +81,14 @@ GemvCfg pick_gemv(int tokens, int rows_out, int nkb, int groups) {
   return c;
 }
 
-template <int MT, int WARPS, bool GROUPED, bool SWIGLU>
-q4k_status launch_gemv_t(const CUtensorMap& tmap, const GemvParams& p, int tiles, int groups,
-                         cudaStream_t s) {
-  auto* k = gemv_kernel<MT, WARPS, GROUPED, SWIGLU>;
+template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU>
+q4k_status launch_gemv_t(const GemvParams& p, int rows_total, int tiles, int groups, cudaStream_t s) {
+  auto* k = gemv_kernel<MT, WARPS, TILES, GROUPED, SWIGLU>;
   static std::atomic<size_t> smem_set[kMaxDevices];  // one per instantiation
-  const size_t smem = GemvSmem<MT, WARPS>::total(p.wstages, p.xstages);
+  CUtensorMap tmap;
+  if (!make_tmap_w_rowgroup(&tmap, p.W, rows_total, (int64_t)p.nkb * BLOCK_BYTES, 16 * TILES))
+    return Q4K_ERR_CUDA;
+  const size_t smem = GemvSmem<MT, WARPS, TILES>::total(p.wstages, p.xstages);
   if (ensure_smem(k, smem, smem_set) != cudaSuccess) return Q4K_ERR_LAUNCH;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * p.ksplit), (unsigned)groups, 1);
@@ -112,19 +118,16 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
   p.xstages = c.xstages;
   p.rows_pad = rows + kXPadRows;
   p.xprep = static_cast<const uint8_t*>(ws);
-  CUtensorMap tmap;
-  const int64_t row_bytes = (int64_t)p.nkb * BLOCK_BYTES;
-  const int64_t total_rows = GROUPED ? (int64_t)p.E * p.N : p.N;
-  if (!make_tmap_w_rowgroup(&tmap, p.W, total_rows, row_bytes)) return Q4K_ERR_CUDA;
+  const int total_rows = (int)(GROUPED ? (int64_t)p.E * p.N : p.N);
   const int64_t recs = (int64_t)p.rows_pad * p.nkb;
   gemv_prep_kernel<<<(unsigned)((recs + 7) / 8), 256, 0, s>>>(X, gather, rows, p.rows_pad, K, p.nkb,
                                                                static_cast<uint8_t*>(ws));
   const q4k_status st = launch_status(cudaGetLastError());
   if (st != Q4K_OK) return st;
-  const int tiles = (rows_out + 32 * c.warps - 1) / (32 * c.warps);
-  if (c.mt == 1) return launch_gemv_t<1, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
-  if (c.mt == 2) return launch_gemv_t<2, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
-  return launch_gemv_t<4, 4, GROUPED, SWIGLU>(tmap, p, tiles, groups, s);
+  const int tiles = (rows_out + 128 - 1) / 128;
+  if (c.mt == 1) return launch_gemv_t<1, 8, 1, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
+  if (c.mt == 2) return launch_gemv_t<2, 8, 1, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
+  return launch_gemv_t<4, 4, 2, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
 }
 
 // Fixed scratch of moe_route_permute_noalloc: one array per device that loads

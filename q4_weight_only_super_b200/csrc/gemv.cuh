@@ -468,16 +468,17 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
       }
     }
 
-    // ---- CTA partial -> shared memory: red[local row][token] ----
+    // ---- CTA partial -> shared memory, token-major: red[token][local row] ----
 #pragma unroll
     for (int tt = 0; tt < TILES; ++tt)
 #pragma unroll
       for (int f = 0; f < MT; ++f) {
         const int lr = warp * WROWS + tt * 16 + g;
-        red[(size_t)lr * TOK + 8 * f + 2 * t] = acc[tt][f][0];
-        red[(size_t)lr * TOK + 8 * f + 2 * t + 1] = acc[tt][f][1];
-        red[(size_t)(lr + 8) * TOK + 8 * f + 2 * t] = acc[tt][f][2];
-        red[(size_t)(lr + 8) * TOK + 8 * f + 2 * t + 1] = acc[tt][f][3];
+        const int i0 = 8 * f + 2 * t;
+        red[(size_t)i0 * ROWS + lr] = acc[tt][f][0];
+        red[(size_t)(i0 + 1) * ROWS + lr] = acc[tt][f][1];
+        red[(size_t)i0 * ROWS + lr + 8] = acc[tt][f][2];
+        red[(size_t)(i0 + 1) * ROWS + lr + 8] = acc[tt][f][3];
       }
   }
 
@@ -488,33 +489,43 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     __syncthreads();
   }
 
-  if (rank == 0) {
-    const int outw = SWIGLU ? ROWS / 2 : ROWS;
-    for (int it = threadIdx.x; it < outw * TOK; it += blockDim.x) {
-      const int i = it / outw;       // token
-      const int lr = it % outw;      // local output row (consecutive threads -> consecutive n)
-      if (i >= count) continue;
-      float v = red[(size_t)lr * TOK + i];
-      float u = SWIGLU ? red[(size_t)(lr + ROWS / 2) * TOK + i] : 0.f;
-      for (int r = 1; r < p.ksplit; ++r) {
-        const float* rr = cluster.map_shared_rank(red, r);
-        v += rr[(size_t)lr * TOK + i];
-        if (SWIGLU) u += rr[(size_t)(lr + ROWS / 2) * TOK + i];
+  // Cluster reduction, spread over the ranks: rank r sums a 1/ksplit slice of the
+  // (token, 4 output rows) vectors over all ranks' partials, always in rank order
+  // 0, 1, ..., so the result does not depend on which rank reduces it.
+  {
+    constexpr int OUTW = SWIGLU ? ROWS / 2 : ROWS;
+    constexpr int VPT = OUTW / 4;  // float4 vectors per token
+    const int nvec = count * VPT;
+    const int per = (nvec + p.ksplit - 1) / p.ksplit;
+    const int v0 = rank * per, v1 = min(nvec, v0 + per);
+    for (int v = v0 + (int)threadIdx.x; v < v1; v += blockDim.x) {
+      const int i = v / VPT, lr = (v % VPT) * 4;
+      float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f), u4 = g4;
+      for (int r = 0; r < p.ksplit; ++r) {
+        const float* rr = p.ksplit > 1 ? cluster.map_shared_rank(red, r) : red;
+        const float4 a4 = *reinterpret_cast<const float4*>(rr + (size_t)i * ROWS + lr);
+        g4.x += a4.x; g4.y += a4.y; g4.z += a4.z; g4.w += a4.w;
+        if (SWIGLU) {
+          const float4 b4 = *reinterpret_cast<const float4*>(rr + (size_t)i * ROWS + lr + ROWS / 2);
+          u4.x += b4.x; u4.y += b4.y; u4.z += b4.z; u4.w += b4.w;
+        }
       }
       if (SWIGLU) {
         const int half = p.N / 2;
         const int n = tile * (ROWS / 2) + lr;
-        if (n < half) {
-          const __nv_bfloat16 hb = __float2bfloat16_rn(silu_mul(v, u));
-          static_cast<uint16_t*>(p.out)[(int64_t)(row_base + i) * half + n] = __bfloat16_as_ushort(hb);
+        if (n < half) {  // half % 16 == 0, so all four are in range
+          uint2 o;
+          o.x = pack_bf16x2(silu_mul(g4.x, u4.x), silu_mul(g4.y, u4.y));
+          o.y = pack_bf16x2(silu_mul(g4.z, u4.z), silu_mul(g4.w, u4.w));
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + (int64_t)(row_base + i) * half + n) = o;
         }
       } else {
         const int n = tile * ROWS + lr;
-        if (n < p.N) static_cast<float*>(p.out)[(int64_t)(row_base + i) * p.N + n] = v;
+        if (n < p.N) *reinterpret_cast<float4*>(static_cast<float*>(p.out) + (int64_t)(row_base + i) * p.N + n) = g4;
       }
     }
   }
-  if (p.ksplit > 1) cluster.sync();  // keep every CTA's shared memory alive until rank 0 is done
+  if (p.ksplit > 1) cluster.sync();  // keep every CTA's shared memory alive until all ranks are done
 }
 
 // Raw Q4_K rows as bytes [rows][row_bytes], box 160 bytes x box_rows rows (one super-block

@@ -183,12 +183,12 @@ struct GemvSmem {
   static constexpr int warp_tile = 16 * TILES * kGemvPitch;
   static constexpr size_t wstage = (size_t)WARPS * warp_tile;
   static constexpr size_t xstage = (size_t)TOK * kXRec;
-  static __host__ __device__ size_t xring_off(int ws) { return (size_t)ws * wstage; }
-  static __host__ __device__ size_t red_off(int ws, int xsn) { return xring_off(ws) + (size_t)xsn * xstage; }
-  static __host__ __device__ size_t bar_off(int ws, int xsn) {
+  static constexpr __host__ __device__ size_t xring_off(int ws) { return (size_t)ws * wstage; }
+  static constexpr __host__ __device__ size_t red_off(int ws, int xsn) { return xring_off(ws) + (size_t)xsn * xstage; }
+  static constexpr __host__ __device__ size_t bar_off(int ws, int xsn) {
     return red_off(ws, xsn) + (size_t)16 * TILES * WARPS * TOK * 4;
   }
-  static __host__ __device__ size_t total(int ws, int xsn) { return bar_off(ws, xsn) + 16 * (ws + xsn) + 16; }
+  static constexpr __host__ __device__ size_t total(int ws, int xsn) { return bar_off(ws, xsn) + 16 * (ws + xsn) + 16; }
 };
 
 // The eight six-bit scales and mins of a block, four per word as bytes:

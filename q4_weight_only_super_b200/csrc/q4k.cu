@@ -54,31 +54,78 @@ struct GemvCfg {
   int mt, warps, tiles, ksplit, wstages, xstages;
 };
 
-constexpr int kSms = 148;
+// Ring depths per token class (weight stages, activation stages). Every class
+// must fit two CTAs per SM: 228 KiB of shared memory per SM, 1 KiB of it
+// reserved per CTA. Then one cluster-fit table serves every class, so the K
+// split -- and with it the summation order -- does not depend on the class.
+constexpr size_t kGemvTwoPerSm = 233472 / 2 - 1024;
+constexpr int kGemvStages[3][2] = {{4, 6}, {4, 2}, {3, 2}};  // mt = 1, 2, 4
+static_assert(GemvSmem<1, 8, 1>::total(kGemvStages[0][0], kGemvStages[0][1]) <= kGemvTwoPerSm, "mt 1");
+static_assert(GemvSmem<2, 8, 1>::total(kGemvStages[1][0], kGemvStages[1][1]) <= kGemvTwoPerSm, "mt 2");
+static_assert(GemvSmem<4, 4, 2>::total(kGemvStages[2][0], kGemvStages[2][1]) <= kGemvTwoPerSm, "mt 4");
+
+// fit[d][ks]: clusters of ks GEMV CTAs that can be resident at once on device d
+// (a cluster must sit inside one GPC, so this is below 2 * SMs / ks).
+std::atomic<int> g_gemv_fit[kMaxDevices][9];
+std::atomic<size_t> g_gemv_fit_smem_set[kMaxDevices];
+
+q4k_status gemv_cluster_fit(int ks, int* fit) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices || ks < 1 || ks > 8) return Q4K_ERR_CUDA;
+  int v = g_gemv_fit[dev][ks].load();
+  if (v <= 0) {
+    auto* k = gemv_kernel<1, 8, 1, false, false>;
+    const size_t smem = GemvSmem<1, 8, 1>::total(kGemvStages[0][0], kGemvStages[0][1]);
+    if (ensure_smem(k, smem, g_gemv_fit_smem_set) != cudaSuccess) return launch_status(cudaErrorUnknown);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(ks * 64), 1, 1);
+    cfg.blockDim = dim3(32 * (8 + 2), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&v, k, &cfg) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      return Q4K_ERR_CUDA;
+    }
+    g_gemv_fit[dev][ks].store(v);
+  }
+  *fit = v;
+  return Q4K_OK;
+}
 
 // Launch shape for `tokens` (<= 32) tokens against `rows_out` weight rows per
 // matrix and `nkb` super-blocks per row, with `groups` matrices (experts)
-// processed side by side. Depends only on (token class, rows, nkb, groups), so
-// the summation order of a token's result never depends on the batch. Two
-// CTAs fit per SM; the K split (cluster size) is the largest that keeps every
-// CTA resident at once.
-GemvCfg pick_gemv(int tokens, int rows_out, int nkb, int groups) {
+// processed side by side. Depends only on (rows, nkb, groups) and the device,
+// so the summation order of a token's result never depends on the batch. The
+// K split (cluster size, at most 8) is the largest that keeps every cluster
+// resident at once: a cluster that does not fit waits for a whole second wave.
+q4k_status pick_gemv(int tokens, int rows_out, int nkb, int groups, GemvCfg* out) {
   GemvCfg c;
   c.mt = tokens <= 8 ? 1 : (tokens <= 16 ? 2 : 4);
+  const int cls = c.mt == 1 ? 0 : (c.mt == 2 ? 1 : 2);
   // 128 weight rows per CTA: 8 warps x one 16-row tile up to 16 tokens (more warps
   // to hide latency), 4 warps x two tiles at 32 tokens (each activation fragment
   // feeds two MMAs)
   c.tiles = c.mt == 4 ? 2 : 1;
   c.warps = c.mt == 4 ? 4 : 8;
-  c.wstages = c.mt == 4 ? 3 : 4;
-  c.xstages = c.mt == 1 ? 6 : (c.mt == 2 ? 3 : 2);
-  const long tiles = (rows_out + 128 - 1) / 128;
-  const long slots = (long)kSms * 2;
-  long ks = slots / std::max(1L, tiles * groups);
-  ks = std::max(1L, std::min<long>(ks, 8));
-  ks = std::min<long>(ks, nkb);
-  c.ksplit = (int)ks;
-  return c;
+  c.wstages = kGemvStages[cls][0];
+  c.xstages = kGemvStages[cls][1];
+  const long clusters = (long)((rows_out + 128 - 1) / 128) * groups;
+  int ks = std::max(1, std::min(8, nkb));
+  for (; ks > 1; --ks) {
+    int fit = 0;
+    const q4k_status st = gemv_cluster_fit(ks, &fit);
+    if (st != Q4K_OK) return st;
+    if ((long)fit >= clusters) break;
+  }
+  c.ksplit = ks;
+  *out = c;
+  return Q4K_OK;
 }
 
 template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU>
@@ -208,7 +255,9 @@ q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
   p.M = M;
   p.N = N;
   p.nkb = K / QK;
-  const GemvCfg c = pick_gemv(M, N, p.nkb, 1);
+  GemvCfg c;
+  const q4k_status st = pick_gemv(M, N, p.nkb, 1, &c);
+  if (st != Q4K_OK) return st;
   return launch_gemv<false, false>(c, p, X, nullptr, M, K, ws, N, 1, static_cast<cudaStream_t>(stream));
 }
 
@@ -339,7 +388,9 @@ q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uin
     const int groups = std::min(E, rows);
     // The same launch shape (hence the same K partition and summation order) for
     // the fp32 and the SwiGLU outputs: a SwiGLU CTA covers as many weight rows.
-    const GemvCfg c = pick_gemv(hint, N, nkb, groups);
+    GemvCfg c;
+    const q4k_status st = pick_gemv(hint, N, nkb, groups, &c);
+    if (st != Q4K_OK) return st;
     if (act == Q4K_ACT_SWIGLU)
       return launch_gemv<true, true>(c, p, A, row_gather, rows, K, ws, N, groups, s);
     return launch_gemv<true, false>(c, p, A, row_gather, rows, K, ws, N, groups, s);

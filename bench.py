@@ -10,11 +10,18 @@ shaped like the dense and MoE decode/prefill workloads:
 
 The headline metric is the decode GEMV's effective HBM bandwidth (weight bytes
 per second over the ten GEMV launches of a step); the prefill GEMM TFLOP/s and
-the MoE layer tokens/s are reported beside it. Every kernel is timed with CUDA
-events on the stream it runs on, with L2 flushed (a 256 MiB write) before each
-timed launch. Weights and activations are resident in HBM before timing
-starts; the `e2e` figure repeats the GEMV measurement through the C ABI with
-host (pinned) activations copied in and results copied out inside the timing.
+the MoE layer tokens/s are reported beside it. All timing uses CUDA events on
+the stream the kernels run on. The decode GEMVs and the prefill GEMMs run as
+back-to-back launches over rotating copies of their weight matrices (as the
+layers of a model do): 6 copies of gate+up (600 MB), 10 of down (500 MB), 3 of
+the prefill matrix, so no launch finds its weights in the 126 MB L2; a
+sequence's time over its launch count is the per-launch time. The MoE layers
+(four launches each) and their stages are timed after a clean L2 flush (a
+256 MiB write, then a 256 MiB read of another buffer, so no dirty lines are
+left to be written back during the timed launches). Weights and activations
+are resident in HBM before timing starts; the `e2e` figure repeats the GEMV
+measurement through the C ABI with host (pinned) activations copied in and
+results copied out inside the timing.
 
 `--impl reference` times the CPU oracle instead, on a bounded sample.
 Under torchrun each rank runs an independent replica (the path has no
@@ -54,30 +61,59 @@ def _peaks():
 # ----------------------------------------------------------------- clocks ---
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clock and throttle reasons (every 20 ms) from the
+    start of warm-up to the end of the timed region. Each sample carries the
+    host wall time at which it was read; the clock figures reported are those of
+    the samples inside the timed region, or of the whole loaded span when the
+    timed region was too short to hold one (said in `window`)."""
 
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.samples = []  # (host time, line)
+        self.window = None
 
-    def start(self):
+    def start(self, wait_s: float = 3.0):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except OSError:
             self.proc = None
+            return
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < wait_s:  # let the first sample arrive
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, t_begin: float, t_end: float):
+        self.window = (t_begin, t_end)
+
+    def _parse(self, lines):
+        sm, mx, reasons = [], [], set()
+        for ln in lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(self.NAMES, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return sm, mx, reasons
 
     def stop(self):
         if self.proc is None:
@@ -88,49 +124,74 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.t.join(timeout=2)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
+        timed = [ln for t, ln in self.samples if self.window and self.window[0] <= t <= self.window[1]]
+        sm, mx, reasons = self._parse(timed)
+        window = "timed region"
+        if not sm:
+            sm, mx, reasons = self._parse([ln for _, ln in self.samples])
+            window = "warm-up and timed region (none fell inside the timed region alone)"
+        _, _, all_reasons = self._parse([ln for _, ln in self.samples])
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "window": window,
+                "reasons_whole_run": sorted(all_reasons), "samples_whole_run": len(self.samples)}
 
 
 # ------------------------------------------------------------ GPU harness ---
 
 class Timer:
-    """Per-kernel CUDA-event timing on the current stream, L2 flushed before each launch."""
+    """CUDA-event timing on the current stream: single launches after a clean L2
+    flush (`run`), or back-to-back launch sequences (`run_seq`)."""
 
     def __init__(self, torch):
         self.torch = torch
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-        self.pending = []  # (key, start, end)
+        self.read_buf = torch.ones(256 << 20, dtype=torch.uint8, device="cuda")
+        self.pending = []  # (key, start, end, launches)
         self.times = {}
+
+    def flush(self):
+        self.flush_buf.fill_(1)
+        self.read_buf.view(self.torch.int64).sum()
 
     def run(self, key, fn):
         t = self.torch
-        self.flush_buf.fill_(1)
+        self.flush()
         s, e = t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True)
         s.record()
         out = fn()
         e.record()
-        self.pending.append((key, s, e))
+        self.pending.append((key, s, e, 1))
         return out
+
+    def begin(self):
+        """Start event of a timed region (the caller launches, then calls `end`)."""
+        t = self.torch
+        self.flush()
+        s = t.cuda.Event(enable_timing=True)
+        s.record()
+        return s
+
+    def end(self, key, s, launches=1):
+        e = self.torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.pending.append((key, s, e, launches))
+
+    def run_seq(self, key, fns):
+        """Launch fns back to back; the per-launch time is the sequence time / len(fns).
+        The GPU sleeps first (untimed) so that the host has queued the whole sequence."""
+        t = self.torch
+        t.cuda._sleep(400000)
+        s, e = t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True)
+        s.record()
+        for f in fns:
+            f()
+        e.record()
+        self.pending.append((key, s, e, len(fns)))
 
     def collect(self):
         self.torch.cuda.synchronize()
-        for key, s, e in self.pending:
-            self.times.setdefault(key, []).append(s.elapsed_time(e) * 1e-3)
+        for key, s, e, n in self.pending:
+            self.times.setdefault(key, []).append(s.elapsed_time(e) * 1e-3 / n)
         self.pending.clear()
 
 
@@ -142,10 +203,14 @@ def build_workloads(torch, q, synth):
     W = {}
     dd = synth.dense_decode(1)
     W["dec"] = {k: dev(v) for k, v in dd.items()}
+    # rotating copies of the decode weights: 6 x 100 MB (gate+up), 10 x 50 MB (down)
+    W["dec_copies"] = {"gate_up": [W["dec"]["W_gate_up"]] + [W["dec"]["W_gate_up"].clone() for _ in range(5)],
+                       "down": [W["dec"]["W_down"]] + [W["dec"]["W_down"].clone() for _ in range(9)]}
     W["dec_shapes"] = {p: (dd[f"W_{p}"].shape[0], dd[f"W_{p}"].shape[1] * 256) for p in ("gate_up", "down")}
     W["dec_host_X"] = {p: torch.from_numpy(dd[f"X_{p}"].view(np.int16)).pin_memory() for p in ("gate_up", "down")}
     Wp, Xp = synth.dense_prefill(2)
     W["pre"] = (dev(Wp), dev(Xp), Wp.shape[0], Wp.shape[1] * 256)
+    W["pre_copies"] = [W["pre"][0]] + [W["pre"][0].clone() for _ in range(2)]
     del Wp, Xp
     md = synth.moe_decode(3, 32)
     W["moe_dec"] = {k: dev(md[k]) for k in ("logits", "X", "W_gate_up", "W_down")}
@@ -157,21 +222,56 @@ def build_workloads(torch, q, synth):
     need = max(q.q4k_workspace_bytes(q.OP_GEMV, 32, 0, 17408),
                q.q4k_workspace_bytes(q.OP_GROUPED, 32 * 8, 0, 2048))
     W["ws"] = torch.empty(need, dtype=torch.uint8, device="cuda")
+    # outputs, allocated once: decode Y (32 tokens x the widest projection), prefill Y
+    W["dec_Y"] = torch.empty(32 * max(n for n, _ in W["dec_shapes"].values()), dtype=torch.float32, device="cuda")
+    W["pre_Y"] = torch.empty(4096 * W["pre"][2], dtype=torch.float32, device="cuda")
     return W
 
 
-def moe_layer_gpu(q, tm, key, d, M, dims, topk=8):
+def moe_buffers(torch, q, d, M, dims, topk=8):
+    """Outputs and scratch of one MoE layer at M tokens, allocated once per M (as a
+    serving loop would), so that the timed region holds no allocation."""
+    bufs = d.setdefault("bufs", {})
+    if M not in bufs:
+        E, H, F = dims
+        rows = M * topk
+        i32 = dict(dtype=torch.int32, device="cuda")
+        bufs[M] = {
+            "route": dict(topk_ids=torch.empty(M, topk, **i32),
+                          topk_w=torch.empty(M, topk, dtype=torch.float32, device="cuda"),
+                          expert_offsets=torch.empty(E + 1, **i32), perm=torch.empty(rows, **i32),
+                          inv_perm=torch.empty(rows, **i32), row_token=torch.empty(rows, **i32)),
+            "route_ws": torch.empty(max(16, q.q4k_workspace_bytes(q.OP_ROUTE, M, E=E, topk=topk)),
+                                    dtype=torch.uint8, device="cuda"),
+            "h": torch.empty(rows, F, dtype=torch.bfloat16, device="cuda"),
+            "o": torch.empty(rows, H, dtype=torch.float32, device="cuda"),
+            "y": torch.empty(M, H, dtype=torch.float32, device="cuda"),
+        }
+    return bufs[M]
+
+
+def moe_layer_gpu(q, tm, key, d, M, dims, topk=8, staged=True):
+    """One MoE layer (four launches). staged: each stage timed on its own after a
+    flush (the breakdown); else the four launches timed together (the layer time)."""
+    import torch
     E, H, F = dims
     rows = M * topk
+    b = moe_buffers(torch, q, d, M, dims, topk)
     logits, X = d["logits"][:M], d["X"][:M]
-    r = tm.run(key + ":route", lambda: q.moe_route_permute(logits, topk))
     ws = d.get("ws") if M <= 32 else None
-    h = tm.run(key + ":gate_up", lambda: q.moe_q4k_grouped(d["W_gate_up"], E, 2 * F, H, X, r["expert_offsets"],
-                                                            rows, M, q.ACT_SWIGLU, row_gather=r["row_token"],
-                                                            ws=ws))
-    o = tm.run(key + ":down", lambda: q.moe_q4k_grouped(d["W_down"], E, H, F, h, r["expert_offsets"], rows, M,
-                                                         q.ACT_NONE, ws=ws))
-    return tm.run(key + ":combine", lambda: q.moe_combine(o, r["inv_perm"], r["topk_w"], M, topk, H)), r
+    stage = (lambda k, fn: tm.run(key + ":" + k, fn)) if staged else (lambda k, fn: fn())
+    if not staged:
+        s = tm.begin()
+    r = stage("route", lambda: q.moe_route_permute(logits, topk, out=b["route"], ws=b["route_ws"]))
+    h = stage("gate_up", lambda: q.moe_q4k_grouped(d["W_gate_up"], E, 2 * F, H, X, r["expert_offsets"],
+                                                  rows, M, q.ACT_SWIGLU, row_gather=r["row_token"],
+                                                  out=b["h"], ws=ws))
+    o = stage("down", lambda: q.moe_q4k_grouped(d["W_down"], E, H, F, h, r["expert_offsets"], rows, M,
+                                               q.ACT_NONE, out=b["o"], ws=ws))
+    y = stage("combine", lambda: q.moe_combine(o, r["inv_perm"], r["topk_w"], M, topk, H, Y=b["y"]))
+    if not staged:
+        tm.end(key + ":layer", s)
+    return y, r
 
 
 def run_step(q, tm, W):
@@ -179,19 +279,24 @@ def run_step(q, tm, W):
     for M in (1, 4, 8, 16, 32):
         for p in ("gate_up", "down"):
             N, K = W["dec_shapes"][p]
-            Wt, Xt = W["dec"][f"W_{p}"], W["dec"][f"X_{p}"][:M]
-            tm.run(f"gemv:{p}:M{M}", lambda: q.q4k_gemv(Wt, Xt, N, K, ws=W["ws"]))
-            launches += 1
-    Wt, Xt, N, K = W["pre"]
+            Xt = W["dec"][f"X_{p}"][:M]
+            Y = W["dec_Y"][:M * N].view(M, N)
+            fns = [lambda Wt=Wt: q.q4k_gemv(Wt, Xt, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_copies"][p]]
+            tm.run_seq(f"gemv:{p}:M{M}", fns)
+            launches += 2 * len(fns)  # activation pre-pass + GEMV per call
+    _, Xt, N, K = W["pre"]
     for M in (512, 4096):
-        tm.run(f"gemm:M{M}", lambda: q.q4k_gemm(Wt, Xt[:M], N, K))
-        launches += 1
+        Y = W["pre_Y"][:M * N].view(M, N)
+        fns = [lambda Wt=Wt: q.q4k_gemm(Wt, Xt[:M], N, K, Y=Y) for Wt in W["pre_copies"]]
+        tm.run_seq(f"gemm:M{M}", fns)
+        launches += len(fns)
     W["moe_dec"]["ws"] = W["ws"]
-    for M in (1, 8, 32):
-        moe_layer_gpu(q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"])
+    for staged in (True, False):
+        for M in (1, 8, 32):
+            moe_layer_gpu(q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"], staged=staged)
+            launches += 5  # route (histogram + permute), gate_up, down, combine
+        moe_layer_gpu(q, tm, "moe_pre:M4096", W["moe_pre"], 4096, W["moe_dims"], staged=staged)
         launches += 5
-    moe_layer_gpu(q, tm, "moe_pre:M4096", W["moe_pre"], 4096, W["moe_dims"])
-    launches += 5
     return launches
 
 
@@ -252,16 +357,41 @@ def summarize(tm, W, peaks):
         comp[f"gemm_M{M}_us"] = round(t * 1e6, 1)
     for key, M in (("moe_dec", 1), ("moe_dec", 8), ("moe_dec", 32), ("moe_pre", 4096)):
         parts = [T[f"{key}:M{M}:{s}"] for s in ("route", "gate_up", "down", "combine")]
-        comp[f"{key}_M{M}_tokens_per_s"] = round(M / sum(parts), 1)
-        comp[f"{key}_M{M}_us"] = {s: round(x * 1e6, 2) for s, x in zip(("route", "gate_up", "down", "combine"), parts)}
+        comp[f"{key}_M{M}_tokens_per_s"] = round(M / T[f"{key}:M{M}:layer"], 1)
+        comp[f"{key}_M{M}_layer_us"] = round(T[f"{key}:M{M}:layer"] * 1e6, 2)
+        comp[f"{key}_M{M}_stage_us"] = {s: round(x * 1e6, 2) for s, x in zip(("route", "gate_up", "down", "combine"), parts)}
     gbps = gemv_bytes / gemv_time / 1e9
-    # dominant kernel by time in a step
-    dom = max(T.items(), key=lambda kv: kv[1])
+    # dominant kernel: the one with the most device time per step (single kernels
+    # only: whole-layer timings are not kernels); GEMV/GEMM times are per launch,
+    # so weigh them by their launches per step
+    per_step = {}
+    for k, v in T.items():
+        if k.endswith(":layer"):
+            continue
+        n = 1
+        if k.startswith("gemv:"):
+            n = len(W["dec_copies"][k.split(":")[1]])
+        elif k.startswith("gemm:"):
+            n = len(W["pre_copies"])
+        per_step[k] = v * n
+    dom = max(per_step.items(), key=lambda kv: kv[1])
     return gbps, comp, T, dom
+
+
+# DRAM bytes (read + write) per launch of each kernel, from one ncu capture of the
+# same kernel code (dram__bytes_read.sum + dram__bytes_write.sum); the captures
+# and their commands are summarised in profiles/. None where not captured.
+TRAFFIC = {
+    "gemv:gate_up:M1": 102.685952e6 + 4.229888e6,   # profiles/gemv_gate_up_34816x5120_M1.md
+    "gemm:M512": 55.47e6 + 3.73e6,                  # profiles/gemm_prefill_17408x5120.md
+    "gemm:M4096": 334.03e6 + 238.74e6,              # profiles/gemm_prefill_17408x5120.md
+}
 
 
 def roofline_for(key, T, W, peaks, traffic=None):
     t = T[key]
+    if traffic is None:
+        traffic = TRAFFIC.get(key)
     if key.startswith("gemm:"):
         M = int(key.split("M")[-1])
         _, _, N, K = W["pre"]
@@ -471,6 +601,8 @@ def main():
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
+    clk = ClockSampler(local)
+    clk.start()
     for _ in range(args.warmup):
         run_step(q, tm, W)
     tm.collect()
@@ -478,9 +610,8 @@ def main():
     st = q.q4k_last_device_status()
     assert st == 0, f"device status {st} after warm-up"
 
-    clk = ClockSampler(local)
     barrier()
-    clk.start()
+    t_wall0 = time.time()
     t0 = time.perf_counter()
     s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s_ev.record()
@@ -490,6 +621,7 @@ def main():
     e_ev.record()
     barrier()
     wall = time.perf_counter() - t0
+    clk.mark(t_wall0, time.time())
     clocks = clk.stop()
     tm.collect()
     step_s = s_ev.elapsed_time(e_ev) * 1e-3 / args.steps
@@ -516,7 +648,9 @@ def main():
             "config": {"workload": "Q4_K dense decode GEMV gate+up 34816x5120 and down 5120x17408 at "
                                    "M=1,4,8,16,32 (seed 1); step also runs prefill GEMM 17408x5120 at "
                                    "M=512,4096 and MoE layers (128 experts, top-8) at M=1,8,32,4096",
-                       "l2": "256 MiB flush write before every timed kernel",
+                       "l2": "GEMV/GEMM: back-to-back launches over rotating weight copies (600 MB gate+up, "
+                             "500 MB down, 150 MB prefill), no flush; MoE: clean flush (256 MiB write + 256 MiB "
+                             "read) before each timed layer and stage",
                        "parallelism": "replicas" if world > 1 else "single GPU",
                        "moe_prefill_hot_experts": W["moe_pre_hot"]},
             "frac_of_hbm_peak": round(gbps_all / world / peaks["hbm"], 4),

@@ -96,6 +96,10 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const uint16_t* __restri
                                                         int rows_pad, int K, int nkb,
                                                         uint8_t* __restrict__ ws) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // X and the gather indices may come from the previous kernel. (The GEMV, the
+  // only reader of this workspace, never signals its dependents early, so this
+  // pre-pass cannot start while an earlier GEMV still reads the workspace.)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (w >= (int64_t)rows_pad * nkb) return;  // uniform per warp
@@ -234,6 +238,9 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
   // ---- which tokens / matrix ----
   int expert = 0, row_base = 0, count = p.M;
   if (GROUPED) {
+    // the expert offsets come from the routing kernels: wait for the pre-pass
+    // (which itself waited for them) before reading
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // Find the blockIdx.y-th expert with a non-empty row range (every warp does
     // the same scan, so the result is uniform).
     const int want = (int)blockIdx.y;

@@ -17,19 +17,17 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
   return va > vb || (va == vb && ia < ib);
 }
 
-// Routing: one warp per token. Iterated arg-max over the E logits (each lane
-// holds E/32 of them), softmax over the selected logits in fp32. Each CTA
-// also writes the expert histogram of its tile of tokens to counts[cta][E].
-__global__ void __launch_bounds__(32 * kRouteWarps)
-route_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* __restrict__ ids,
-             float* __restrict__ wts, int32_t* __restrict__ counts) {
-  __shared__ int hist[kMaxE];
+// Routing of one tile of kRouteTokPerCta tokens: one warp per token. Iterated
+// arg-max over the E logits (each lane holds E/32 of them), softmax over the
+// selected logits in fp32. `hist` (shared, E entries, zeroed by the caller)
+// receives the tile's expert histogram.
+__device__ __forceinline__ void route_tile(const float* __restrict__ logits, int M, int E, int topk,
+                                           int32_t* __restrict__ ids, float* __restrict__ wts, int* hist,
+                                           int tile) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-  __syncthreads();
   const int per_lane = (E + 31) / 32;  // <= 32
   for (int tt = 0; tt < kRouteTokPerWarp; ++tt) {
-    const int tok = blockIdx.x * kRouteTokPerCta + warp * kRouteTokPerWarp + tt;
+    const int tok = tile * kRouteTokPerCta + warp * kRouteTokPerWarp + tt;
     if (tok >= M) break;  // uniform per warp
     const float* row = logits + (int64_t)tok * E;
     float v[32];
@@ -75,33 +73,35 @@ route_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* 
       atomicAdd(&hist[id], 1);
     }
   }
+}
+
+// Routing of any number of tokens: CTA b routes token tile b and writes its
+// expert histogram to counts[b][E]. The logits may come from the previous
+// kernel (programmatic dependent launch: wait first, then let the permutation
+// kernel launch).
+__global__ void __launch_bounds__(32 * kRouteWarps)
+route_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* __restrict__ ids,
+             float* __restrict__ wts, int32_t* __restrict__ counts) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ int hist[kMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  route_tile(logits, M, E, topk, ids, wts, hist, blockIdx.x);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)blockIdx.x * E + e] = hist[e];
 }
 
-// Permutation: CTA b places the (token, slot) pairs of its token tile. Its
-// base position for expert e is offsets[e] + (rows of e in tiles < b); inside
-// the tile the pairs are placed in flat-index order (stable sort by expert).
-__global__ void __launch_bounds__(256)
-permute_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ counts, int M, int E,
-               int topk, int ntiles, int32_t* __restrict__ expert_offsets, int32_t* __restrict__ perm,
-               int32_t* __restrict__ inv_perm, int32_t* __restrict__ row_token) {
-  __shared__ int base[kMaxE];
-  __shared__ int total[kMaxE];
-  __shared__ int warp_sums[32];
-  const int b = blockIdx.x;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int before = 0, all = 0;
-    for (int bb = 0; bb < ntiles; ++bb) {
-      const int c = counts[(int64_t)bb * E + e];
-      all += c;
-      if (bb < b) before += c;
-    }
-    total[e] = all;
-    base[e] = before;
-  }
-  __syncthreads();
-  // exclusive scan of total[] over experts (E <= 1024): thread i owns a run of experts
+// Exclusive scan of the per-expert totals (E <= 1024, 256 threads): expert e's
+// rows start at the running sum of the totals before it. base[e] (holding this
+// tile's offset inside expert e) gets that start added; the CTA with
+// `write_offsets` stores expert_offsets[0..E]. Then warp 0 places the tile's
+// (token, slot) pairs f in [f0, f1) in flat-index order (stable sort by expert).
+__device__ __forceinline__ void scan_and_place(int* base, const int* total, int* warp_sums, int E,
+                                               bool write_offsets, int32_t* __restrict__ expert_offsets,
+                                               const int32_t* ids, int f0, int f1, int topk,
+                                               int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+                                               int32_t* __restrict__ row_token) {
   {
     const int per = (E + blockDim.x - 1) / blockDim.x;
     const int e0 = threadIdx.x * per;
@@ -129,22 +129,20 @@ permute_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ coun
     int excl = incl - run + (warp > 0 ? warp_sums[warp - 1] : 0);
     for (int e = e0; e < e0 + per && e < E; ++e) {
       const int tot = total[e];
-      if (b == 0) expert_offsets[e] = excl;
+      if (write_offsets) expert_offsets[e] = excl;
       base[e] += excl;
       excl += tot;
     }
-    if (b == 0 && threadIdx.x == blockDim.x - 1) expert_offsets[E] = excl;  // grand total
+    if (write_offsets && threadIdx.x == blockDim.x - 1) expert_offsets[E] = excl;  // grand total
   }
   __syncthreads();
   // stable placement by warp 0, 32 pairs at a time in flat-index order
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    const int f0 = b * kRouteTokPerCta * topk;
-    const int f1 = min(M, (b + 1) * kRouteTokPerCta) * topk;
     for (int fs = f0; fs < f1; fs += 32) {
       const int f = fs + lane;
       const bool act = f < f1;
-      const int e = act ? ids[f] : -1 - lane;
+      const int e = act ? __ldcg(ids + f) : -1 - lane;  // L2: ids may be this kernel's own stores
       const bool ok = !act || (e >= 0 && e < E);
       if (!ok) latch_status(Q4K_ERR_DEVICE_BOUNDS);
       const unsigned peers = __match_any_sync(0xffffffffu, e);
@@ -162,10 +160,61 @@ permute_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ coun
   }
 }
 
+// Permutation: CTA b places the (token, slot) pairs of its token tile. Its
+// base position for expert e is offsets[e] + (rows of e in tiles < b).
+__global__ void __launch_bounds__(256)
+permute_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ counts, int M, int E,
+               int topk, int ntiles, int32_t* __restrict__ expert_offsets, int32_t* __restrict__ perm,
+               int32_t* __restrict__ inv_perm, int32_t* __restrict__ row_token) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // ids and counts come from route_kernel
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ int base[kMaxE];
+  __shared__ int total[kMaxE];
+  __shared__ int warp_sums[32];
+  const int b = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int before = 0, all = 0;
+    for (int bb = 0; bb < ntiles; ++bb) {
+      const int c = counts[(int64_t)bb * E + e];
+      all += c;
+      if (bb < b) before += c;
+    }
+    total[e] = all;
+    base[e] = before;
+  }
+  __syncthreads();
+  scan_and_place(base, total, warp_sums, E, b == 0, expert_offsets, ids, b * kRouteTokPerCta * topk,
+                 min(M, (b + 1) * kRouteTokPerCta) * topk, topk, perm, inv_perm, row_token);
+}
+
+// Routing and permutation of at most kRouteTokPerCta tokens in one CTA (one
+// launch instead of two; no histogram leaves shared memory).
+__global__ void __launch_bounds__(256)
+route_permute_one_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* __restrict__ ids,
+                         float* __restrict__ wts, int32_t* __restrict__ expert_offsets,
+                         int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+                         int32_t* __restrict__ row_token) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ int base[kMaxE];
+  __shared__ int total[kMaxE];
+  __shared__ int warp_sums[32];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    total[e] = 0;
+    base[e] = 0;
+  }
+  __syncthreads();
+  route_tile(logits, M, E, topk, ids, wts, total, 0);
+  __syncthreads();  // also orders this CTA's id stores before the placement reads them
+  scan_and_place(base, total, warp_sums, E, true, expert_offsets, ids, 0, M * topk, topk, perm, inv_perm,
+                 row_token);
+}
+
 // y[t][h] = sum_j w[t][j] * O[inv_perm[t*topk + j]][h], j in increasing order.
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ O, const int32_t* __restrict__ inv_perm,
                const float* __restrict__ w, int M, int topk, int H, float* __restrict__ Y) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // O comes from the expert GEMV
   const int t = blockIdx.y;
   const int h4 = blockIdx.x * blockDim.x + threadIdx.x;  // index of a float4
   if (h4 * 4 >= H) return;

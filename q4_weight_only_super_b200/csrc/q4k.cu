@@ -48,6 +48,23 @@ q4k_status launch_status(cudaError_t e) {
   return Q4K_ERR_LAUNCH;
 }
 
+// Launch `k` as a programmatic dependent of the previous kernel in `s`: it may
+// start while that kernel finishes; every such kernel here executes
+// griddepcontrol.wait before it reads anything the previous kernel writes.
+template <typename... KArgs, typename... Args>
+q4k_status launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return launch_status(cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...));
+}
+
 // ---------------------------------------------------------------- GEMV ----
 
 struct GemvCfg {
@@ -60,8 +77,8 @@ struct GemvCfg {
 // split -- and with it the summation order -- does not depend on the class.
 constexpr size_t kGemvTwoPerSm = 233472 / 2 - 1024;
 constexpr int kGemvStages[3][2] = {{4, 6}, {4, 2}, {3, 2}};  // mt = 1, 2, 4
-static_assert(GemvSmem<1, 8, 1>::total(kGemvStages[0][0], kGemvStages[0][1]) <= kGemvTwoPerSm, "mt 1");
-static_assert(GemvSmem<2, 8, 1>::total(kGemvStages[1][0], kGemvStages[1][1]) <= kGemvTwoPerSm, "mt 2");
+static_assert(GemvSmem<1, 4, 2>::total(kGemvStages[0][0], kGemvStages[0][1]) <= kGemvTwoPerSm, "mt 1");
+static_assert(GemvSmem<2, 4, 2>::total(kGemvStages[1][0], kGemvStages[1][1]) <= kGemvTwoPerSm, "mt 2");
 static_assert(GemvSmem<4, 4, 2>::total(kGemvStages[2][0], kGemvStages[2][1]) <= kGemvTwoPerSm, "mt 4");
 
 // fit[d][ks]: clusters of ks GEMV CTAs that can be resident at once on device d
@@ -74,12 +91,12 @@ q4k_status gemv_cluster_fit(int ks, int* fit) {
   if (dev < 0 || dev >= kMaxDevices || ks < 1 || ks > 8) return Q4K_ERR_CUDA;
   int v = g_gemv_fit[dev][ks].load();
   if (v <= 0) {
-    auto* k = gemv_kernel<1, 8, 1, false, false>;
-    const size_t smem = GemvSmem<1, 8, 1>::total(kGemvStages[0][0], kGemvStages[0][1]);
+    auto* k = gemv_kernel<1, 4, 2, false, false>;
+    const size_t smem = GemvSmem<1, 4, 2>::total(kGemvStages[0][0], kGemvStages[0][1]);
     if (ensure_smem(k, smem, g_gemv_fit_smem_set) != cudaSuccess) return launch_status(cudaErrorUnknown);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(ks * 64), 1, 1);
-    cfg.blockDim = dim3(32 * (8 + 2), 1, 1);
+    cfg.blockDim = dim3(32 * (4 + 2), 1, 1);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -108,11 +125,11 @@ q4k_status pick_gemv(int tokens, int rows_out, int nkb, int groups, GemvCfg* out
   GemvCfg c;
   c.mt = tokens <= 8 ? 1 : (tokens <= 16 ? 2 : 4);
   const int cls = c.mt == 1 ? 0 : (c.mt == 2 ? 1 : 2);
-  // 128 weight rows per CTA: 8 warps x one 16-row tile up to 16 tokens (more warps
-  // to hide latency), 4 warps x two tiles at 32 tokens (each activation fragment
-  // feeds two MMAs)
-  c.tiles = c.mt == 4 ? 2 : 1;
-  c.warps = c.mt == 4 ? 4 : 8;
+  // 128 weight rows per CTA: 4 consumer warps x two 16-row tiles, so each
+  // activation fragment, barrier wait and min-term operand serves 32 rows
+  // (measured 2-6% faster than 8 warps x one tile at 1..16 tokens)
+  c.tiles = 2;
+  c.warps = 4;
   c.wstages = kGemvStages[cls][0];
   c.xstages = kGemvStages[cls][1];
   const long clusters = (long)((rows_out + 128 - 1) / 128) * groups;
@@ -167,13 +184,12 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
   p.xprep = static_cast<const uint8_t*>(ws);
   const int total_rows = (int)(GROUPED ? (int64_t)p.E * p.N : p.N);
   const int64_t recs = (int64_t)p.rows_pad * p.nkb;
-  gemv_prep_kernel<<<(unsigned)((recs + 7) / 8), 256, 0, s>>>(X, gather, rows, p.rows_pad, K, p.nkb,
-                                                               static_cast<uint8_t*>(ws));
-  const q4k_status st = launch_status(cudaGetLastError());
+  const q4k_status st = launch_pdl(gemv_prep_kernel, dim3((unsigned)((recs + 7) / 8)), dim3(256), s, X, gather,
+                                   rows, p.rows_pad, K, p.nkb, static_cast<uint8_t*>(ws));
   if (st != Q4K_OK) return st;
   const int tiles = (rows_out + 128 - 1) / 128;
-  if (c.mt == 1) return launch_gemv_t<1, 8, 1, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
-  if (c.mt == 2) return launch_gemv_t<2, 8, 1, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
+  if (c.mt == 1) return launch_gemv_t<1, 4, 2, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
+  if (c.mt == 2) return launch_gemv_t<2, 4, 2, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
   return launch_gemv_t<4, 4, 2, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
 }
 
@@ -316,13 +332,15 @@ q4k_status moe_route_permute(const float* logits, int M, int E, int topk, int32_
     return Q4K_ERR_ALIGN;
   if (ws_bytes < q4k_workspace_bytes(Q4K_OP_ROUTE, M, 0, 0, E, topk)) return Q4K_ERR_WORKSPACE;
   const int tiles = (M + kRouteTokPerCta - 1) / kRouteTokPerCta;
+  if (tiles == 1)  // one CTA routes and places everything: one launch, no histogram in ws
+    return launch_pdl(route_permute_one_kernel, dim3(1), dim3(32 * kRouteWarps), s, logits, M, E, topk,
+                      topk_ids, topk_w, expert_offsets, perm, inv_perm, row_token);
   int32_t* counts = static_cast<int32_t*>(ws);
-  route_kernel<<<tiles, 32 * kRouteWarps, 0, s>>>(logits, M, E, topk, topk_ids, topk_w, counts);
-  q4k_status st = launch_status(cudaGetLastError());
+  const q4k_status st = launch_pdl(route_kernel, dim3(tiles), dim3(32 * kRouteWarps), s, logits, M, E, topk,
+                                   topk_ids, topk_w, counts);
   if (st != Q4K_OK) return st;
-  permute_kernel<<<tiles, 256, 0, s>>>(topk_ids, counts, M, E, topk, tiles, expert_offsets, perm,
-                                       inv_perm, row_token);
-  return launch_status(cudaGetLastError());
+  return launch_pdl(permute_kernel, dim3(tiles), dim3(256), s, topk_ids, counts, M, E, topk, tiles,
+                    expert_offsets, perm, inv_perm, row_token);
 }
 
 // The no-allocation variant: same checks and kernels as moe_route_permute, with
@@ -421,9 +439,8 @@ q4k_status moe_combine(const float* O, const int32_t* inv_perm, const float* top
   if (H % 4 || M > 65535 || topk > kMaxTopk) return Q4K_ERR_UNSUPPORTED;
   const int n4 = H / 4;
   dim3 grid((n4 + 255) / 256, M);
-  combine_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(O, inv_perm, topk_w, M, topk,
-                                                                       H, Y);
-  return launch_status(cudaGetLastError());
+  return launch_pdl(combine_kernel, grid, dim3(256), static_cast<cudaStream_t>(stream), O, inv_perm, topk_w, M,
+                    topk, H, Y);
 }
 
 q4k_status q4k_last_device_status(void* stream) {

@@ -48,7 +48,11 @@ constexpr uint32_t kBTileBytes = kGemmBN * 128;       // 32 KB per K step
 constexpr uint32_t kWRawPart = kGemmBN * 16;          // 4 KB: one 16-byte column per row
 constexpr uint32_t kWRawBytes = 3 * kWRawPart;        // header, quants 0-15, quants 16-31
 constexpr uint32_t kSmemA = 0;
+// epilogue staging: per epilogue warp 32 rows x kEpiPitch words, inside the
+// activation stages (free once the last MMA has completed)
+constexpr int kEpiPitch = 36;
 constexpr uint32_t kSmemB = kSmemA + kStagesAW * kATileBytes;
+static_assert(kDqWarps * 32 * kEpiPitch * 4 <= kStagesAW * kATileBytes, "epilogue staging fits the A stages");
 constexpr uint32_t kSmemW = kSmemB + kStagesB * kBTileBytes;
 constexpr uint32_t kSmemBar = kSmemW + kStagesAW * kWRawBytes;
 constexpr uint32_t kSmemTotal = kSmemBar + 256;
@@ -465,48 +469,64 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       if (ok && __all_sync(0xffffffffu, mbar_wait(bar_tmem_full, 0, abort_flag))) {
         tc_fence_after();
         const int q = warp & 3, hm = (warp - 2) >> 2;
-        const int ml = hm * 128 + q * 32 + lane;  // row within the 256-row tile
-        const int mrow = m0 + ml;
-        const bool in = GROUPED ? (mrow < count) : (mrow < p.M);
+        const int mbase = m0 + hm * 128 + q * 32;  // first of this warp's 32 token rows
+        const int limit = GROUPED ? count : p.M;
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(hm * 256);
+        // Coalesced stores through a per-warp staging tile (the activation stages are
+        // free once the last MMA has completed): tcgen05.ld gives each lane 32 columns of
+        // its own row; the tile is written back so that every store instruction covers
+        // whole 64- or 128-byte segments of four or eight rows.
+        uint32_t* stg = reinterpret_cast<uint32_t*>(smem + kSmemA) + (warp - 2) * (32 * kEpiPitch);
         if (SWIGLU) {
           const int half = p.N / 2;
-          uint16_t* out = static_cast<uint16_t*>(p.Y) + (int64_t)(row_base + mrow) * half +
-                          n_tile * (kGemmBN / 2);
+          uint16_t* out = static_cast<uint16_t*>(p.Y) + (int64_t)row_base * half + n_tile * (kGemmBN / 2);
 #pragma unroll 1
           for (int cb = 0; cb < 4; ++cb) {
             uint32_t g[32], u[32];
             tmem_ld32(tbase + cb * 32, g);
             tmem_ld32(tbase + 128 + cb * 32, u);
-            if (in) {
 #pragma unroll
-              for (int i = 0; i < 32; i += 8) {
-                uint4 o;
-                uint32_t* op = &o.x;
+            for (int i = 0; i < 32; i += 8) {
+              uint4 o;
+              uint32_t* op = &o.x;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float g0 = __uint_as_float(g[i + 2 * e]), g1 = __uint_as_float(g[i + 2 * e + 1]);
-                  const float u0 = __uint_as_float(u[i + 2 * e]), u1 = __uint_as_float(u[i + 2 * e + 1]);
-                  op[e] = pack_bf16x2(silu_mul(g0, u0), silu_mul(g1, u1));
-                }
-                *reinterpret_cast<uint4*>(out + cb * 32 + i) = o;
+              for (int e = 0; e < 4; ++e) {
+                const float g0 = __uint_as_float(g[i + 2 * e]), g1 = __uint_as_float(g[i + 2 * e + 1]);
+                const float u0 = __uint_as_float(u[i + 2 * e]), u1 = __uint_as_float(u[i + 2 * e + 1]);
+                op[e] = pack_bf16x2(silu_mul(g0, u0), silu_mul(g1, u1));
               }
+              *reinterpret_cast<uint4*>(stg + lane * kEpiPitch + i / 2) = o;
             }
+            __syncwarp();
+            // 32 rows x 64 bytes: each instruction stores eight rows (four lanes per row)
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int r = it * 8 + (lane >> 2), c = lane & 3;
+              if (mbase + r < limit)
+                *reinterpret_cast<uint4*>(out + (int64_t)(mbase + r) * half + cb * 32 + c * 8) =
+                    *reinterpret_cast<const uint4*>(stg + r * kEpiPitch + c * 4);
+            }
+            __syncwarp();
           }
         } else {
-          float* out = static_cast<float*>(p.Y) + (int64_t)((GROUPED ? row_base : 0) + mrow) * p.N +
-                       n_tile * kGemmBN;
+          float* out = static_cast<float*>(p.Y) + (int64_t)(GROUPED ? row_base : 0) * p.N + n_tile * kGemmBN;
 #pragma unroll 1
           for (int cb = 0; cb < 8; ++cb) {
             uint32_t v[32];
             tmem_ld32(tbase + cb * 32, v);
-            if (in) {
 #pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(out + cb * 32 + i) =
-                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<uint4*>(stg + lane * kEpiPitch + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            __syncwarp();
+            // 32 rows x 128 bytes: each instruction stores four rows (eight lanes per row)
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int r = it * 4 + (lane >> 3), c = lane & 7;
+              if (mbase + r < limit)
+                *reinterpret_cast<float4*>(out + (int64_t)(mbase + r) * p.N + cb * 32 + c * 4) =
+                    *reinterpret_cast<const float4*>(stg + r * kEpiPitch + c * 4);
             }
+            __syncwarp();
           }
         }
       }

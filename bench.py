@@ -250,18 +250,17 @@ def moe_buffers(torch, q, d, M, dims, topk=8):
     return bufs[M]
 
 
-def moe_layer_gpu(q, tm, key, d, M, dims, topk=8, staged=True):
-    """One MoE layer (four launches). staged: each stage timed on its own after a
-    flush (the breakdown); else the four launches timed together (the layer time)."""
+def moe_layer_calls(q, d, M, dims, topk=8, stage=None):
+    """Issue one MoE layer on the current stream: routing + permutation, gate_up
+    grouped GEMV with SwiGLU, down grouped GEMV, combine. `stage(name, fn)` wraps
+    each call (timing); None runs them plainly (also under CUDA-graph capture)."""
     import torch
     E, H, F = dims
     rows = M * topk
     b = moe_buffers(torch, q, d, M, dims, topk)
     logits, X = d["logits"][:M], d["X"][:M]
     ws = d.get("ws") if M <= 32 else None
-    stage = (lambda k, fn: tm.run(key + ":" + k, fn)) if staged else (lambda k, fn: fn())
-    if not staged:
-        s = tm.begin()
+    stage = stage or (lambda k, fn: fn())
     r = stage("route", lambda: q.moe_route_permute(logits, topk, out=b["route"], ws=b["route_ws"]))
     h = stage("gate_up", lambda: q.moe_q4k_grouped(d["W_gate_up"], E, 2 * F, H, X, r["expert_offsets"],
                                                   rows, M, q.ACT_SWIGLU, row_gather=r["row_token"],
@@ -269,9 +268,35 @@ def moe_layer_gpu(q, tm, key, d, M, dims, topk=8, staged=True):
     o = stage("down", lambda: q.moe_q4k_grouped(d["W_down"], E, H, F, h, r["expert_offsets"], rows, M,
                                                q.ACT_NONE, out=b["o"], ws=ws))
     y = stage("combine", lambda: q.moe_combine(o, r["inv_perm"], r["topk_w"], M, topk, H, Y=b["y"]))
-    if not staged:
-        tm.end(key + ":layer", s)
     return y, r
+
+
+def moe_layer_gpu(q, tm, key, d, M, dims, topk=8, staged=True):
+    """One MoE layer. staged: each stage timed on its own after a flush (the
+    breakdown); else the whole layer timed as issued from the host (the layer time)."""
+    if staged:
+        return moe_layer_calls(q, d, M, dims, topk, stage=lambda k, fn: tm.run(key + ":" + k, fn))
+    s = tm.begin()
+    out = moe_layer_calls(q, d, M, dims, topk)
+    tm.end(key + ":layer", s)
+    return out
+
+
+def moe_layer_graph(torch, q, tm, key, d, M, dims, topk=8):
+    """The same layer captured once as a CUDA graph and replayed after a clean
+    flush: device time with no host launch gaps (the serving-loop form)."""
+    graphs = d.setdefault("graphs", {})
+    if M not in graphs:
+        moe_layer_calls(q, d, M, dims, topk)  # attributes and buffers set up outside the capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            moe_layer_calls(q, d, M, dims, topk)
+        torch.cuda.synchronize()
+        graphs[M] = g
+    s = tm.begin()
+    graphs[M].replay()
+    tm.end(key + ":graph", s)
 
 
 def run_step(q, tm, W):
@@ -291,12 +316,16 @@ def run_step(q, tm, W):
         tm.run_seq(f"gemm:M{M}", fns)
         launches += len(fns)
     W["moe_dec"]["ws"] = W["ws"]
+    import torch
     for staged in (True, False):
         for M in (1, 8, 32):
             moe_layer_gpu(q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"], staged=staged)
-            launches += 5  # route (histogram + permute), gate_up, down, combine
+            launches += 6  # routing+permutation, 2 x (activation pre-pass + grouped GEMV), combine
         moe_layer_gpu(q, tm, "moe_pre:M4096", W["moe_pre"], 4096, W["moe_dims"], staged=staged)
-        launches += 5
+        launches += 5  # routing, permutation, 2 grouped GEMMs, combine
+    for M in (1, 8, 32):
+        moe_layer_graph(torch, q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"])
+        launches += 6
     return launches
 
 
@@ -360,13 +389,16 @@ def summarize(tm, W, peaks):
         comp[f"{key}_M{M}_tokens_per_s"] = round(M / T[f"{key}:M{M}:layer"], 1)
         comp[f"{key}_M{M}_layer_us"] = round(T[f"{key}:M{M}:layer"] * 1e6, 2)
         comp[f"{key}_M{M}_stage_us"] = {s: round(x * 1e6, 2) for s, x in zip(("route", "gate_up", "down", "combine"), parts)}
+        if f"{key}:M{M}:graph" in T:
+            comp[f"{key}_M{M}_graph_us"] = round(T[f"{key}:M{M}:graph"] * 1e6, 2)
+            comp[f"{key}_M{M}_graph_tokens_per_s"] = round(M / T[f"{key}:M{M}:graph"], 1)
     gbps = gemv_bytes / gemv_time / 1e9
     # dominant kernel: the one with the most device time per step (single kernels
     # only: whole-layer timings are not kernels); GEMV/GEMM times are per launch,
     # so weigh them by their launches per step
     per_step = {}
     for k, v in T.items():
-        if k.endswith(":layer"):
+        if k.endswith((":layer", ":graph")):
             continue
         n = 1
         if k.startswith("gemv:"):

@@ -18,24 +18,26 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
 }
 
 // Routing of one tile of kRouteTokPerCta tokens: one warp per token. Iterated
-// arg-max over the E logits (each lane holds E/32 of them), softmax over the
-// selected logits in fp32. `hist` (shared, E entries, zeroed by the caller)
-// receives the tile's expert histogram.
+// arg-max over the E logits (each lane holds PL <= 32 of them, E <= 32*PL),
+// softmax over the selected logits in fp32. `hist` (shared, E entries, zeroed
+// by the caller) receives the tile's expert histogram; `sids` (shared, or
+// nullptr) a copy of the tile's ids, [token in tile][topk].
+template <int PL>
 __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int M, int E, int topk,
                                            int32_t* __restrict__ ids, float* __restrict__ wts, int* hist,
-                                           int tile) {
+                                           int* sids, int tile) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int per_lane = (E + 31) / 32;  // <= 32
   for (int tt = 0; tt < kRouteTokPerWarp; ++tt) {
-    const int tok = tile * kRouteTokPerCta + warp * kRouteTokPerWarp + tt;
+    const int tl = warp * kRouteTokPerWarp + tt;  // token within the tile
+    const int tok = tile * kRouteTokPerCta + tl;
     if (tok >= M) break;  // uniform per warp
     const float* row = logits + (int64_t)tok * E;
-    float v[32];
+    float v[PL];
     uint32_t taken = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < PL; ++i) {
       const int e = i * 32 + lane;
-      v[i] = (i < per_lane && e < E) ? row[e] : 0.f;
+      v[i] = e < E ? row[e] : 0.f;
     }
     float sel_v[kMaxTopk];
     int sel_i[kMaxTopk];
@@ -43,9 +45,9 @@ __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int
       float bv = -INFINITY;  // a lane with no candidate left never wins
       int bi = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < PL; ++i) {
         const int e = i * 32 + lane;
-        if (i < per_lane && e < E && !((taken >> i) & 1u) && ranks_before(v[i], e, bv, bi)) {
+        if (e < E && !((taken >> i) & 1u) && ranks_before(v[i], e, bv, bi)) {
           bv = v[i];
           bi = e;
         }
@@ -70,6 +72,7 @@ __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int
         if (k == lane) { num = expf(sel_v[k] - sel_v[0]); id = sel_i[k]; }
       ids[(int64_t)tok * topk + lane] = id;
       wts[(int64_t)tok * topk + lane] = num / den;
+      if (sids) sids[tl * topk + lane] = id;
       atomicAdd(&hist[id], 1);
     }
   }
@@ -79,6 +82,7 @@ __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int
 // expert histogram to counts[b][E]. The logits may come from the previous
 // kernel (programmatic dependent launch: wait first, then let the permutation
 // kernel launch).
+template <int PL>
 __global__ void __launch_bounds__(32 * kRouteWarps)
 route_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* __restrict__ ids,
              float* __restrict__ wts, int32_t* __restrict__ counts) {
@@ -87,7 +91,7 @@ route_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* 
   __shared__ int hist[kMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  route_tile(logits, M, E, topk, ids, wts, hist, blockIdx.x);
+  route_tile<PL>(logits, M, E, topk, ids, wts, hist, nullptr, blockIdx.x);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)blockIdx.x * E + e] = hist[e];
 }
@@ -96,10 +100,11 @@ route_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* 
 // rows start at the running sum of the totals before it. base[e] (holding this
 // tile's offset inside expert e) gets that start added; the CTA with
 // `write_offsets` stores expert_offsets[0..E]. Then warp 0 places the tile's
-// (token, slot) pairs f in [f0, f1) in flat-index order (stable sort by expert).
+// (token, slot) pairs f in [f0, f1) in flat-index order (stable sort by expert),
+// their experts read from `sids` (shared, indexed f - f0) when given, else from ids.
 __device__ __forceinline__ void scan_and_place(int* base, const int* total, int* warp_sums, int E,
                                                bool write_offsets, int32_t* __restrict__ expert_offsets,
-                                               const int32_t* ids, int f0, int f1, int topk,
+                                               const int32_t* ids, const int* sids, int f0, int f1, int topk,
                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
                                                int32_t* __restrict__ row_token) {
   {
@@ -142,7 +147,8 @@ __device__ __forceinline__ void scan_and_place(int* base, const int* total, int*
     for (int fs = f0; fs < f1; fs += 32) {
       const int f = fs + lane;
       const bool act = f < f1;
-      const int e = act ? __ldcg(ids + f) : -1 - lane;  // L2: ids may be this kernel's own stores
+      // (from L2 when global: they may be this kernel's own stores)
+      const int e = act ? (sids ? sids[f - f0] : __ldcg(ids + f)) : -1 - lane;
       const bool ok = !act || (e >= 0 && e < E);
       if (!ok) latch_status(Q4K_ERR_DEVICE_BOUNDS);
       const unsigned peers = __match_any_sync(0xffffffffu, e);
@@ -183,12 +189,13 @@ permute_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ coun
     base[e] = before;
   }
   __syncthreads();
-  scan_and_place(base, total, warp_sums, E, b == 0, expert_offsets, ids, b * kRouteTokPerCta * topk,
+  scan_and_place(base, total, warp_sums, E, b == 0, expert_offsets, ids, nullptr, b * kRouteTokPerCta * topk,
                  min(M, (b + 1) * kRouteTokPerCta) * topk, topk, perm, inv_perm, row_token);
 }
 
 // Routing and permutation of at most kRouteTokPerCta tokens in one CTA (one
-// launch instead of two; no histogram leaves shared memory).
+// launch instead of two; the histogram and the ids stay in shared memory).
+template <int PL>
 __global__ void __launch_bounds__(256)
 route_permute_one_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* __restrict__ ids,
                          float* __restrict__ wts, int32_t* __restrict__ expert_offsets,
@@ -199,14 +206,15 @@ route_permute_one_kernel(const float* __restrict__ logits, int M, int E, int top
   __shared__ int base[kMaxE];
   __shared__ int total[kMaxE];
   __shared__ int warp_sums[32];
+  __shared__ int sids[kRouteTokPerCta * kMaxTopk];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     total[e] = 0;
     base[e] = 0;
   }
   __syncthreads();
-  route_tile(logits, M, E, topk, ids, wts, total, 0);
-  __syncthreads();  // also orders this CTA's id stores before the placement reads them
-  scan_and_place(base, total, warp_sums, E, true, expert_offsets, ids, 0, M * topk, topk, perm, inv_perm,
+  route_tile<PL>(logits, M, E, topk, ids, wts, total, sids, 0);
+  __syncthreads();
+  scan_and_place(base, total, warp_sums, E, true, expert_offsets, ids, sids, 0, M * topk, topk, perm, inv_perm,
                  row_token);
 }
 

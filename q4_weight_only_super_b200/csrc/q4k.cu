@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 #include "dequant.cuh"
@@ -193,6 +194,18 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
   return launch_gemv_t<4, 4, 2, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
 }
 
+// Routing kernels keep each lane's share of a logit row in registers: pick the
+// instantiation whose per-lane slot count PL covers E (E <= 32 * PL).
+template <typename F>
+q4k_status route_pl_dispatch(int E, F&& f) {
+  if (E <= 32) return f(std::integral_constant<int, 1>());
+  if (E <= 64) return f(std::integral_constant<int, 2>());
+  if (E <= 128) return f(std::integral_constant<int, 4>());
+  if (E <= 256) return f(std::integral_constant<int, 8>());
+  if (E <= 512) return f(std::integral_constant<int, 16>());
+  return f(std::integral_constant<int, 32>());
+}
+
 // Fixed scratch of moe_route_permute_noalloc: one array per device that loads
 // this library, alive until process exit. Host code must not pass the symbol
 // itself to a kernel (on the host it names a host-side stand-in, not device
@@ -333,11 +346,15 @@ q4k_status moe_route_permute(const float* logits, int M, int E, int topk, int32_
   if (ws_bytes < q4k_workspace_bytes(Q4K_OP_ROUTE, M, 0, 0, E, topk)) return Q4K_ERR_WORKSPACE;
   const int tiles = (M + kRouteTokPerCta - 1) / kRouteTokPerCta;
   if (tiles == 1)  // one CTA routes and places everything: one launch, no histogram in ws
-    return launch_pdl(route_permute_one_kernel, dim3(1), dim3(32 * kRouteWarps), s, logits, M, E, topk,
-                      topk_ids, topk_w, expert_offsets, perm, inv_perm, row_token);
+    return route_pl_dispatch(E, [&](auto pl) {
+      return launch_pdl(route_permute_one_kernel<decltype(pl)::value>, dim3(1), dim3(32 * kRouteWarps), s, logits,
+                        M, E, topk, topk_ids, topk_w, expert_offsets, perm, inv_perm, row_token);
+    });
   int32_t* counts = static_cast<int32_t*>(ws);
-  const q4k_status st = launch_pdl(route_kernel, dim3(tiles), dim3(32 * kRouteWarps), s, logits, M, E, topk,
-                                   topk_ids, topk_w, counts);
+  const q4k_status st = route_pl_dispatch(E, [&](auto pl) {
+    return launch_pdl(route_kernel<decltype(pl)::value>, dim3(tiles), dim3(32 * kRouteWarps), s, logits, M, E,
+                      topk, topk_ids, topk_w, counts);
+  });
   if (st != Q4K_OK) return st;
   return launch_pdl(permute_kernel, dim3(tiles), dim3(256), s, topk_ids, counts, M, E, topk, tiles,
                     expert_offsets, perm, inv_perm, row_token);
@@ -369,8 +386,11 @@ q4k_status moe_route_permute_noalloc(const float* logits, int M, int E, int topk
   if (sst != Q4K_OK) return sst;
   // route_kernel writes every histogram entry permute_kernel reads, so the
   // array's previous contents never matter and nothing is cleared.
-  route_kernel<<<tiles, 32 * kRouteWarps, 0, s>>>(logits, M, E, topk, topk_ids, topk_w, counts);
-  q4k_status st = launch_status(cudaGetLastError());
+  q4k_status st = route_pl_dispatch(E, [&](auto pl) {
+    route_kernel<decltype(pl)::value><<<tiles, 32 * kRouteWarps, 0, s>>>(logits, M, E, topk, topk_ids, topk_w,
+                                                                          counts);
+    return launch_status(cudaGetLastError());
+  });
   if (st != Q4K_OK) return st;
   permute_kernel<<<tiles, 256, 0, s>>>(topk_ids, counts, M, E, topk, tiles, expert_offsets, perm,
                                        inv_perm, row_token);

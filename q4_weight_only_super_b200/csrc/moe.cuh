@@ -17,18 +17,34 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
   return va > vb || (va == vb && ia < ib);
 }
 
-// Routing of one tile of kRouteTokPerCta tokens: one warp per token. Iterated
-// arg-max over the E logits (each lane holds PL <= 32 of them, E <= 32*PL),
-// softmax over the selected logits in fp32. `hist` (shared, E entries, zeroed
-// by the caller) receives the tile's expert histogram; `sids` (shared, or
-// nullptr) a copy of the tile's ids, [token in tile][topk].
-template <int PL>
+// Unsigned key with the order of the fp32 value (finite values; -0 and +0
+// equal, as in the float comparison).
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Routing of one tile of kRouteTokPerCta tokens: a warp per token, tokens
+// dealt round-robin over the NW warps of the CTA. Iterated arg-max over the E logits (each
+// lane holds PL <= 32 of them, E <= 32*PL): per round each lane takes its best
+// remaining (logit, id), the warp takes the largest logit (a reduce-max over
+// order keys) and, among lanes holding it, the smallest id (a reduce-min) --
+// the order "higher logit first, equal logits to the lower id". Softmax over
+// the selected logits in fp32. `hist` (shared, E entries, zeroed by the caller)
+// receives the tile's expert histogram; `sids` (shared, or nullptr) a copy of
+// the tile's ids [token in tile][topk]; `tmask` (shared, or nullptr) bit t of
+// entry e set when token t of the tile selected expert e.
+template <int PL, int NW>
 __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int M, int E, int topk,
                                            int32_t* __restrict__ ids, float* __restrict__ wts, int* hist,
-                                           int* sids, int tile) {
+                                           int* sids, unsigned* tmask, int tile) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int tt = 0; tt < kRouteTokPerWarp; ++tt) {
-    const int tl = warp * kRouteTokPerWarp + tt;  // token within the tile
+  static_assert(kRouteTokPerCta % NW == 0, "whole tokens per warp");
+  for (int tt = 0; tt < kRouteTokPerCta / NW; ++tt) {
+    const int tl = tt * NW + warp;  // token within the tile
     const int tok = tile * kRouteTokPerCta + tl;
     if (tok >= M) break;  // uniform per warp
     const float* row = logits + (int64_t)tok * E;
@@ -39,9 +55,13 @@ __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int
       const int e = i * 32 + lane;
       v[i] = e < E ? row[e] : 0.f;
     }
-    float sel_v[kMaxTopk];
+    float sel_v[kMaxTopk];  // fully unrolled below, so these stay in registers
     int sel_i[kMaxTopk];
-    for (int k = 0; k < topk; ++k) {
+#pragma unroll
+    for (int k = 0; k < kMaxTopk; ++k) {
+      sel_v[k] = 0.f;
+      sel_i[k] = 0;
+      if (k >= topk) continue;
       float bv = -INFINITY;  // a lane with no candidate left never wins
       int bi = 0x7fffffff;
 #pragma unroll
@@ -52,27 +72,28 @@ __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int
           bi = e;
         }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (ranks_before(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      sel_v[k] = bv;
-      sel_i[k] = bi;
+      const uint32_t key = bi == 0x7fffffff ? 0u : order_key(bv);
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+      const int wi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0x7fffffffu);
+      if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
+      sel_v[k] = key_value(kmax);
+      sel_i[k] = wi;
     }
     // softmax over the selected logits; sel_v[0] is the largest
     float den = 0.f;
-    for (int k = 0; k < topk; ++k) den += expf(sel_v[k] - sel_v[0]);
+#pragma unroll
+    for (int k = 0; k < kMaxTopk; ++k)
+      if (k < topk) den += expf(sel_v[k] - sel_v[0]);
     if (lane < topk) {
       float num = 0.f;
       int id = 0;
-      for (int k = 0; k < topk; ++k)
+#pragma unroll
+      for (int k = 0; k < kMaxTopk; ++k)
         if (k == lane) { num = expf(sel_v[k] - sel_v[0]); id = sel_i[k]; }
       ids[(int64_t)tok * topk + lane] = id;
       wts[(int64_t)tok * topk + lane] = num / den;
       if (sids) sids[tl * topk + lane] = id;
+      if (tmask) atomicOr(&tmask[id], 1u << tl);
       atomicAdd(&hist[id], 1);
     }
   }
@@ -91,7 +112,7 @@ route_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* 
   __shared__ int hist[kMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  route_tile<PL>(logits, M, E, topk, ids, wts, hist, nullptr, blockIdx.x);
+  route_tile<PL, kRouteWarps>(logits, M, E, topk, ids, wts, hist, nullptr, nullptr, blockIdx.x);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)blockIdx.x * E + e] = hist[e];
 }
@@ -194,28 +215,79 @@ permute_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ coun
 }
 
 // Routing and permutation of at most kRouteTokPerCta tokens in one CTA (one
-// launch instead of two; the histogram and the ids stay in shared memory).
+// launch instead of two; the histogram, the ids and the per-expert token masks
+// stay in shared memory). A token selects an expert at most once, so the rank
+// of pair f = t*topk + j among expert e's pairs in flat order is the number of
+// earlier tokens that selected e: the popcount of e's mask below bit t. Every
+// pair is placed by its own thread.
+constexpr int kRouteOneWarps = kRouteTokPerCta;  // one warp per token
+
 template <int PL>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(32 * kRouteOneWarps)
 route_permute_one_kernel(const float* __restrict__ logits, int M, int E, int topk, int32_t* __restrict__ ids,
                          float* __restrict__ wts, int32_t* __restrict__ expert_offsets,
                          int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
                          int32_t* __restrict__ row_token) {
+  static_assert(kRouteTokPerCta <= 32, "one mask bit per token of the tile");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ int base[kMaxE];
   __shared__ int total[kMaxE];
+  __shared__ int start[kMaxE];
+  __shared__ unsigned tmask[kMaxE];
   __shared__ int warp_sums[32];
   __shared__ int sids[kRouteTokPerCta * kMaxTopk];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     total[e] = 0;
-    base[e] = 0;
+    tmask[e] = 0u;
   }
   __syncthreads();
-  route_tile<PL>(logits, M, E, topk, ids, wts, total, sids, 0);
+  route_tile<PL, kRouteOneWarps>(logits, M, E, topk, ids, wts, total, sids, tmask, 0);
   __syncthreads();
-  scan_and_place(base, total, warp_sums, E, true, expert_offsets, ids, sids, 0, M * topk, topk, perm, inv_perm,
-                 row_token);
+  // exclusive scan of the per-expert totals -> expert_offsets and start[e]
+  {
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = threadIdx.x * per;
+    int run = 0;
+    for (int e = e0; e < e0 + per && e < E; ++e) run += total[e];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = run;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int nw = blockDim.x / 32;
+      int ws = lane < nw ? warp_sums[lane] : 0;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, ws, off);
+        if (lane >= off) ws += o;
+      }
+      if (lane < nw) warp_sums[lane] = ws;
+    }
+    __syncthreads();
+    int excl = incl - run + (warp > 0 ? warp_sums[warp - 1] : 0);
+    for (int e = e0; e < e0 + per && e < E; ++e) {
+      expert_offsets[e] = excl;
+      start[e] = excl;
+      excl += total[e];
+    }
+    if (threadIdx.x == blockDim.x - 1) expert_offsets[E] = excl;
+  }
+  __syncthreads();
+  for (int f = threadIdx.x; f < M * topk; f += blockDim.x) {
+    const int t = f / topk;
+    const int e = sids[f];
+    if (e < 0 || e >= E) {
+      latch_status(Q4K_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    const int pos = start[e] + __popc(tmask[e] & ((1u << t) - 1u));
+    perm[pos] = f;
+    inv_perm[f] = pos;
+    row_token[pos] = t;
+  }
 }
 
 // y[t][h] = sum_j w[t][j] * O[inv_perm[t*topk + j]][h], j in increasing order.

@@ -347,7 +347,7 @@ q4k_status moe_route_permute(const float* logits, int M, int E, int topk, int32_
   const int tiles = (M + kRouteTokPerCta - 1) / kRouteTokPerCta;
   if (tiles == 1)  // one CTA routes and places everything: one launch, no histogram in ws
     return route_pl_dispatch(E, [&](auto pl) {
-      return launch_pdl(route_permute_one_kernel<decltype(pl)::value>, dim3(1), dim3(32 * kRouteWarps), s, logits,
+      return launch_pdl(route_permute_one_kernel<decltype(pl)::value>, dim3(1), dim3(32 * kRouteOneWarps), s, logits,
                         M, E, topk, topk_ids, topk_w, expert_offsets, perm, inv_perm, row_token);
     });
   int32_t* counts = static_cast<int32_t*>(ws);

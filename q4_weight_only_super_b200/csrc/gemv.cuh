@@ -228,6 +228,8 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int SW = p.wstages, SX = p.xstages;
+  if (threadIdx.x == 32 * WARPS)  // the weight-TMA thread: fetch the descriptor while the rest sets up
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
 
   const int rank = (int)(blockIdx.x % (unsigned)p.ksplit);
   const int tile = (int)(blockIdx.x / (unsigned)p.ksplit);
@@ -242,20 +244,28 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     // (which itself waited for them) before reading
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // Find the blockIdx.y-th expert with a non-empty row range (every warp does
-    // the same scan, so the result is uniform).
+    // the same scan, so the result is uniform). The offsets of 128 experts are
+    // loaded at once: one memory latency instead of one per 32 experts.
     const int want = (int)blockIdx.y;
     int found = -1, seen = 0;
-    for (int e0 = 0; e0 < p.E && found < 0; e0 += 32) {
-      const int e = e0 + lane;
-      const bool ne = e < p.E && p.offsets[e + 1] > p.offsets[e];
-      const unsigned bal = __ballot_sync(0xffffffffu, ne);
-      const int n = __popc(bal);
-      if (want < seen + n) {
-        unsigned b = bal;
-        for (int i = 0; i < want - seen; ++i) b &= b - 1;
-        found = e0 + __ffs(b) - 1;
+    for (int e0 = 0; e0 < p.E && found < 0; e0 += 128) {
+      bool ne[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = e0 + 32 * i + lane;
+        ne[i] = e < p.E && __ldg(p.offsets + e + 1) > __ldg(p.offsets + e);
       }
-      seen += n;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const unsigned bal = __ballot_sync(0xffffffffu, ne[i]);
+        const int n = __popc(bal);
+        if (found < 0 && want < seen + n) {
+          unsigned b = bal;
+          for (int j = 0; j < want - seen; ++j) b &= b - 1;
+          found = e0 + 32 * i + __ffs(b) - 1;
+        }
+        seen += n;
+      }
     }
     if (found < 0) return;  // uniform over the cluster (depends on blockIdx.y only)
     expert = found;

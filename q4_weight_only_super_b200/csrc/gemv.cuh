@@ -335,15 +335,17 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     // ---------------- activation producer: bulk copies of prepared records ----------------
     if (lane == 0) {
       asm volatile("griddepcontrol.wait;" ::: "memory");  // the pre-pass has finished
+      // only the token groups that hold rows of this call (or expert) are copied
+      const uint32_t xbytes = (uint32_t)(((count + 7) / 8) * 8 * kXRec);
       int issued = 0;
       int s = 0;
       uint32_t ph = 0;
       for (int ks = 0; ks < nk; ++ks) {
         if (ks >= SX) mbar_wait(xempty(s), ph ^ 1u, abort_flag);
         if (*abort_flag) break;
-        mbar_arrive_expect_tx(xfull(s), (uint32_t)L::xstage);
+        mbar_arrive_expect_tx(xfull(s), xbytes);
         const uint8_t* src = p.xprep + ((int64_t)(kb0 + ks) * p.rows_pad + row_base) * kXRec;
-        bulk_copy_g2s(smem_u32(xring) + (uint32_t)(s * L::xstage), src, (uint32_t)L::xstage, xfull(s));
+        bulk_copy_g2s(smem_u32(xring) + (uint32_t)(s * L::xstage), src, xbytes, xfull(s));
         ++issued;
         if (++s == SX) {
           s = 0;
@@ -433,6 +435,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
             }
 #pragma unroll
             for (int f = 0; f < MT; ++f) {
+              if (GROUPED && 8 * f >= count) break;  // token groups past this expert's rows
               const uint4 bx = *reinterpret_cast<const uint4*>(xb + (8 * f + g) * kXRec + (j * 4 + t) * 16);
 #pragma unroll
               for (int tt = 0; tt < TILES; ++tt) {
@@ -459,6 +462,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         }
 #pragma unroll
         for (int f = 0; f < MT; ++f) {
+          if (GROUPED && 8 * f >= count) break;
           const uint8_t* rg = xb + (8 * f + g) * kXRec;
           const uint32_t bh = *reinterpret_cast<const uint32_t*>(rg + 512 + 4 * t);
           const uint32_t bl = *reinterpret_cast<const uint32_t*>(rg + 528 + 4 * t);

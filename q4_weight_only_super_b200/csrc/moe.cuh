@@ -291,8 +291,10 @@ route_permute_one_kernel(const float* __restrict__ logits, int M, int E, int top
 }
 
 // y[t][h] = sum_j w[t][j] * O[inv_perm[t*topk + j]][h], j in increasing order.
-// All of a token's row indices and weights are loaded first, then all its O
-// rows, then they are added in slot order: two memory latencies, not 2*topk.
+// Slots are taken eight at a time: their row indices and weights are loaded
+// first, then their O rows, then they are added in slot order (two memory
+// latencies per eight slots, at a register count that keeps the large-M case
+// bandwidth-bound).
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ O, const int32_t* __restrict__ inv_perm,
                const float* __restrict__ w, int M, int topk, int H, float* __restrict__ Y) {
@@ -301,35 +303,39 @@ combine_kernel(const float* __restrict__ O, const int32_t* __restrict__ inv_perm
   const int h4 = blockIdx.x * blockDim.x + threadIdx.x;  // index of a float4
   if (h4 * 4 >= H) return;
   const int rows = M * topk;
-  int r[kMaxTopk];
-  float wj[kMaxTopk];
-#pragma unroll
-  for (int j = 0; j < kMaxTopk; ++j) {
-    r[j] = -1;
-    wj[j] = 0.f;
-    if (j < topk) {
-      r[j] = __ldg(inv_perm + (int64_t)t * topk + j);
-      wj[j] = __ldg(w + (int64_t)t * topk + j);
-    }
-  }
-  float4 o[kMaxTopk];
-#pragma unroll
-  for (int j = 0; j < kMaxTopk; ++j) {
-    o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < topk && r[j] >= 0 && r[j] < rows) o[j] = *reinterpret_cast<const float4*>(O + (int64_t)r[j] * H + 4 * h4);
-  }
+  constexpr int B = 8;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = 0; j0 < topk; j0 += B) {
+    int r[B];
+    float wj[B];
 #pragma unroll
-  for (int j = 0; j < kMaxTopk; ++j) {
-    if (j >= topk) continue;
-    if (r[j] < 0 || r[j] >= rows) {
-      latch_status(Q4K_ERR_DEVICE_BOUNDS);
-      continue;
+    for (int j = 0; j < B; ++j) {
+      r[j] = -1;
+      wj[j] = 0.f;
+      if (j0 + j < topk) {
+        r[j] = __ldg(inv_perm + (int64_t)t * topk + j0 + j);
+        wj[j] = __ldg(w + (int64_t)t * topk + j0 + j);
+      }
     }
-    acc.x = fmaf(wj[j], o[j].x, acc.x);
-    acc.y = fmaf(wj[j], o[j].y, acc.y);
-    acc.z = fmaf(wj[j], o[j].z, acc.z);
-    acc.w = fmaf(wj[j], o[j].w, acc.w);
+    float4 o[B];
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + j < topk && r[j] >= 0 && r[j] < rows)
+        o[j] = *reinterpret_cast<const float4*>(O + (int64_t)r[j] * H + 4 * h4);
+    }
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      if (j0 + j >= topk) break;
+      if (r[j] < 0 || r[j] >= rows) {
+        latch_status(Q4K_ERR_DEVICE_BOUNDS);
+        continue;
+      }
+      acc.x = fmaf(wj[j], o[j].x, acc.x);
+      acc.y = fmaf(wj[j], o[j].y, acc.y);
+      acc.z = fmaf(wj[j], o[j].z, acc.z);
+      acc.w = fmaf(wj[j], o[j].w, acc.w);
+    }
   }
   *reinterpret_cast<float4*>(Y + (int64_t)t * H + 4 * h4) = acc;
 }

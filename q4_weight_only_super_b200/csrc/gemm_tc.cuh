@@ -42,7 +42,7 @@ constexpr int kGemmBK = 64;
 constexpr int kStagesAW = 3;
 constexpr int kStagesB = 2;
 constexpr int kDqWarps = 8;
-constexpr int kGatherWarps = 4;
+constexpr int kGatherWarps = 8;  // grouped: activation-row gather (4 were the bound, 8 measured 10% faster)
 constexpr uint32_t kATileBytes = kGemmBM * 128;       // 32 KB per K step
 constexpr uint32_t kBTileBytes = kGemmBN * 128;       // 32 KB per K step
 constexpr uint32_t kWRawPart = kGemmBN * 16;          // 4 KB: one 16-byte column per row
@@ -532,23 +532,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       }
     } else if (GROUPED) {
       // ---------------- activation rows: load, bf16 -> fp16, store swizzled ----------------
-      const int gt = (warp - 2 - kDqWarps) * 32 + lane;  // 0..127
+      constexpr int RS = kGatherWarps * 4;                // row stride: 8 lanes cover a 128-byte row
+      const int gt = (warp - 2 - kDqWarps) * 32 + lane;  // 0..32*kGatherWarps-1
       const int ch = gt & 7;                              // 16-byte chunk within the 128-byte row
-      const int r0 = gt >> 3;                             // rows r0, r0+16, ...
-      const uint16_t* src_row[kGemmBM / 16];
+      const int r0 = gt >> 3;                             // rows r0, r0+RS, ...
+      const uint16_t* src_row[kGemmBM / RS];
 #pragma unroll
-      for (int j = 0; j < kGemmBM / 16; ++j) {
-        const int mrow = m0 + r0 + 16 * j;
+      for (int j = 0; j < kGemmBM / RS; ++j) {
+        const int mrow = m0 + r0 + RS * j;
         src_row[j] = nullptr;
         if (mrow < count) {
           const int64_t sr = p.gather ? p.gather[row_base + mrow] : (row_base + mrow);
           src_row[j] = p.X + sr * p.K + ch * 8;
         }
       }
-      uint4 buf[kGemmBM / 16];
+      uint4 buf[kGemmBM / RS];
       auto load = [&](int ks) {
 #pragma unroll
-        for (int j = 0; j < kGemmBM / 16; ++j)
+        for (int j = 0; j < kGemmBM / RS; ++j)
           buf[j] = src_row[j] ? ldg_u4(src_row[j] + ks * kGemmBK) : make_uint4(0u, 0u, 0u, 0u);
       };
       uint32_t amax = 0;  // largest |bf16| bit pattern seen, per 16-bit half
@@ -560,7 +561,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
           break;
         uint8_t* a_dst = smem + kSmemA + s * kATileBytes;
 #pragma unroll
-        for (int j = 0; j < kGemmBM / 16; ++j) {
+        for (int j = 0; j < kGemmBM / RS; ++j) {
           const uint32_t w[4] = {buf[j].x, buf[j].y, buf[j].z, buf[j].w};
           uint4 o;
           uint32_t* op = &o.x;
@@ -569,7 +570,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             amax = __vmaxu2(amax, w[e] & 0x7FFF7FFFu);
             op[e] = pack_f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
           }
-          *reinterpret_cast<uint4*>(a_dst + sw128_offset(r0 + 16 * j, ch)) = o;
+          *reinterpret_cast<uint4*>(a_dst + sw128_offset(r0 + RS * j, ch)) = o;
         }
         fence_async_smem();
         __syncwarp();

@@ -159,7 +159,7 @@ q4k_status moe_route_permute_noalloc(const float* logits, int M, int E, int topk
  *   rows       total rows = off[E] (host value; must match the device array).
  *   max_rows_hint  upper bound on any single expert's row count (for a
  *              top-k layer over M tokens: M). <= 32 selects the GEMV-style
- *              decode kernel (same arithmetic as q4k_gemv);
+ *              decode kernel (the arithmetic of q4k_gemv);
  *              larger selects the tcgen05 grouped GEMM, whose operands are
  *              fp16: weights RN_fp16 of the fp32 dequant, activations
  *              converted from bf16 (|values| must stay below 65504, else

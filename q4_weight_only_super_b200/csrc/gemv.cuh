@@ -20,11 +20,19 @@
 //    dependent of the pre-pass, so its weight stream starts while the pre-pass
 //    runs and only the activation copies wait for it.
 //  * Consumer warps own 16 or 32 weight rows each (one or two 16-row MMA
-//    tiles; with two, every activation fragment feeds two MMAs). The A operand is fp16 q*sc, exact
-//    (q*sc <= 945): a nibble ORed into 0x6400 is 1024+q (low nibble) or
-//    1024+16q (high nibble), and one fp16x2 FMA with (sc or sc/16) and
-//    -1024*that removes the bias exactly. So the mma.sync m16n8k16 accumulator
-//    (fp32) runs over the whole super-block: C = sum_k sc*q*x'.
+//    tiles; with two, every activation fragment feeds two MMAs). The A operand
+//    takes one of two exact forms:
+//    - 1..16 tokens: the nibble field itself read as fp16 bits -- q * 2^-24 for
+//      a low nibble, 16q * 2^-24 for a high one, fp16 subnormals that the
+//      tensor core multiplies exactly -- one AND per two weights. A sub-block's
+//      two k-steps accumulate on their own (C_j, fp32) and the block sum is
+//      C = sum_j s_j * C_j with s_j = sc_j (sc_j/16 for high nibbles) as an
+//      exact fp32; 2^24 is folded into d.
+//    - 17..32 tokens: fp16 q*sc (<= 945, exact): a nibble ORed into 0x6400 is
+//      1024+q (low) or 1024+16q (high), and one fp16x2 FMA with (sc or sc/16)
+//      and -1024*that removes the bias, so the mma.sync m16n8k16 accumulator
+//      runs over the whole super-block (scaling per result would grow with the
+//      four token groups).
 //  * The min term, dmin * sum_j m_j * X_j over the eight sub-blocks, is one
 //    more MMA per tile: A = m_j (fp16, exact), B = the sub-block sums
 //    (hi + lo, two MMAs), k = sub-block index.
@@ -36,8 +44,9 @@
 //    a thread-block cluster of KSPLIT CTAs covers the whole K range and its
 //    partial sums are reduced in rank order through distributed shared memory
 //    (deterministic, no atomics). The decomposition depends only on (N, K), and
-//    the pre-pass record of a row depends only on that row, so a token's
-//    result never depends on the other tokens in the batch.
+//    the pre-pass record of a row depends only on that row, so within a token
+//    class (1..16, 17..32) a token's result never depends on the other tokens
+//    in the batch.
 #pragma once
 #include <cooperative_groups.h>
 
@@ -222,6 +231,10 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
                                                                    GemvParams p) {
   using L = GemvSmem<MT, WARPS, TILES>;
   constexpr int TOK = 8 * MT;
+  // 1..16 tokens: the subnormal-nibble A operand with per-sub-block scaling after the
+  // MMA (fewer instructions per weight); 17..32: fp16 sc*q built before the MMA
+  // (the per-result scaling would grow with the token groups).
+  constexpr bool SUBN = MT <= 2;
   constexpr int WROWS = 16 * TILES;    // weight rows per consumer warp
   constexpr int ROWS = WROWS * WARPS;  // weight rows per CTA
   extern __shared__ __align__(128) uint8_t smem[];
@@ -411,6 +424,55 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           for (int h = 0; h < 2; ++h) {
             const int j = 2 * c + h;  // sub-block
             const uint32_t msk = h ? 0x00F000F0u : 0x000F000Fu;
+            if (SUBN) {
+              // A = the raw nibble field as fp16 bits: q * 2^-24 (low nibble) or 16q * 2^-24
+              // (high), fp16 subnormals, which the tensor core multiplies exactly. The
+              // sub-block's two k-steps accumulate on their own; its scale, sc (sc/16 for
+              // high nibbles) as an exact fp32, is applied to the per-row results.
+              float fs[R];
+#pragma unroll
+              for (int r = 0; r < R; ++r) {  // 0x4B0000sc = 2^23 + sc; 0x490000sc = 2^19 + sc/16
+                const uint32_t bits = __byte_perm(scw[r][j >> 2], h ? 0x49000000u : 0x4B000000u,
+                                                  0x7650u | (uint32_t)(j & 3));
+                fs[r] = __uint_as_float(bits) - (h ? 524288.f : 8388608.f);
+              }
+              uint32_t A[TILES][2][4];
+#pragma unroll
+              for (int tt = 0; tt < TILES; ++tt) {
+                const int ra = 2 * tt, rb = 2 * tt + 1;
+#pragma unroll
+                for (int st = 0; st < 2; ++st) {
+                  A[tt][st][0] = (st ? qv[ra][c].y : qv[ra][c].x) & msk;
+                  A[tt][st][1] = (st ? qv[rb][c].y : qv[rb][c].x) & msk;
+                  A[tt][st][2] = qs8[ra][st] & msk;
+                  A[tt][st][3] = qs8[rb][st] & msk;
+                }
+              }
+#pragma unroll
+              for (int f = 0; f < MT; ++f) {
+                if (GROUPED && 8 * f >= count) break;  // token groups past this expert's rows
+                const uint4 bx = *reinterpret_cast<const uint4*>(xb + (8 * f + g) * kXRec + (j * 4 + t) * 16);
+#pragma unroll
+                for (int tt = 0; tt < TILES; ++tt) {
+                  float Cj[4];
+                  mma_f16_16816(Cj, A[tt][0][0], A[tt][0][1], A[tt][0][2], A[tt][0][3], bx.x, bx.y, true);
+                  mma_f16_16816(Cj, A[tt][1][0], A[tt][1][1], A[tt][1][2], A[tt][1][3], bx.z, bx.w, false);
+                  const float fa = fs[2 * tt], fb = fs[2 * tt + 1];
+                  if (j == 0) {
+                    C[tt][f][0] = fa * Cj[0];
+                    C[tt][f][1] = fa * Cj[1];
+                    C[tt][f][2] = fb * Cj[2];
+                    C[tt][f][3] = fb * Cj[3];
+                  } else {
+                    C[tt][f][0] = fmaf(fa, Cj[0], C[tt][f][0]);
+                    C[tt][f][1] = fmaf(fa, Cj[1], C[tt][f][1]);
+                    C[tt][f][2] = fmaf(fb, Cj[2], C[tt][f][2]);
+                    C[tt][f][3] = fmaf(fb, Cj[3], C[tt][f][3]);
+                  }
+                }
+              }
+              continue;
+            }
             // per row: multiplier (sc, or sc/16 for high nibbles) and bias -1024 * multiplier
             __half2 mul[R], cst[R];
 #pragma unroll
@@ -457,7 +519,8 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         float dd[R], dn[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          dd[r] = half_bits_to_float(hdx[r]);
+          // the subnormal form's products carry 2^-24: fold 2^24 into d
+          dd[r] = (SUBN ? 16777216.f : 1.f) * half_bits_to_float(hdx[r]);
           dn[r] = 64.f * half_bits_to_float(hdx[r] >> 16);
         }
 #pragma unroll

@@ -97,16 +97,23 @@ def test_gemv_dense_decode_sampled(decode_inputs, proj, M):
 
 
 def test_gemv_batch_invariance_and_determinism(decode_inputs):
-    """Row m of an M-token call is bit-identical to the one-token call on row m."""
+    """Within a token class (1..16 tokens: subnormal-nibble operand, per-sub-block
+    scaling; 17..32: fp16 sc*q operand), row m of an M-token call is bit-identical
+    to the same token in any other call of that class; repeated calls are
+    bit-identical."""
     inp, d = decode_inputs
     N, K = inp["W_down"].shape[0], inp["W_down"].shape[1] * 256
     W, X = d["W_down"], d["X_down"]
+    y16 = q.q4k_gemv(W, X[:16], N, K)
+    assert torch.equal(y16, q.q4k_gemv(W, X[:16], N, K))
+    for M in (1, 4, 8, 9):
+        assert torch.equal(q.q4k_gemv(W, X[:M], N, K), y16[:M])
+    for m in (0, 7, 13):
+        assert torch.equal(q.q4k_gemv(W, X[m:m + 1], N, K)[0], y16[m])
     y32 = q.q4k_gemv(W, X[:32], N, K)
     assert torch.equal(y32, q.q4k_gemv(W, X[:32], N, K))
-    for M in (4, 8, 16):
-        assert torch.equal(q.q4k_gemv(W, X[:M], N, K), y32[:M])
-    for m in (0, 7, 13, 31):
-        assert torch.equal(q.q4k_gemv(W, X[m:m + 1], N, K)[0], y32[m])
+    assert torch.equal(q.q4k_gemv(W, X[:17], N, K), y32[:17])
+    assert torch.equal(q.q4k_gemv(W, X[13:30], N, K), y32[13:30])
 
 
 # ---------------------------------------------------------------- MoE route --

@@ -91,10 +91,33 @@ q4k_status q4k_dequant(const void* W, int64_t nblocks, int out_bf16, void* out, 
  *   magnitude of its 256-block). The 4-bit weights and their six-bit scales
  *   enter exactly; products accumulate in fp32. Calls sharing `ws` must be
  *   ordered on one stream.
- * Row m of the result does not depend on the other rows of X (bit-identical
- * to the M == 1 call on that row). */
+ * Within a token class (M = 1..16, M = 17..32) row m of the result does not
+ * depend on the other rows of X (bit-identical to any other call of the same
+ * class on that row). */
 q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                     void* ws, size_t ws_bytes, void* stream);
+
+/* Load-time repack of Q4_K weights for the decode GEMV (hipEngine 0.3.0
+ * README, "GGUF Support": the decode-repacked layouts). A byte permutation:
+ * the same 144 bytes per super-block, so the same HBM traffic.
+ *   Wr[((T*(K/256) + kb)*128 + r)*144 + b] holds super-block kb of weight row
+ *   128*T + r (rows are grouped in 128-row tiles; a tile's super-block column
+ *   is contiguous). Inside the 144 bytes, bytes 0..15 (d, dmin, scales) are
+ *   unchanged and quant byte 32c + 8t + e (chunk c, quarter t, e = 0..7) moves
+ *   to 16 + 32t + 8c + e: the eight bytes a GEMV thread takes from each chunk
+ *   lie together. Rows past N (up to the next multiple of 128) are zero.
+ *   q4k_repacked_bytes(N, K) = ceil(N/128)*128 * K/256 * 144 (0 for a bad
+ *   shape). W and Wr are device buffers of the caller, 16-byte aligned, not
+ *   overlapping. */
+int64_t q4k_repacked_bytes(int N, int K);
+q4k_status q4k_repack(const void* W, int N, int K, void* Wr, void* stream);
+
+/* q4k_gemv on repacked weights (same arguments, Wr from q4k_repack with the
+ * same N, K): each 128-row tile streams as one contiguous run per super-block
+ * column and every thread reads its quant bytes with two 16-byte loads. Same
+ * arithmetic in the same order as q4k_gemv: bit-identical results. */
+q4k_status q4k_gemv_repacked(const void* Wr, const uint16_t* X, float* Y, int M, int N, int K,
+                             void* ws, size_t ws_bytes, void* stream);
 
 /* Prefill GEMM on tcgen05 tensor cores with the Q4_K weights dequantised
  * tile by tile into shared memory (hipEngine 0.3.0 README, "GGUF Support":

@@ -339,3 +339,55 @@ def quantize_brute_force(w: np.ndarray, d: float, dmin: float):
         if not found:
             raise ValueError(f"sub-block {j} has no exact Q4_K representation")
     return sc_out, m_out, q_out
+
+
+# --------------------------------------------------------------------------
+# Load-time decode repack (hipEngine 0.3.0 README, "GGUF Support": the
+# "decode-repacked" layouts). Reading R17: the pages name repacked layouts
+# but give none; the layout taken here is a pure byte permutation (the same
+# 144 bytes per super-block):
+#   * rows are grouped in tiles of 128; tile T's super-block column kb is the
+#     contiguous run of rows 128T .. 128T+127, so the output is indexed
+#     [T][kb][r][144];
+#   * inside a row-block, bytes 0..15 (d, dmin, packed scales) stay, and the
+#     quant byte at 16 + 32c + 8t + e (chunk c, quarter t, e = 0..7) moves to
+#     16 + 32t + 8c + e;
+#   * rows past N, up to the next multiple of 128, are zero bytes.
+# --------------------------------------------------------------------------
+
+REPACK_ROWS = 128
+
+
+def repack_ref(W_blocks: np.ndarray) -> np.ndarray:
+    """The repacked byte array (flat uint8) of W_blocks [N][K/256][144]."""
+    N, nkb, _ = W_blocks.shape
+    tiles = -(-N // REPACK_ROWS)
+    out = np.zeros((tiles, nkb, REPACK_ROWS, BLOCK_BYTES), dtype=np.uint8)
+    for n in range(N):
+        T, r = divmod(n, REPACK_ROWS)
+        for kb in range(nkb):
+            src = W_blocks[n, kb]
+            dst = out[T, kb, r]
+            dst[:16] = src[:16]
+            for c in range(4):
+                for t in range(4):
+                    dst[16 + 32 * t + 8 * c:16 + 32 * t + 8 * c + 8] = src[16 + 32 * c + 8 * t:16 + 32 * c + 8 * t + 8]
+    return out.reshape(-1)
+
+
+def unrepack_ref(Wr: np.ndarray, N: int, K: int) -> np.ndarray:
+    """Inverse of repack_ref: the [N][K/256][144] blocks back from the flat bytes."""
+    nkb = K // QK
+    tiles = -(-N // REPACK_ROWS)
+    R = Wr.reshape(tiles, nkb, REPACK_ROWS, BLOCK_BYTES)
+    out = np.zeros((N, nkb, BLOCK_BYTES), dtype=np.uint8)
+    for n in range(N):
+        T, r = divmod(n, REPACK_ROWS)
+        for kb in range(nkb):
+            src = R[T, kb, r]
+            dst = out[n, kb]
+            dst[:16] = src[:16]
+            for c in range(4):
+                for t in range(4):
+                    dst[16 + 32 * c + 8 * t:16 + 32 * c + 8 * t + 8] = src[16 + 32 * t + 8 * c:16 + 32 * t + 8 * c + 8]
+    return out

@@ -14,7 +14,8 @@ import os
 import torch
 
 __all__ = [
-    "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemm", "moe_route_permute",
+    "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_repack", "q4k_gemv_repacked", "q4k_gemm",
+    "moe_route_permute",
     "moe_route_permute_noalloc",
     "moe_q4k_grouped", "moe_combine", "q4k_workspace_bytes", "q4k_last_device_status",
     "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "OP_GEMV", "EXPORTS",
@@ -30,6 +31,9 @@ _p, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size
 EXPORTS = {
     "q4k_dequant": (_i, [_p, _i64, _i, _p, _p]),
     "q4k_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
+    "q4k_repacked_bytes": (_i64, [_i, _i]),
+    "q4k_repack": (_i, [_p, _i, _i, _p, _p]),
+    "q4k_gemv_repacked": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "q4k_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "moe_route_permute": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_route_permute_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
@@ -115,6 +119,28 @@ def q4k_gemv(W, X, N: int, K: int, Y=None, ws=None, stream=None):
     ws = _scratch(q4k_workspace_bytes(OP_GEMV, M, N, K), X.device, ws)
     _check("q4k_gemv", lib().q4k_gemv(_ptr(W), _ptr(_bits16(X)), _ptr(Y), M, N, K, _ptr(ws), ws.numel(),
                                       _stream(stream)))
+    return Y
+
+
+def q4k_repack(W, N: int, K: int, Wr=None, stream=None):
+    """Repacked copy of Q4_K weights W [N][K/256][144] for q4k_gemv_repacked (uint8, flat)."""
+    nb = lib().q4k_repacked_bytes(N, K)
+    if nb <= 0:
+        raise ValueError(f"q4k_repack: bad shape N={N} K={K}")
+    if Wr is None:
+        Wr = torch.empty(nb, dtype=torch.uint8, device=W.device)
+    _check("q4k_repack", lib().q4k_repack(_ptr(W), N, K, _ptr(Wr), _stream(stream)))
+    return Wr
+
+
+def q4k_gemv_repacked(Wr, X, N: int, K: int, Y=None, ws=None, stream=None):
+    """q4k_gemv on weights from q4k_repack (bit-identical results)."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
+    ws = _scratch(q4k_workspace_bytes(OP_GEMV, M, N, K), X.device, ws)
+    _check("q4k_gemv_repacked", lib().q4k_gemv_repacked(_ptr(Wr), _ptr(_bits16(X)), _ptr(Y), M, N, K, _ptr(ws),
+                                                        ws.numel(), _stream(stream)))
     return Y
 
 

@@ -190,10 +190,16 @@ constexpr int kGemvPitch = 160;
 //   xring [xstages][8*MT tokens][576 B]            activation records (bulk-copy destination)
 //   red   [16*TILES*WARPS rows][8*MT] fp32         per-CTA partial result
 //   bars  wfull, wempty [wstages], xfull, xempty [xstages]; abort flag
-template <int MT, int WARPS, int TILES>
+// Repacked weights (q4k_repack): 128-row tiles whose super-block columns are
+// contiguous and whose row-blocks keep each thread's 32 quant bytes together;
+// the stage is one bulk copy and the smem pitch the block size itself.
+constexpr int kRepackRows = 128;
+
+template <int MT, int WARPS, int TILES, bool REPACK = false>
 struct GemvSmem {
   static constexpr int TOK = 8 * MT;
-  static constexpr int warp_tile = 16 * TILES * kGemvPitch;
+  static constexpr int pitch = REPACK ? BLOCK_BYTES : kGemvPitch;
+  static constexpr int warp_tile = 16 * TILES * pitch;
   static constexpr size_t wstage = (size_t)WARPS * warp_tile;
   static constexpr size_t xstage = (size_t)TOK * kXRec;
   static constexpr __host__ __device__ size_t xring_off(int ws) { return (size_t)ws * wstage; }
@@ -226,10 +232,11 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
 // GROUPED: blockIdx.y enumerates non-empty experts (the y-th expert with a
 // non-zero row count); SWIGLU: the first WARPS/2 consumer warps hold gate rows
 // and the last WARPS/2 the matching up rows (at +N/2).
-template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU>
+template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false>
 __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                                    GemvParams p) {
-  using L = GemvSmem<MT, WARPS, TILES>;
+  using L = GemvSmem<MT, WARPS, TILES, REPACK>;
+  static_assert(!REPACK || (!GROUPED && 16 * TILES * WARPS == kRepackRows), "repacked: dense, 128-row tiles");
   constexpr int TOK = 8 * MT;
   // 1..16 tokens: the subnormal-nibble A operand with per-sub-block scaling after the
   // MMA (fewer instructions per weight); 17..32: fp16 sc*q built before the MMA
@@ -241,7 +248,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int SW = p.wstages, SX = p.xstages;
-  if (threadIdx.x == 32 * WARPS)  // the weight-TMA thread: fetch the descriptor while the rest sets up
+  if (!REPACK && threadIdx.x == 32 * WARPS)  // the weight-TMA thread: fetch the descriptor while the rest sets up
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
 
   const int rank = (int)(blockIdx.x % (unsigned)p.ksplit);
@@ -326,8 +333,12 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         mbar_arrive_expect_tx(wfull(s), (uint32_t)(WARPS * L::warp_tile));
         const uint32_t dst = smem_u32(smem) + (uint32_t)(s * L::wstage);
         const int x = (kb0 + ks) * BLOCK_BYTES;
+        if (REPACK) {  // the tile's super-block column is one contiguous 18 KB run
+          const uint8_t* src = p.W + ((size_t)tile * p.nkb + (kb0 + ks)) * (size_t)L::wstage;
+          bulk_copy_g2s(dst, src, (uint32_t)L::wstage, wfull(s));
+        }
 #pragma unroll
-        for (int w = 0; w < WARPS; ++w) {
+        for (int w = 0; w < (REPACK ? 0 : WARPS); ++w) {
           int r0 = SWIGLU ? tile * (ROWS / 2) + WROWS * (w % (WARPS / 2)) : tile * ROWS + WROWS * w;
           r0 = min(r0, lim);  // rows past the end read zeros (or are ignored)
           const int row = expert * p.N + (SWIGLU && w >= WARPS / 2 ? p.N / 2 : 0) + r0;
@@ -395,12 +406,21 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
       uint2 qv[R][4];  // [row][chunk]
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        const uint8_t* rp = wt + (g + 8 * r) * kGemvPitch;
+        const uint8_t* rp = wt + (g + 8 * r) * L::pitch;
         const uint4 hd = *reinterpret_cast<const uint4*>(rp);
         hdx[r] = hd.x;
         unpack_scales(hd.y, hd.z, hd.w, scw[r], mnw[r]);
+        if (REPACK) {  // this thread's bytes [8t, 8t+8) of chunks 0..3, stored together
+          const uint4 q01 = *reinterpret_cast<const uint4*>(rp + 16 + 32 * t);
+          const uint4 q23 = *reinterpret_cast<const uint4*>(rp + 32 + 32 * t);
+          qv[r][0] = make_uint2(q01.x, q01.y);
+          qv[r][1] = make_uint2(q01.z, q01.w);
+          qv[r][2] = make_uint2(q23.x, q23.y);
+          qv[r][3] = make_uint2(q23.z, q23.w);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) qv[r][c] = *reinterpret_cast<const uint2*>(rp + 16 + 32 * c + 8 * t);
+          for (int c = 0; c < 4; ++c) qv[r][c] = *reinterpret_cast<const uint2*>(rp + 16 + 32 * c + 8 * t);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(wempty(sw));  // the weight tile is in registers: release it
@@ -610,6 +630,35 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     }
   }
   if (p.ksplit > 1) cluster.sync();  // keep every CTA's shared memory alive until all ranks are done
+}
+
+// Load-time repack (one thread per 8-byte unit of the output): row r of 128-row
+// tile T, super-block kb lands at ((T*nkb + kb)*128 + r)*144; inside the 144
+// bytes the header (units 0..1) stays and quant unit 2 + 4t + c takes the
+// source's unit 2 + 4c + t (bytes [8t, 8t+8) of chunk c), so the eight bytes a
+// GEMV thread t needs from each chunk follow one another. Rows past N are zero.
+__global__ void __launch_bounds__(256) repack_kernel(const uint8_t* __restrict__ W, int N, int nkb,
+                                                     uint8_t* __restrict__ Wr, int64_t units) {
+  const int64_t row_bytes = (int64_t)nkb * BLOCK_BYTES;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t blk = u / 18;  // output row-block, tile-major
+    const int pu = (int)(u - blk * 18);
+    const int r = (int)(blk % kRepackRows);
+    const int64_t tk = blk / kRepackRows;
+    const int kb = (int)(tk % nkb);
+    const int64_t row = (tk / nkb) * kRepackRows + r;
+    uint2 v = make_uint2(0u, 0u);
+    if (row < N) {
+      const int su = pu < 2 ? pu : 2 + 4 * ((pu - 2) & 3) + ((pu - 2) >> 2);
+      v = *reinterpret_cast<const uint2*>(W + row * row_bytes + (int64_t)kb * BLOCK_BYTES + 8 * su);
+    }
+    *reinterpret_cast<uint2*>(Wr + blk * BLOCK_BYTES + 8 * pu) = v;
+  }
+}
+
+inline int64_t repacked_bytes(int N, int K) {
+  return (int64_t)((N + kRepackRows - 1) / kRepackRows) * kRepackRows * (K / QK) * BLOCK_BYTES;
 }
 
 // Raw Q4_K rows as bytes [rows][row_bytes], box 160 bytes x box_rows rows (one super-block

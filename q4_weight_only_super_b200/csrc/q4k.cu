@@ -146,14 +146,14 @@ q4k_status pick_gemv(int tokens, int rows_out, int nkb, int groups, GemvCfg* out
   return Q4K_OK;
 }
 
-template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU>
+template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false>
 q4k_status launch_gemv_t(const GemvParams& p, int rows_total, int tiles, int groups, cudaStream_t s) {
-  auto* k = gemv_kernel<MT, WARPS, TILES, GROUPED, SWIGLU>;
+  auto* k = gemv_kernel<MT, WARPS, TILES, GROUPED, SWIGLU, REPACK>;
   static std::atomic<size_t> smem_set[kMaxDevices];  // one per instantiation
-  CUtensorMap tmap;
-  if (!make_tmap_w_rowgroup(&tmap, p.W, rows_total, (int64_t)p.nkb * BLOCK_BYTES, 16 * TILES))
+  CUtensorMap tmap = {};  // repacked weights stream by plain bulk copies: no tensor map
+  if (!REPACK && !make_tmap_w_rowgroup(&tmap, p.W, rows_total, (int64_t)p.nkb * BLOCK_BYTES, 16 * TILES))
     return Q4K_ERR_CUDA;
-  const size_t smem = GemvSmem<MT, WARPS, TILES>::total(p.wstages, p.xstages);
+  const size_t smem = GemvSmem<MT, WARPS, TILES, REPACK>::total(p.wstages, p.xstages);
   if (ensure_smem(k, smem, smem_set) != cudaSuccess) return Q4K_ERR_LAUNCH;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * p.ksplit), (unsigned)groups, 1);
@@ -175,7 +175,7 @@ q4k_status launch_gemv_t(const GemvParams& p, int rows_total, int tiles, int gro
 }
 
 // Activation pre-pass (rows of X, gathered when `gather` is set) then the GEMV.
-template <bool GROUPED, bool SWIGLU>
+template <bool GROUPED, bool SWIGLU, bool REPACK = false>
 q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const int32_t* gather,
                        int rows, int K, void* ws, int rows_out, int groups, cudaStream_t s) {
   p.ksplit = c.ksplit;
@@ -189,9 +189,9 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
                                    rows, p.rows_pad, K, p.nkb, static_cast<uint8_t*>(ws));
   if (st != Q4K_OK) return st;
   const int tiles = (rows_out + 128 - 1) / 128;
-  if (c.mt == 1) return launch_gemv_t<1, 4, 2, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
-  if (c.mt == 2) return launch_gemv_t<2, 4, 2, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
-  return launch_gemv_t<4, 4, 2, GROUPED, SWIGLU>(p, total_rows, tiles, groups, s);
+  if (c.mt == 1) return launch_gemv_t<1, 4, 2, GROUPED, SWIGLU, REPACK>(p, total_rows, tiles, groups, s);
+  if (c.mt == 2) return launch_gemv_t<2, 4, 2, GROUPED, SWIGLU, REPACK>(p, total_rows, tiles, groups, s);
+  return launch_gemv_t<4, 4, 2, GROUPED, SWIGLU, REPACK>(p, total_rows, tiles, groups, s);
 }
 
 // Routing kernels keep each lane's share of a logit row in registers: pick the
@@ -288,6 +288,44 @@ q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
   const q4k_status st = pick_gemv(M, N, p.nkb, 1, &c);
   if (st != Q4K_OK) return st;
   return launch_gemv<false, false>(c, p, X, nullptr, M, K, ws, N, 1, static_cast<cudaStream_t>(stream));
+}
+
+
+int64_t q4k_repacked_bytes(int N, int K) {
+  if (N <= 0 || K <= 0 || K % QK) return 0;
+  return repacked_bytes(N, K);
+}
+
+q4k_status q4k_repack(const void* W, int N, int K, void* Wr, void* stream) {
+  if (N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (N == 0) return Q4K_OK;
+  if (!W || !Wr) return Q4K_ERR_NULL;
+  if (!aligned16(W) || !aligned16(Wr)) return Q4K_ERR_ALIGN;
+  const int64_t units = repacked_bytes(N, K) / 8;
+  const int64_t grid = std::min<int64_t>((units + 255) / 256, 148 * 32);
+  repack_kernel<<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(W), N, K / QK, static_cast<uint8_t*>(Wr), units);
+  return launch_status(cudaGetLastError());
+}
+
+q4k_status q4k_gemv_repacked(const void* Wr, const uint16_t* X, float* Y, int M, int N, int K, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (M == 0 || N == 0) return Q4K_OK;
+  if (!Wr || !X || !Y || !ws) return Q4K_ERR_NULL;
+  if (!aligned16(Wr) || !aligned16(X) || !aligned16(Y) || !aligned16(ws)) return Q4K_ERR_ALIGN;
+  if (M > 32 || N % 16) return Q4K_ERR_UNSUPPORTED;
+  if (ws_bytes < gemv_ws_bytes(M, K)) return Q4K_ERR_WORKSPACE;
+  GemvParams p = {};
+  p.W = static_cast<const uint8_t*>(Wr);
+  p.out = Y;
+  p.M = M;
+  p.N = N;
+  p.nkb = K / QK;
+  GemvCfg c;
+  const q4k_status st = pick_gemv(M, N, p.nkb, 1, &c);  // the raw-layout choice: same sums, same order
+  if (st != Q4K_OK) return st;
+  return launch_gemv<false, false, true>(c, p, X, nullptr, M, K, ws, N, 1, static_cast<cudaStream_t>(stream));
 }
 
 q4k_status q4k_gemm(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws,

@@ -116,6 +116,39 @@ def test_gemv_batch_invariance_and_determinism(decode_inputs):
     assert torch.equal(q.q4k_gemv(W, X[13:30], N, K), y32[13:30])
 
 
+# ------------------------------------------------------------ decode repack --
+
+@pytest.mark.parametrize("N,K", [(16, 256), (200, 512), (1040, 256 * 69)])
+def test_repack_matches_reference(N, K):
+    W, _ = synth.gemv_small(300, N=N, K=K, M=1)
+    Wr = host(q.q4k_repack(dev(W), N, K))
+    assert np.array_equal(Wr, O.repack_ref(W))
+
+
+@pytest.mark.parametrize("N,K", [(16, 256), (272, 4096), (1040, 256 * 69)])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 17, 32])
+def test_gemv_repacked_equals_raw_and_oracle(N, K, M):
+    """Same arithmetic in the same order as q4k_gemv: bit-identical; and within tolerance."""
+    W, X = synth.gemv_small(310 + M, N=N, K=K, M=M)
+    Wd, Xd = dev(W), dev(X)
+    y_raw = q.q4k_gemv(Wd, Xd, N, K)
+    y_rep = q.q4k_gemv_repacked(q.q4k_repack(Wd, N, K), Xd, N, K)
+    assert torch.equal(y_rep, y_raw)
+    Y, S = O.matmul_ref(W, X)
+    _assert_tol(host(y_rep), Y, S, f"repacked N={N} K={K} M={M}")
+
+
+@pytest.mark.parametrize("proj", ["gate_up", "down"])
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_gemv_repacked_dense_decode(decode_inputs, proj, M):
+    inp, d = decode_inputs
+    W = inp[f"W_{proj}"]
+    N, K = W.shape[0], W.shape[1] * 256
+    Wr = q.q4k_repack(d[f"W_{proj}"], N, K)
+    X = d[f"X_{proj}"][:M]
+    assert torch.equal(q.q4k_gemv_repacked(Wr, X, N, K), q.q4k_gemv(d[f"W_{proj}"], X, N, K))
+
+
 # ---------------------------------------------------------------- MoE route --
 
 def _route_and_check(logits, topk=8):

@@ -361,3 +361,58 @@ def _d_dmin_swapped(blocks):
                                  dict(scale_min_pairs=_hi_bits_wrong), dict(block_d_dmin=_d_dmin_swapped)])
 def test_planted_mistakes_are_caught(mut):
     assert not _golden_ok(_Mutant(**mut))
+
+
+# ------------------------------------------------------------ decode repack --
+# repack_ref is a byte permutation; these pins check it against properties the
+# layout definition fixes, each chosen so that a plausible slip (chunk and
+# quarter swapped, rows and blocks swapped in the tile order, the header moved,
+# padding rows not zero) fails one of them.
+
+def _tagged_blocks(N, nkb):
+    """Blocks whose header names (row, block) and whose quant bytes are 0..127."""
+    W = np.zeros((N, nkb, O.BLOCK_BYTES), dtype=np.uint8)
+    for n in range(N):
+        for kb in range(nkb):
+            W[n, kb, 0] = n & 255
+            W[n, kb, 1] = n >> 8
+            W[n, kb, 2] = kb
+            W[n, kb, 3] = 0xA5
+            W[n, kb, 16:] = np.arange(128, dtype=np.uint8)
+    return W
+
+
+def test_repack_tile_order_and_padding():
+    N, nkb = 200, 3  # two tiles, the second ragged (72 rows)
+    Wr = O.repack_ref(_tagged_blocks(N, nkb))
+    assert Wr.size == 2 * nkb * 128 * 144
+    for n, kb in [(0, 0), (1, 0), (127, 2), (128, 0), (130, 1), (199, 2)]:
+        off = ((n // 128 * nkb + kb) * 128 + n % 128) * 144
+        assert Wr[off] == n & 255 and Wr[off + 1] == n >> 8 and Wr[off + 2] == kb and Wr[off + 3] == 0xA5
+    # rows 200..255 of the second tile are zero
+    R = Wr.reshape(2, nkb, 128, 144)
+    assert not R[1, :, 72:, :].any()
+
+
+def test_repack_quarter_runs():
+    """A GEMV thread t reads 32 consecutive bytes at 16 + 32t: quant bytes
+    [8t, 8t+8) of chunks 0, 1, 2, 3 in that order (byte values 0..127 = index)."""
+    R = O.repack_ref(_tagged_blocks(1, 1)).reshape(128, 144)[0]
+    expect = {0: [0, 32, 64, 96], 1: [8, 40, 72, 104], 2: [16, 48, 80, 112], 3: [24, 56, 88, 120]}
+    for t, starts in expect.items():
+        run = R[16 + 32 * t:16 + 32 * t + 32]
+        assert list(run) == [s + e for s in starts for e in range(8)]
+
+
+def test_repack_round_trip_and_byte_multisets():
+    rng = np.random.default_rng(17)
+    N, nkb = 300, 4
+    W = rng.integers(0, 256, size=(N, nkb, 144), dtype=np.uint8)
+    Wr = O.repack_ref(W)
+    assert np.array_equal(O.unrepack_ref(Wr, N, nkb * 256), W)
+    R = Wr.reshape(-1, nkb, 128, 144)
+    for n in (0, 77, 128, 299):
+        for kb in range(nkb):
+            blk = R[n // 128, kb, n % 128]
+            assert np.array_equal(blk[:16], W[n, kb, :16])
+            assert np.array_equal(np.sort(blk[16:]), np.sort(W[n, kb, 16:]))

@@ -13,7 +13,7 @@ HEADER = os.path.join(ROOT, "include", "q4k.h")
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(?:q4k_status|size_t|const char\*)\s+(\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(?:q4k_status|size_t|int64_t|const char\*)\s+(\w+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -26,7 +26,8 @@ def L():
 
 def test_header_declares_the_boundary():
     names = _declared()
-    for n in ("q4k_gemv", "q4k_gemm", "moe_route_permute", "moe_q4k_grouped", "moe_combine"):
+    for n in ("q4k_gemv", "q4k_gemm", "moe_route_permute", "moe_q4k_grouped", "moe_combine",
+              "q4k_repack", "q4k_repacked_bytes", "q4k_gemv_repacked"):
         assert n in names
 
 
@@ -83,3 +84,20 @@ def test_workspace_size(L):
     # GEMV: (K/256) blocks x (M + 32 padding rows) x 576-byte records
     assert L.q4k_workspace_bytes(4, 1, 34816, 5120, 0, 0) == 20 * 33 * 576
     assert L.q4k_workspace_bytes(3, 256, 1536, 2048, 128, 8) == 8 * 288 * 576
+
+
+def test_repack_arguments(L):
+    fake = 4096
+    big = 1 << 30
+    # 128-row tiles x (K/256) super-blocks x 144 bytes; N padded to the tile
+    assert L.q4k_repacked_bytes(200, 512) == 2 * 2 * 128 * 144
+    assert L.q4k_repacked_bytes(128, 256) == 128 * 144
+    assert L.q4k_repacked_bytes(0, 256) == 0 and L.q4k_repacked_bytes(16, 100) == 0
+    assert L.q4k_repack(fake, 16, 100, fake, None) == 3       # K % 256
+    assert L.q4k_repack(None, 16, 256, fake, None) == 1
+    assert L.q4k_repack(fake, 16, 256, fake + 8, None) == 2   # misaligned
+    assert L.q4k_repack(None, 0, 256, None, None) == 0        # empty: no-op
+    assert L.q4k_gemv_repacked(fake, fake, fake, 33, 16, 256, fake, big, None) == 4
+    assert L.q4k_gemv_repacked(fake, fake, fake, 1, 24, 256, fake, big, None) == 4
+    assert L.q4k_gemv_repacked(fake, fake, fake, 1, 16, 256, fake, 64, None) == 5
+    assert L.q4k_gemv_repacked(None, None, None, 0, 16, 256, None, 0, None) == 0

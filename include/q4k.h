@@ -208,6 +208,18 @@ q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uin
 q4k_status moe_combine(const float* O, const int32_t* inv_perm, const float* topk_w,
                        int M, int topk, int H, float* Y, void* stream);
 
+/* The combine fused with the residual add (hipEngine 0.3.0 README, "Core
+ * principles": the gate_combine_residual composite).
+ *   y[t][h] = residual[t][h] + (sum_{j=0..topk-1} topk_w[t][j] * O[inv_perm[t*topk + j]][h]),
+ *   the sum taken as in moe_combine, then one fp32 add, so the result equals
+ *   moe_combine's followed by an fp32 add of residual, bit for bit.
+ * residual fp32 [M][H], caller-owned; it may be the same buffer as Y (in
+ * place). Shapes, alignment and errors as moe_combine; a null residual is
+ * Q4K_ERR_NULL. */
+q4k_status moe_combine_residual(const float* O, const int32_t* inv_perm, const float* topk_w,
+                                const float* residual, int M, int topk, int H, float* Y,
+                                void* stream);
+
 /* Bytes of device workspace an entry point needs for these sizes
  * (Q4K_OP_ROUTE: moe_route_permute with M tokens and E experts;
  *  Q4K_OP_GEMV: q4k_gemv with M tokens and K inputs;

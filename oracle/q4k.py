@@ -255,6 +255,19 @@ def combine_ref(O: np.ndarray, inv_perm: np.ndarray, w: np.ndarray):
     return y, S
 
 
+def combine_residual_ref(O: np.ndarray, inv_perm: np.ndarray, w: np.ndarray, R: np.ndarray):
+    """The gate_combine_residual composite (hipEngine 0.3.0 README, "Core
+    principles"): y[t] = R[t] + sum_j w[t,j] * O[inv_perm[t*topk + j]], fp64.
+
+    Reading R18: the pages name the fused composite but not its order of
+    operations; the sum over j is formed first (as in ``combine_ref``) and the
+    residual added last. Returns ``(y, S)`` with ``S = |R| + sum_j |w*O|``.
+    """
+    y, S = combine_ref(O, inv_perm, w)
+    R = np.asarray(R, dtype=np.float64)
+    return R + y, np.abs(R) + S
+
+
 def moe_layer_ref(logits, X_bits, W_gate_up, W_down, topk: int):
     """End-to-end fp64 MoE layer (no intermediate rounding): y[t] =
     sum_j w[t,j] * W_down[e_j] @ (SiLU(W_gate[e_j] x_t) * (W_up[e_j] x_t))."""

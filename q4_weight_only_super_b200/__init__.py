@@ -17,7 +17,7 @@ __all__ = [
     "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_repack", "q4k_gemv_repacked", "q4k_gemm",
     "moe_route_permute",
     "moe_route_permute_noalloc",
-    "moe_q4k_grouped", "moe_combine", "q4k_workspace_bytes", "q4k_last_device_status",
+    "moe_q4k_grouped", "moe_combine", "moe_combine_residual", "q4k_workspace_bytes", "q4k_last_device_status",
     "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "OP_GEMV", "EXPORTS",
 ]
 
@@ -39,6 +39,7 @@ EXPORTS = {
     "moe_route_permute_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
     "moe_q4k_grouped": (_i, [_p, _i, _i, _i, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
     "moe_combine": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
+    "moe_combine_residual": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "q4k_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "q4k_last_device_status": (_i, [_p]),
     "q4k_status_string": (ctypes.c_char_p, [_i]),
@@ -229,6 +230,15 @@ def moe_combine(O, inv_perm, topk_w, M: int, topk: int, H: int, Y=None, stream=N
         Y = torch.empty(M, H, dtype=torch.float32, device=O.device)
     _check("moe_combine", lib().moe_combine(_ptr(O), _ptr(inv_perm), _ptr(topk_w), M, topk, H,
                                             _ptr(Y), _stream(stream)))
+    return Y
+
+
+def moe_combine_residual(O, inv_perm, topk_w, residual, M: int, topk: int, H: int, Y=None, stream=None):
+    """y[t] = residual[t] + sum_j topk_w[t,j] * O[inv_perm[t*topk+j]] (Y may be residual)."""
+    if Y is None:
+        Y = torch.empty(M, H, dtype=torch.float32, device=O.device)
+    _check("moe_combine_residual", lib().moe_combine_residual(_ptr(O), _ptr(inv_perm), _ptr(topk_w), _ptr(residual),
+                                                              M, topk, H, _ptr(Y), _stream(stream)))
     return Y
 
 

@@ -295,9 +295,13 @@ route_permute_one_kernel(const float* __restrict__ logits, int M, int E, int top
 // first, then their O rows, then they are added in slot order (two memory
 // latencies per eight slots, at a register count that keeps the large-M case
 // bandwidth-bound).
+// RESID: y = residual + (the weighted sum), one final fp32 add (the
+// gate_combine_residual composite); residual may be Y itself (each thread reads
+// its four values before it writes them).
+template <bool RESID>
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ O, const int32_t* __restrict__ inv_perm,
-               const float* __restrict__ w, int M, int topk, int H, float* __restrict__ Y) {
+               const float* __restrict__ w, int M, int topk, int H, const float* residual, float* Y) {
   asm volatile("griddepcontrol.wait;" ::: "memory");  // O comes from the expert GEMV
   const int t = blockIdx.y;
   const int h4 = blockIdx.x * blockDim.x + threadIdx.x;  // index of a float4
@@ -336,6 +340,13 @@ combine_kernel(const float* __restrict__ O, const int32_t* __restrict__ inv_perm
       acc.z = fmaf(wj[j], o[j].z, acc.z);
       acc.w = fmaf(wj[j], o[j].w, acc.w);
     }
+  }
+  if (RESID) {
+    const float4 rv = *reinterpret_cast<const float4*>(residual + (int64_t)t * H + 4 * h4);
+    acc.x = rv.x + acc.x;
+    acc.y = rv.y + acc.y;
+    acc.z = rv.z + acc.z;
+    acc.w = rv.w + acc.w;
   }
   *reinterpret_cast<float4*>(Y + (int64_t)t * H + 4 * h4) = acc;
 }

@@ -497,8 +497,22 @@ q4k_status moe_combine(const float* O, const int32_t* inv_perm, const float* top
   if (H % 4 || M > 65535 || topk > kMaxTopk) return Q4K_ERR_UNSUPPORTED;
   const int n4 = H / 4;
   dim3 grid((n4 + 255) / 256, M);
-  return launch_pdl(combine_kernel, grid, dim3(256), static_cast<cudaStream_t>(stream), O, inv_perm, topk_w, M,
-                    topk, H, Y);
+  return launch_pdl(combine_kernel<false>, grid, dim3(256), static_cast<cudaStream_t>(stream), O, inv_perm, topk_w,
+                    M, topk, H, static_cast<const float*>(nullptr), Y);
+}
+
+q4k_status moe_combine_residual(const float* O, const int32_t* inv_perm, const float* topk_w,
+                                const float* residual, int M, int topk, int H, float* Y, void* stream) {
+  if (M < 0 || topk <= 0 || H <= 0) return Q4K_ERR_SHAPE;
+  if (M == 0) return Q4K_OK;
+  if (!O || !inv_perm || !topk_w || !residual || !Y) return Q4K_ERR_NULL;
+  if (!aligned16(O) || !aligned16(inv_perm) || !aligned16(topk_w) || !aligned16(residual) || !aligned16(Y))
+    return Q4K_ERR_ALIGN;
+  if (H % 4 || M > 65535 || topk > kMaxTopk) return Q4K_ERR_UNSUPPORTED;
+  const int n4 = H / 4;
+  dim3 grid((n4 + 255) / 256, M);
+  return launch_pdl(combine_kernel<true>, grid, dim3(256), static_cast<cudaStream_t>(stream), O, inv_perm, topk_w,
+                    M, topk, H, residual, Y);
 }
 
 q4k_status q4k_last_device_status(void* stream) {

@@ -27,7 +27,7 @@ def L():
 def test_header_declares_the_boundary():
     names = _declared()
     for n in ("q4k_gemv", "q4k_gemm", "moe_route_permute", "moe_q4k_grouped", "moe_combine",
-              "q4k_repack", "q4k_repacked_bytes", "q4k_gemv_repacked"):
+              "q4k_repack", "q4k_repacked_bytes", "q4k_gemv_repacked", "moe_combine_residual"):
         assert n in names
 
 
@@ -72,6 +72,9 @@ def test_argument_errors_return_before_launch(L):
     # grouped: bad activation code, combine: H % 4
     assert L.moe_q4k_grouped(fake, 4, 64, 256, fake, None, fake, 8, 8, 7, fake, None, 0, None) == 4
     assert L.moe_combine(fake, fake, fake, 2, 2, 6, fake, None) == 4
+    assert L.moe_combine_residual(fake, fake, fake, fake, 2, 2, 6, fake, None) == 4
+    assert L.moe_combine_residual(fake, fake, fake, None, 2, 2, 8, fake, None) == 1
+    assert L.moe_combine_residual(None, None, None, None, 0, 2, 8, None, None) == 0
     # empty problems are no-ops
     assert L.q4k_gemv(None, None, None, 0, 16, 256, None, 0, None) == 0
     assert L.moe_combine(None, None, None, 0, 2, 8, None, None) == 0

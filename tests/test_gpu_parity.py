@@ -206,6 +206,25 @@ def test_combine():
     assert np.all(np.abs(y - Y) <= 1e-6 * S + 1e-30)
 
 
+def test_combine_residual():
+    """Within tolerance of the oracle; bit-identical to the plain combine followed
+    by an fp32 add of the residual; in place (Y = residual) gives the same."""
+    rng = np.random.default_rng(6)
+    M, topk, H = 37, 8, 2048
+    Od = rng.standard_normal((M * topk, H)).astype(np.float32)
+    inv = rng.permutation(M * topk).astype(np.int32)
+    w = rng.random((M, topk)).astype(np.float32)
+    R = rng.standard_normal((M, H)).astype(np.float32)
+    Odd, invd, wd, Rd = dev(Od), dev(inv), dev(w), dev(R)
+    y = q.moe_combine_residual(Odd, invd, wd, Rd, M, topk, H)
+    Y, S = O.combine_residual_ref(Od, inv, w, R)
+    assert np.all(np.abs(host(y) - Y) <= 1e-6 * S + 1e-30)
+    assert torch.equal(y, Rd + q.moe_combine(Odd, invd, wd, M, topk, H))
+    Ri = Rd.clone()
+    q.moe_combine_residual(Odd, invd, wd, Ri, M, topk, H, Y=Ri)
+    assert torch.equal(Ri, y)
+
+
 def test_combine_bad_index_latches_status():
     M, topk, H = 2, 2, 8
     Od = torch.zeros(M * topk, H, device="cuda")

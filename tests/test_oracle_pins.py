@@ -263,6 +263,30 @@ def test_combine_linear_and_gather():
     np.testing.assert_array_equal(yg, O1[inv.reshape(M, topk)[:, 1]])
 
 
+def test_combine_residual_reduces_and_adds():
+    """Zero weights give the residual itself; a zero residual gives the plain
+    combine; the residual enters once, unscaled, whatever the weights."""
+    rng = np.random.default_rng(5)
+    M, topk, H = 4, 3, 8
+    Od = rng.standard_normal((M * topk, H))
+    inv = rng.permutation(M * topk).astype(np.int32)
+    w = rng.random((M, topk))
+    R = rng.standard_normal((M, H))
+    y0, S0 = O.combine_residual_ref(Od, inv, np.zeros((M, topk)), R)
+    np.testing.assert_array_equal(y0, R)
+    np.testing.assert_array_equal(S0, np.abs(R))
+    yc, _ = O.combine_ref(Od, inv, w)
+    yz, _ = O.combine_residual_ref(Od, inv, w, np.zeros((M, H)))
+    np.testing.assert_array_equal(yz, yc)
+    # one-hot weights: residual plus the gathered row, element by element
+    onehot = np.zeros((M, topk))
+    onehot[:, 2] = 1.0
+    yg, _ = O.combine_residual_ref(Od, inv, onehot, R)
+    for t in range(M):
+        for hh in range(H):
+            assert yg[t, hh] == R[t, hh] + Od[inv[t * topk + 2], hh]
+
+
 def test_moe_layer_token_permutation_and_expert_relabel():
     inp, topk = _small_moe(31)
     y = O.moe_layer_ref(inp["logits"], inp["X"], inp["W_gate_up"], inp["W_down"], topk)

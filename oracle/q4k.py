@@ -123,6 +123,57 @@ def f64_to_bf16_bits(a: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Q5_K super-block (sibling K-quant; hipEngine 0.3.0 README, "GGUF Support":
+# the tensor-family table lists Q5_K beside Q4_K, Q8_0 and Q6_K). Reading R19:
+# the pages give no byte layout; the one taken is the llama.cpp-style K-quant
+# block of 256 weights in 176 bytes: fp16 d, fp16 dmin, the same 12-byte
+# six-bit (scale, min) packing as Q4_K (bytes 4..15), 32 bytes qh of fifth
+# bits (bytes 16..47) and the 128 bytes of low nibbles laid out as Q4_K's
+# (bytes 48..175). Weight i = 64c + 32h + l takes its low four bits from
+# nibble h of byte 48 + 32c + l and its fifth bit from bit 2c + h of qh[l]:
+# q = nibble + 16 * bit in 0..31, w = d*sc_j*q - dmin*m_j with j = i // 32.
+# --------------------------------------------------------------------------
+
+Q5_BLOCK_BYTES = 176
+
+
+def quants_q5(blocks: np.ndarray) -> np.ndarray:
+    """The 256 five-bit quants (0..31) of each Q5_K block, in weight order."""
+    b = np.asarray(blocks, dtype=np.uint8)
+    qh = b[..., 16:48].astype(np.int64)
+    qs = b[..., 48:176].astype(np.int64)
+    q = np.empty(qs.shape[:-1] + (QK,), dtype=np.int64)
+    for c in range(4):
+        for h in range(2):
+            low = (qs[..., 32 * c: 32 * c + 32] >> (4 * h)) & 15
+            high = (qh >> (2 * c + h)) & 1
+            q[..., 64 * c + 32 * h: 64 * c + 32 * h + 32] = low + 16 * high
+    return q
+
+
+def dequant_exact_q5(blocks: np.ndarray) -> np.ndarray:
+    """Exact Q5_K weights in fp64 (``[..., nb, 176]`` -> ``[..., nb*256]``); every
+    term is an integer multiple of 2^-24 below 2^17, so fp64 holds it exactly."""
+    d, dmin = block_d_dmin(blocks)
+    sc, m = scale_min_pairs(blocks)
+    q = quants_q5(blocks)
+    j = np.arange(QK) // SUB
+    w = d[..., None] * sc[..., j] * q - dmin[..., None] * m[..., j]
+    return w.reshape(w.shape[:-2] + (w.shape[-2] * QK,))
+
+
+def matmul_ref_q5(W_blocks: np.ndarray, X_bits: np.ndarray):
+    """``matmul_ref`` for Q5_K weights ``[N][K/256][176]``: ``(Y, S)`` in fp64."""
+    W = dequant_exact_q5(W_blocks)
+    X = bf16_to_f64(X_bits)
+    return X @ W.T, np.abs(X) @ np.abs(W).T
+
+
+def matmul_rows_ref_q5(W_blocks: np.ndarray, X_bits: np.ndarray, rows: np.ndarray):
+    return matmul_ref_q5(np.asarray(W_blocks)[rows], X_bits)
+
+
+# --------------------------------------------------------------------------
 # Dense matmul: Y[m, n] = sum_k W[n, k] * X[m, k]
 # --------------------------------------------------------------------------
 
@@ -319,6 +370,23 @@ def make_block(d: float, dmin: float, sc, m, q) -> np.ndarray:
     b[2:4] = np.array([dmin], dtype="<f2").view(np.uint8)
     b[4:16] = pack_scale_min(np.asarray(sc), np.asarray(m))
     b[16:144] = pack_quants(np.asarray(q))
+    return b
+
+
+def make_block_q5(d: float, dmin: float, sc, m, q) -> np.ndarray:
+    """Assemble one 176-byte Q5_K block from d, dmin (rounded to binary16), eight
+    (sc, m) pairs and 256 quants in 0..31 (Reading R19)."""
+    q = np.asarray(q, dtype=np.int64)
+    b = np.zeros(Q5_BLOCK_BYTES, dtype=np.uint8)
+    b[0:2] = np.array([d], dtype="<f2").view(np.uint8)
+    b[2:4] = np.array([dmin], dtype="<f2").view(np.uint8)
+    b[4:16] = pack_scale_min(np.asarray(sc), np.asarray(m))
+    qh = np.zeros(32, dtype=np.int64)
+    for c in range(4):
+        for h in range(2):
+            qh |= ((q[64 * c + 32 * h: 64 * c + 32 * h + 32] >> 4) & 1) << (2 * c + h)
+    b[16:48] = qh.astype(np.uint8)
+    b[48:176] = pack_quants(q & 15)
     return b
 
 

@@ -59,6 +59,30 @@ def q4k_random_blocks(rng: np.random.Generator, nrows: int, K: int) -> np.ndarra
     return out.reshape(nrows, K // BLOCK_WEIGHTS, BLOCK_BYTES)
 
 
+Q5_BLOCK_BYTES = 176  # bytes per Q5_K super-block
+
+
+def q5k_random_blocks(rng: np.random.Generator, nrows: int, K: int) -> np.ndarray:
+    """Random Q5_K matrix: uint8 ``[nrows][K/256][176]``, drawn like Q4_K blocks
+    (d, dmin, scale bytes) and then the 32 fifth-bit bytes and the 128 nibble
+    bytes as uniform bytes, so every five-bit quant is uniform on 0..31."""
+    if K % BLOCK_WEIGHTS:
+        raise ValueError("K must be a multiple of 256")
+    nb = nrows * (K // BLOCK_WEIGHTS)
+    d = (np.abs(rng.standard_normal(nb)) * 1e-3).astype(np.float16)
+    dmin = (np.abs(rng.standard_normal(nb)) * 1e-3).astype(np.float16)
+    sc = rng.integers(0, 256, size=(nb, 12), dtype=np.uint8)
+    qh = rng.integers(0, 256, size=(nb, 32), dtype=np.uint8)
+    qs = rng.integers(0, 256, size=(nb, 128), dtype=np.uint8)
+    out = np.empty((nb, Q5_BLOCK_BYTES), dtype=np.uint8)
+    out[:, 0:2] = d.astype("<f2").view(np.uint8).reshape(nb, 2)
+    out[:, 2:4] = dmin.astype("<f2").view(np.uint8).reshape(nb, 2)
+    out[:, 4:16] = sc
+    out[:, 16:48] = qh
+    out[:, 48:176] = qs
+    return out.reshape(nrows, K // BLOCK_WEIGHTS, Q5_BLOCK_BYTES)
+
+
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """fp32 array -> bf16 bit patterns (uint16), round to nearest even (torch CPU cast)."""
     import torch
@@ -98,6 +122,26 @@ def dense_decode(seed: int = 1, Mmax: int = 32, scale_rows: float = 1.0):
     ndn = max(16, int(ndn * scale_rows) // 16 * 16)
     Wgu = q4k_random_blocks(rng, ngu, kgu)
     Wdn = q4k_random_blocks(rng, ndn, kdn)
+    Xgu = bf16_normal(rng, (Mmax, kgu))
+    Xdn = bf16_normal(rng, (Mmax, kdn))
+    return dict(W_gate_up=Wgu, W_down=Wdn, X_gate_up=Xgu, X_down=Xdn)
+
+
+def gemv_small_q5(seed: int = 0, N: int = 256, K: int = 2048, M: int = 1):
+    """Single-matrix Q5_K GEMV case. Order: W, X."""
+    rng = np.random.default_rng(seed)
+    W = q5k_random_blocks(rng, N, K)
+    X = bf16_normal(rng, (M, K))
+    return W, X
+
+
+def dense_decode_q5(seed: int = 5, Mmax: int = 32):
+    """The dense decode shapes with Q5_K weights (gate+up 34816 x 5120, down
+    5120 x 17408). Order: W_gate_up, W_down, X_gate_up, X_down."""
+    rng = np.random.default_rng(seed)
+    (ngu, kgu), (ndn, kdn) = DENSE_DECODE["gate_up"], DENSE_DECODE["down"]
+    Wgu = q5k_random_blocks(rng, ngu, kgu)
+    Wdn = q5k_random_blocks(rng, ndn, kdn)
     Xgu = bf16_normal(rng, (Mmax, kgu))
     Xdn = bf16_normal(rng, (Mmax, kdn))
     return dict(W_gate_up=Wgu, W_down=Wdn, X_gate_up=Xgu, X_down=Xdn)

@@ -440,3 +440,85 @@ def test_repack_round_trip_and_byte_multisets():
             blk = R[n // 128, kb, n % 128]
             assert np.array_equal(blk[:16], W[n, kb, :16])
             assert np.array_equal(np.sort(blk[16:]), np.sort(W[n, kb, 16:]))
+
+
+# ------------------------------------------------------------------ Q5_K --
+
+def _scalar_weight_q5(block, i):
+    """Scalar restatement of one Q5_K weight, used only as brute force (Reading R19)."""
+    d = float(np.frombuffer(bytes(block[0:2]), "<f2")[0])
+    dmin = float(np.frombuffer(bytes(block[2:4]), "<f2")[0])
+    s = [int(v) for v in block[4:16]]
+    j = i // 32
+    if j < 4:
+        sc, m = s[j] & 63, s[j + 4] & 63
+    else:
+        sc = (s[j + 4] & 0xF) | ((s[j - 4] >> 6) << 4)
+        m = (s[j + 4] >> 4) | ((s[j] >> 6) << 4)
+    c, rem = divmod(i, 64)
+    h, l = divmod(rem, 32)
+    low = (int(block[48 + 32 * c + l]) >> (4 * h)) & 0xF
+    fifth = (int(block[16 + l]) >> (2 * c + h)) & 1
+    return d * sc * (low + 16 * fifth) - dmin * m
+
+
+def test_q5_one_hot_fifth_bits_and_nibbles():
+    """Bit 2c+h of qh[l] alone adds 16*d*sc_j to weight 64c+32h+l and to no other;
+    nibble h of byte 48+32c+l alone adds d*sc_j*v to that same weight."""
+    sc = np.arange(3, 11)
+    base = O.make_block_q5(1.0, 0.0, sc, np.zeros(8, int), np.zeros(256, int))
+    assert np.all(O.dequant_exact_q5(base[None]) == 0)
+    for c in range(4):
+        for h in range(2):
+            for l in range(32):
+                i = 64 * c + 32 * h + l
+                b = base.copy()
+                b[16 + l] = np.uint8(1 << (2 * c + h))
+                expect = np.zeros(256)
+                expect[i] = 16.0 * sc[i // 32]
+                assert np.array_equal(O.dequant_exact_q5(b[None]), expect), (c, h, l)
+                b = base.copy()
+                b[48 + 32 * c + l] = np.uint8(7 << (4 * h))
+                expect[i] = 7.0 * sc[i // 32]
+                assert np.array_equal(O.dequant_exact_q5(b[None]), expect), (c, h, l)
+
+
+def test_q5_closed_form_and_q4_agreement():
+    """All quants 31 (every nibble 15, every fifth bit set): w = d*s*31 - dmin*t.
+    With no fifth bit set a Q5_K block dequantises like the Q4_K block with the
+    same header and nibbles."""
+    for (d, dmin, s, t) in [(1e-3, 2e-3, 17, 40), (0.25, 0.125, 63, 63)]:
+        blk = O.make_block_q5(d, dmin, [s] * 8, [t] * 8, [31] * 256)
+        assert np.all(blk[16:176] == 0xFF)
+        dh, dmh = float(np.float16(d)), float(np.float16(dmin))
+        assert np.all(O.dequant_exact_q5(blk[None]) == dh * s * 31 - dmh * t)
+    rng = np.random.default_rng(11)
+    W4 = synth.q4k_random_blocks(rng, 3, 512)
+    W5 = np.zeros(W4.shape[:-1] + (176,), np.uint8)
+    W5[..., 0:16] = W4[..., 0:16]
+    W5[..., 48:176] = W4[..., 16:144]
+    np.testing.assert_array_equal(O.dequant_exact_q5(W5), O.dequant_exact(W4))
+
+
+def test_q5_encode_round_trip_and_brute_force_matmul():
+    rng = np.random.default_rng(12)
+    q = rng.integers(0, 32, 256)
+    sc, m = rng.integers(0, 64, 8), rng.integers(0, 64, 8)
+    blk = O.make_block_q5(3e-3, 1e-3, sc, m, q)
+    np.testing.assert_array_equal(O.quants_q5(blk[None])[0], q)
+    W, X = synth.gemv_small_q5(13, N=2, K=256, M=2)
+    Y, S = O.matmul_ref_q5(W, X)
+    xf = O.bf16_to_f64(X)
+    for n in range(2):
+        for t in range(2):
+            prods = [_scalar_weight_q5(W[n, 0], i) * xf[t, i] for i in range(256)]
+            assert abs(Y[t, n] - math.fsum(prods)) <= 1e-12 * math.fsum(abs(p) for p in prods)
+            assert abs(S[t, n] - math.fsum(abs(p) for p in prods)) <= 1e-12 * S[t, n]
+
+
+def test_q5_synth_quants_cover_0_to_31():
+    W, _ = synth.gemv_small_q5(14, N=64, K=512, M=1)
+    q = O.quants_q5(W)
+    assert q.min() == 0 and q.max() == 31
+    counts = np.bincount(q.ravel(), minlength=32)
+    assert counts.min() > 0.8 * counts.mean()

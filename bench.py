@@ -211,6 +211,12 @@ def build_workloads(torch, q, synth):
     W["dec_rep_copies"] = {p: [q.q4k_repack(Wt, *W["dec_shapes"][p]) for Wt in W["dec_copies"][p]]
                            for p in ("gate_up", "down")}
     W["dec_host_X"] = {p: torch.from_numpy(dd[f"X_{p}"].view(np.int16)).pin_memory() for p in ("gate_up", "down")}
+    # the same decode shapes in Q5_K (176-byte blocks): 4 x 122 MB (gate+up), 6 x 61 MB (down)
+    d5 = synth.dense_decode_q5(5)
+    W["dec_q5"] = {k: dev(v) for k, v in d5.items()}
+    W["dec_q5_copies"] = {"gate_up": [W["dec_q5"]["W_gate_up"]] + [W["dec_q5"]["W_gate_up"].clone() for _ in range(3)],
+                          "down": [W["dec_q5"]["W_down"]] + [W["dec_q5"]["W_down"].clone() for _ in range(5)]}
+    del d5
     Wp, Xp = synth.dense_prefill(2)
     W["pre"] = (dev(Wp), dev(Xp), Wp.shape[0], Wp.shape[1] * 256)
     W["pre_copies"] = [W["pre"][0]] + [W["pre"][0].clone() for _ in range(2)]
@@ -315,6 +321,11 @@ def run_step(q, tm, W):
             fns = [lambda Wr=Wr: q.q4k_gemv_repacked(Wr, Xt, N, K, Y=Y, ws=W["ws"]) for Wr in W["dec_rep_copies"][p]]
             tm.run_seq(f"gemv_rep:{p}:M{M}", fns)
             launches += 2 * len(fns)
+            if M in (1, 8, 32):  # Q5_K weights, same shapes
+                X5 = W["dec_q5"][f"X_{p}"][:M]
+                fns = [lambda Wt=Wt: q.q5k_gemv(Wt, X5, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_q5_copies"][p]]
+                tm.run_seq(f"gemv_q5:{p}:M{M}", fns)
+                launches += 2 * len(fns)
     _, Xt, N, K = W["pre"]
     for M in (512, 4096):
         Y = W["pre_Y"][:M * N].view(M, N)
@@ -391,6 +402,14 @@ def summarize(tm, W, peaks):
                 comp["_rep_time"] = rep_time
                 comp[f"gemv_repacked_{p}_M{M}_GBps"] = round(b / tr / 1e9, 1)
                 comp[f"gemv_repacked_{p}_M{M}_us"] = round(tr * 1e6, 2)
+    for M in (1, 8, 32):
+        for p in ("gate_up", "down"):
+            t5 = T.get(f"gemv_q5:{p}:M{M}")
+            if t5:  # Q5_K: 176 bytes per super-block
+                N, K = W["dec_shapes"][p]
+                b5 = N * (K // 256) * 176
+                comp[f"gemv_q5k_{p}_M{M}_GBps"] = round(b5 / t5 / 1e9, 1)
+                comp[f"gemv_q5k_{p}_M{M}_us"] = round(t5 * 1e6, 2)
     Wt, Xt, N, K = W["pre"]
     for M in (512, 4096):
         t = T[f"gemm:M{M}"]
@@ -417,6 +436,8 @@ def summarize(tm, W, peaks):
         n = 1
         if k.startswith(("gemv:", "gemv_rep:")):
             n = len(W["dec_copies"][k.split(":")[1]])
+        elif k.startswith("gemv_q5:"):
+            n = len(W["dec_q5_copies"][k.split(":")[1]])
         elif k.startswith("gemm:"):
             n = len(W["pre_copies"])
         per_step[k] = v * n

@@ -97,6 +97,18 @@ q4k_status q4k_dequant(const void* W, int64_t nblocks, int out_bf16, void* out, 
 q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* Decode GEMV over Q5_K weights, the Q4_K_M files' other large tensor family
+ * (hipEngine 0.3.0 README, "GGUF Support": the tensor-family table lists Q5_K
+ * beside Q4_K). W [N][K/256] Q5_K blocks of 176 bytes: fp16 d, fp16 dmin,
+ * the Q4_K 12-byte six-bit (sc, m) packing, 32 bytes qh, 128 bytes of low
+ * nibbles in the Q4_K order; weight 64c+32h+l = nibble h of byte 48+32c+l
+ * plus 16 x bit 2c+h of qh[l], w = d*sc*q - dmin*m with q in 0..31.
+ * Everything else -- X, Y, ws (q4k_workspace_bytes(Q4K_OP_GEMV, ...)), the
+ * shapes, errors, the arithmetic and the per-class batch invariance -- as
+ * q4k_gemv. */
+q4k_status q5k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
+                    void* ws, size_t ws_bytes, void* stream);
+
 /* Load-time repack of Q4_K weights for the decode GEMV (hipEngine 0.3.0
  * README, "GGUF Support": the decode-repacked layouts). A byte permutation:
  * the same 144 bytes per super-block, so the same HBM traffic.

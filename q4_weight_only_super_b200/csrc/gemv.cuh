@@ -93,6 +93,13 @@ __device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cas
 
 // fp16x2 (1024 + b_lo, 1024 + b_hi) from bytes `lo` and `hi` (0..3) of `word`
 // (each <= 63, so it fits the 10-bit mantissa of 1024).
+// Q5_K: bit b of bytes 0 and 2 of `w`, moved to bit `to` of each 16-bit half
+// (b and to are compile-time constants after unrolling).
+__device__ __forceinline__ uint32_t fifth_bits(uint32_t w, int b, int to) {
+  const uint32_t s = to >= b ? (w << (to - b)) : (w >> (b - to));
+  return s & (0x00010001u << to);
+}
+
 __device__ __forceinline__ uint32_t bytes_1024(uint32_t word, uint32_t lo, uint32_t hi) {
   return __byte_perm(word, 0x64u, (4u << 12) | (hi << 8) | (4u << 4) | lo);
 }
@@ -184,6 +191,11 @@ struct GemvParams {
 // super-block plus the first 16 bytes of the next (read and ignored) -- the
 // 160-byte pitch makes the per-thread 8-byte quant reads bank-conflict-free.
 constexpr int kGemvPitch = 160;
+// Q5_K super-block (Q4_K's fields plus 32 bytes of fifth bits): 176 bytes, read
+// in 176-byte boxes
+constexpr int kQ5BlockBytes = 176;
+constexpr int kQ5QhOff = 16;   // qh[32]: bit 2c+h of qh[l] is the fifth bit of weight 64c+32h+l
+constexpr int kQ5QsOff = 48;   // the 128 nibble bytes, ordered as in Q4_K
 
 // Shared memory layout (dynamic):
 //   wring [wstages][WARPS][16*TILES rows][160 B]   weight tiles (TMA destination)
@@ -195,10 +207,10 @@ constexpr int kGemvPitch = 160;
 // the stage is one bulk copy and the smem pitch the block size itself.
 constexpr int kRepackRows = 128;
 
-template <int MT, int WARPS, int TILES, bool REPACK = false>
+template <int MT, int WARPS, int TILES, bool REPACK = false, bool Q5 = false>
 struct GemvSmem {
   static constexpr int TOK = 8 * MT;
-  static constexpr int pitch = REPACK ? BLOCK_BYTES : kGemvPitch;
+  static constexpr int pitch = Q5 ? kQ5BlockBytes : (REPACK ? BLOCK_BYTES : kGemvPitch);
   static constexpr int warp_tile = 16 * TILES * pitch;
   static constexpr size_t wstage = (size_t)WARPS * warp_tile;
   static constexpr size_t xstage = (size_t)TOK * kXRec;
@@ -232,11 +244,17 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
 // GROUPED: blockIdx.y enumerates non-empty experts (the y-th expert with a
 // non-zero row count); SWIGLU: the first WARPS/2 consumer warps hold gate rows
 // and the last WARPS/2 the matching up rows (at +N/2).
-template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false>
+// Q5: Q5_K weights (176-byte super-blocks; the fifth bit of each quant is ORed
+// into the nibble field before either A form is built, so q runs to 31 and the
+// arithmetic stays exact: q*sc <= 1953 and 1024+16q <= 1520 in fp16).
+template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false, bool Q5 = false>
 __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                                    GemvParams p) {
-  using L = GemvSmem<MT, WARPS, TILES, REPACK>;
+  using L = GemvSmem<MT, WARPS, TILES, REPACK, Q5>;
   static_assert(!REPACK || (!GROUPED && 16 * TILES * WARPS == kRepackRows), "repacked: dense, 128-row tiles");
+  static_assert(!Q5 || (!GROUPED && !REPACK), "Q5_K: dense raw layout");
+  constexpr int BB = Q5 ? kQ5BlockBytes : BLOCK_BYTES;  // bytes per super-block
+  constexpr int QO = Q5 ? kQ5QsOff : 16;                 // offset of the nibble bytes
   constexpr int TOK = 8 * MT;
   // 1..16 tokens: the subnormal-nibble A operand with per-sub-block scaling after the
   // MMA (fewer instructions per weight); 17..32: fp16 sc*q built before the MMA
@@ -332,7 +350,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         if (*abort_flag) break;
         mbar_arrive_expect_tx(wfull(s), (uint32_t)(WARPS * L::warp_tile));
         const uint32_t dst = smem_u32(smem) + (uint32_t)(s * L::wstage);
-        const int x = (kb0 + ks) * BLOCK_BYTES;
+        const int x = (kb0 + ks) * BB;
         if (REPACK) {  // the tile's super-block column is one contiguous 18 KB run
           const uint8_t* src = p.W + ((size_t)tile * p.nkb + (kb0 + ks)) * (size_t)L::wstage;
           bulk_copy_g2s(dst, src, (uint32_t)L::wstage, wfull(s));
@@ -404,6 +422,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
       uint32_t hdx[R];
       uint32_t scw[R][2], mnw[R][2];
       uint2 qv[R][4];  // [row][chunk]
+      uint2 qhv[R];    // Q5: this thread's fifth-bit bytes qh[8t .. 8t+7] of each row
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const uint8_t* rp = wt + (g + 8 * r) * L::pitch;
@@ -419,8 +438,9 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           qv[r][3] = make_uint2(q23.z, q23.w);
         } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) qv[r][c] = *reinterpret_cast<const uint2*>(rp + 16 + 32 * c + 8 * t);
+          for (int c = 0; c < 4; ++c) qv[r][c] = *reinterpret_cast<const uint2*>(rp + QO + 32 * c + 8 * t);
         }
+        if (Q5) qhv[r] = *reinterpret_cast<const uint2*>(rp + kQ5QhOff + 8 * t);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(wempty(sw));  // the weight tile is in registers: release it
@@ -444,6 +464,20 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           for (int h = 0; h < 2; ++h) {
             const int j = 2 * c + h;  // sub-block
             const uint32_t msk = h ? 0x00F000F0u : 0x000F000Fu;
+            // Q5: fifth bits of the four weights in bytes {0,2} (e = 0) and {1,3} (e = 1) of
+            // each quant word, at bit 4 (low nibbles: q + 16*bit) or 8 (high: 16q + 256*bit)
+            uint32_t hb[R][2][2];  // [row][k-step][byte pair]
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+              for (int st = 0; st < 2; ++st) {
+                hb[r][st][0] = hb[r][st][1] = 0u;
+                if (Q5) {
+                  const uint32_t wq = st ? qhv[r].y : qhv[r].x;
+                  hb[r][st][0] = fifth_bits(wq, j, 4 + 4 * h);
+                  hb[r][st][1] = fifth_bits(wq >> 8, j, 4 + 4 * h);
+                }
+              }
             if (SUBN) {
               // A = the raw nibble field as fp16 bits: q * 2^-24 (low nibble) or 16q * 2^-24
               // (high), fp16 subnormals, which the tensor core multiplies exactly. The
@@ -462,10 +496,10 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
                 const int ra = 2 * tt, rb = 2 * tt + 1;
 #pragma unroll
                 for (int st = 0; st < 2; ++st) {
-                  A[tt][st][0] = (st ? qv[ra][c].y : qv[ra][c].x) & msk;
-                  A[tt][st][1] = (st ? qv[rb][c].y : qv[rb][c].x) & msk;
-                  A[tt][st][2] = qs8[ra][st] & msk;
-                  A[tt][st][3] = qs8[rb][st] & msk;
+                  A[tt][st][0] = and_or((st ? qv[ra][c].y : qv[ra][c].x), msk, hb[ra][st][0]);
+                  A[tt][st][1] = and_or((st ? qv[rb][c].y : qv[rb][c].x), msk, hb[rb][st][0]);
+                  A[tt][st][2] = and_or(qs8[ra][st], msk, hb[ra][st][1]);
+                  A[tt][st][3] = and_or(qs8[rb][st], msk, hb[rb][st][1]);
                 }
               }
 #pragma unroll
@@ -509,10 +543,10 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
               for (int st = 0; st < 2; ++st) {
                 const uint32_t wa = st ? qv[ra][c].y : qv[ra][c].x, wb = st ? qv[rb][c].y : qv[rb][c].x;
                 const uint32_t sa = qs8[ra][st], sbw = qs8[rb][st];
-                A[tt][st][0] = h2_bits(__hfma2(bits_h2(and_or(wa, msk, 0x64006400u)), mul[ra], cst[ra]));
-                A[tt][st][1] = h2_bits(__hfma2(bits_h2(and_or(wb, msk, 0x64006400u)), mul[rb], cst[rb]));
-                A[tt][st][2] = h2_bits(__hfma2(bits_h2(and_or(sa, msk, 0x64006400u)), mul[ra], cst[ra]));
-                A[tt][st][3] = h2_bits(__hfma2(bits_h2(and_or(sbw, msk, 0x64006400u)), mul[rb], cst[rb]));
+                A[tt][st][0] = h2_bits(__hfma2(bits_h2(and_or(wa, msk, 0x64006400u | hb[ra][st][0])), mul[ra], cst[ra]));
+                A[tt][st][1] = h2_bits(__hfma2(bits_h2(and_or(wb, msk, 0x64006400u | hb[rb][st][0])), mul[rb], cst[rb]));
+                A[tt][st][2] = h2_bits(__hfma2(bits_h2(and_or(sa, msk, 0x64006400u | hb[ra][st][1])), mul[ra], cst[ra]));
+                A[tt][st][3] = h2_bits(__hfma2(bits_h2(and_or(sbw, msk, 0x64006400u | hb[rb][st][1])), mul[rb], cst[rb]));
               }
             }
 #pragma unroll
@@ -664,12 +698,12 @@ inline int64_t repacked_bytes(int N, int K) {
 // Raw Q4_K rows as bytes [rows][row_bytes], box 160 bytes x box_rows rows (one super-block
 // per row plus 16 bytes of the next; past the end of a row the box reads zeros).
 inline bool make_tmap_w_rowgroup(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes,
-                                 int box_rows) {
+                                 int box_rows, int box_bytes = kGemvPitch) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  cuuint32_t box[2] = {(cuuint32_t)kGemvPitch, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,

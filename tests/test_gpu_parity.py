@@ -116,6 +116,49 @@ def test_gemv_batch_invariance_and_determinism(decode_inputs):
     assert torch.equal(q.q4k_gemv(W, X[13:30], N, K), y32[13:30])
 
 
+# ---------------------------------------------------------------- Q5_K GEMV --
+
+@pytest.mark.parametrize("N,K", [(16, 256), (48, 512), (272, 4096), (1040, 256 * 69)])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 17, 32])
+def test_q5k_gemv_shapes(N, K, M):
+    W, X = synth.gemv_small_q5(400 + M, N=N, K=K, M=M)
+    y = host(q.q5k_gemv(dev(W), dev(X), N, K))
+    Y, S = O.matmul_ref_q5(W, X)
+    _assert_tol(y, Y, S, f"Q5_K N={N} K={K} M={M}")
+
+
+def test_q5k_gemv_without_fifth_bits_equals_q4k():
+    """A Q5_K matrix whose fifth bits are all zero holds the same weights as the
+    Q4_K matrix with the same header and nibbles; both GEMVs take the same
+    arithmetic in the same order, so the results are bit-identical."""
+    W4, X = synth.gemv_small(410, N=272, K=4096, M=32)
+    W5 = np.zeros(W4.shape[:-1] + (176,), np.uint8)
+    W5[..., 0:16] = W4[..., 0:16]
+    W5[..., 48:176] = W4[..., 16:144]
+    W4d, W5d, Xd = dev(W4), dev(W5), dev(X)
+    for M in (1, 9, 17, 32):
+        assert torch.equal(q.q5k_gemv(W5d, Xd[:M], 272, 4096), q.q4k_gemv(W4d, Xd[:M], 272, 4096)), M
+
+
+@pytest.fixture(scope="module")
+def decode_inputs_q5():
+    inp = synth.dense_decode_q5(5)
+    d = {k: dev(v) for k, v in inp.items()}
+    return inp, d
+
+
+@pytest.mark.parametrize("proj", ["gate_up", "down"])
+@pytest.mark.parametrize("M", [1, 8, 16, 32])
+def test_q5k_gemv_dense_decode_sampled(decode_inputs_q5, proj, M):
+    inp, d = decode_inputs_q5
+    W, X = inp[f"W_{proj}"], inp[f"X_{proj}"][:M]
+    N, K = W.shape[0], W.shape[1] * 256
+    y = host(q.q5k_gemv(d[f"W_{proj}"], d[f"X_{proj}"][:M], N, K))
+    rows = sample_rows(N, 384, seed=50 + M)
+    Y, S = O.matmul_rows_ref_q5(W, X, rows)
+    _assert_tol(y[:, rows], Y, S, f"Q5_K {proj} M={M}")
+
+
 # ------------------------------------------------------------ decode repack --
 
 @pytest.mark.parametrize("N,K", [(16, 256), (200, 512), (1040, 256 * 69)])

@@ -174,6 +174,45 @@ def matmul_rows_ref_q5(W_blocks: np.ndarray, X_bits: np.ndarray, rows: np.ndarra
 
 
 # --------------------------------------------------------------------------
+# Q8_0 block (sibling quant; the same tensor-family table). Reading R20: the
+# llama.cpp-style block of 32 weights in 34 bytes -- fp16 d (little-endian),
+# then 32 signed bytes q (two's complement) -- with w = d * q. A row of K
+# weights is K/32 consecutive blocks.
+# --------------------------------------------------------------------------
+
+Q80_BLOCK_BYTES = 34
+Q80_WEIGHTS = 32
+
+
+def dequant_exact_q80(blocks: np.ndarray) -> np.ndarray:
+    """Exact Q8_0 weights in fp64: ``[..., nb, 34]`` -> ``[..., nb*32]`` (d*q is exact)."""
+    b = np.ascontiguousarray(blocks, dtype=np.uint8)
+    d = b[..., 0:2].copy().view("<f2")[..., 0].astype(np.float64)
+    q = b[..., 2:34].view(np.int8).astype(np.float64)
+    w = d[..., None] * q
+    return w.reshape(w.shape[:-2] + (w.shape[-2] * Q80_WEIGHTS,))
+
+
+def matmul_ref_q80(W_blocks: np.ndarray, X_bits: np.ndarray):
+    """``matmul_ref`` for Q8_0 weights ``[N][K/32][34]``: ``(Y, S)`` in fp64."""
+    W = dequant_exact_q80(W_blocks)
+    X = bf16_to_f64(X_bits)
+    return X @ W.T, np.abs(X) @ np.abs(W).T
+
+
+def matmul_rows_ref_q80(W_blocks: np.ndarray, X_bits: np.ndarray, rows: np.ndarray):
+    return matmul_ref_q80(np.asarray(W_blocks)[rows], X_bits)
+
+
+def make_block_q80(d: float, q) -> np.ndarray:
+    """One 34-byte Q8_0 block from d (rounded to binary16) and 32 values in -128..127."""
+    b = np.zeros(Q80_BLOCK_BYTES, dtype=np.uint8)
+    b[0:2] = np.array([d], dtype="<f2").view(np.uint8)
+    b[2:34] = np.asarray(q, dtype=np.int64).astype(np.int8).view(np.uint8)
+    return b
+
+
+# --------------------------------------------------------------------------
 # Dense matmul: Y[m, n] = sum_k W[n, k] * X[m, k]
 # --------------------------------------------------------------------------
 

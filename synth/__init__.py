@@ -83,6 +83,24 @@ def q5k_random_blocks(rng: np.random.Generator, nrows: int, K: int) -> np.ndarra
     return out.reshape(nrows, K // BLOCK_WEIGHTS, Q5_BLOCK_BYTES)
 
 
+Q80_BLOCK_BYTES = 34  # bytes per Q8_0 block of 32 weights
+
+
+def q80_random_blocks(rng: np.random.Generator, nrows: int, K: int) -> np.ndarray:
+    """Random Q8_0 matrix: uint8 ``[nrows][K/32][34]``. Draw order: d (as for
+    Q4_K blocks), then the 32 quant bytes of every block as uniform bytes (each
+    signed quant uniform on -128..127)."""
+    if K % BLOCK_WEIGHTS:
+        raise ValueError("K must be a multiple of 256")
+    nb = nrows * (K // 32)
+    d = (np.abs(rng.standard_normal(nb)) * 1e-3).astype(np.float16)
+    qs = rng.integers(0, 256, size=(nb, 32), dtype=np.uint8)
+    out = np.empty((nb, Q80_BLOCK_BYTES), dtype=np.uint8)
+    out[:, 0:2] = d.astype("<f2").view(np.uint8).reshape(nb, 2)
+    out[:, 2:34] = qs
+    return out.reshape(nrows, K // 32, Q80_BLOCK_BYTES)
+
+
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """fp32 array -> bf16 bit patterns (uint16), round to nearest even (torch CPU cast)."""
     import torch
@@ -142,6 +160,25 @@ def dense_decode_q5(seed: int = 5, Mmax: int = 32):
     (ngu, kgu), (ndn, kdn) = DENSE_DECODE["gate_up"], DENSE_DECODE["down"]
     Wgu = q5k_random_blocks(rng, ngu, kgu)
     Wdn = q5k_random_blocks(rng, ndn, kdn)
+    Xgu = bf16_normal(rng, (Mmax, kgu))
+    Xdn = bf16_normal(rng, (Mmax, kdn))
+    return dict(W_gate_up=Wgu, W_down=Wdn, X_gate_up=Xgu, X_down=Xdn)
+
+
+def gemv_small_q80(seed: int = 0, N: int = 256, K: int = 2048, M: int = 1):
+    """Single-matrix Q8_0 GEMV case. Order: W, X."""
+    rng = np.random.default_rng(seed)
+    W = q80_random_blocks(rng, N, K)
+    X = bf16_normal(rng, (M, K))
+    return W, X
+
+
+def dense_decode_q80(seed: int = 6, Mmax: int = 32):
+    """The dense decode shapes with Q8_0 weights. Order: W_gate_up, W_down, X_gate_up, X_down."""
+    rng = np.random.default_rng(seed)
+    (ngu, kgu), (ndn, kdn) = DENSE_DECODE["gate_up"], DENSE_DECODE["down"]
+    Wgu = q80_random_blocks(rng, ngu, kgu)
+    Wdn = q80_random_blocks(rng, ndn, kdn)
     Xgu = bf16_normal(rng, (Mmax, kgu))
     Xdn = bf16_normal(rng, (Mmax, kdn))
     return dict(W_gate_up=Wgu, W_down=Wdn, X_gate_up=Xgu, X_down=Xdn)

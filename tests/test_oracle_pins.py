@@ -522,3 +522,45 @@ def test_q5_synth_quants_cover_0_to_31():
     assert q.min() == 0 and q.max() == 31
     counts = np.bincount(q.ravel(), minlength=32)
     assert counts.min() > 0.8 * counts.mean()
+
+
+# ------------------------------------------------------------------ Q8_0 --
+
+def test_q80_one_hot_and_signs():
+    """A block with one nonzero quant v at position l gives w = d*v at weight 32b+l
+    only; the sign follows two's complement (byte 0x80 is -128, 0xFF is -1)."""
+    for l in (0, 1, 17, 31):
+        for v, byte in ((1, 0x01), (127, 0x7F), (-1, 0xFF), (-128, 0x80)):
+            blk = np.zeros(34, np.uint8)
+            blk[0:2] = np.array([0.5], dtype="<f2").view(np.uint8)
+            blk[2 + l] = byte
+            W = np.stack([np.zeros(34, np.uint8), blk])[None]  # one row, two blocks
+            W[0, 0, 0:2] = np.array([1.0], dtype="<f2").view(np.uint8)
+            w = O.dequant_exact_q80(W)[0]
+            expect = np.zeros(64)
+            expect[32 + l] = 0.5 * v
+            assert np.array_equal(w, expect), (l, v)
+
+
+def test_q80_encode_closed_form_and_brute_force():
+    rng = np.random.default_rng(15)
+    q = rng.integers(-128, 128, 32)
+    blk = O.make_block_q80(3e-3, q)
+    dh = float(np.float16(3e-3))
+    np.testing.assert_array_equal(O.dequant_exact_q80(blk[None]), dh * q)
+    W, X = synth.gemv_small_q80(16, N=2, K=256, M=2)
+    Y, S = O.matmul_ref_q80(W, X)
+    xf = O.bf16_to_f64(X)
+    for n in range(2):
+        for t in range(2):
+            prods = []
+            for i in range(256):
+                b = W[n, i // 32]
+                d = float(np.frombuffer(bytes(b[0:2]), "<f2")[0])
+                qv = int(b[2 + i % 32])
+                qv = qv - 256 if qv >= 128 else qv
+                prods.append(d * qv * xf[t, i])
+            assert abs(Y[t, n] - math.fsum(prods)) <= 1e-12 * math.fsum(abs(p) for p in prods)
+    Wq, _ = synth.gemv_small_q80(17, N=64, K=512, M=1)
+    qv = Wq[..., 2:34].view(np.int8)
+    assert qv.min() == -128 and qv.max() == 127

@@ -217,6 +217,12 @@ def build_workloads(torch, q, synth):
     W["dec_q5_copies"] = {"gate_up": [W["dec_q5"]["W_gate_up"]] + [W["dec_q5"]["W_gate_up"].clone() for _ in range(3)],
                           "down": [W["dec_q5"]["W_down"]] + [W["dec_q5"]["W_down"].clone() for _ in range(5)]}
     del d5
+    # and in Q8_0 (34-byte blocks of 32): 2 x 189 MB (gate+up), 3 x 95 MB (down)
+    d8 = synth.dense_decode_q80(6)
+    W["dec_q80"] = {k: dev(v) for k, v in d8.items()}
+    W["dec_q80_copies"] = {"gate_up": [W["dec_q80"]["W_gate_up"], W["dec_q80"]["W_gate_up"].clone()],
+                           "down": [W["dec_q80"]["W_down"]] + [W["dec_q80"]["W_down"].clone() for _ in range(2)]}
+    del d8
     Wp, Xp = synth.dense_prefill(2)
     W["pre"] = (dev(Wp), dev(Xp), Wp.shape[0], Wp.shape[1] * 256)
     W["pre_copies"] = [W["pre"][0]] + [W["pre"][0].clone() for _ in range(2)]
@@ -326,6 +332,10 @@ def run_step(q, tm, W):
                 fns = [lambda Wt=Wt: q.q5k_gemv(Wt, X5, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_q5_copies"][p]]
                 tm.run_seq(f"gemv_q5:{p}:M{M}", fns)
                 launches += 2 * len(fns)
+                X8 = W["dec_q80"][f"X_{p}"][:M]
+                fns = [lambda Wt=Wt: q.q80_gemv(Wt, X8, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_q80_copies"][p]]
+                tm.run_seq(f"gemv_q80:{p}:M{M}", fns)
+                launches += 2 * len(fns)
     _, Xt, N, K = W["pre"]
     for M in (512, 4096):
         Y = W["pre_Y"][:M * N].view(M, N)
@@ -410,6 +420,12 @@ def summarize(tm, W, peaks):
                 b5 = N * (K // 256) * 176
                 comp[f"gemv_q5k_{p}_M{M}_GBps"] = round(b5 / t5 / 1e9, 1)
                 comp[f"gemv_q5k_{p}_M{M}_us"] = round(t5 * 1e6, 2)
+            t8 = T.get(f"gemv_q80:{p}:M{M}")
+            if t8:  # Q8_0: 34 bytes per 32 weights
+                N, K = W["dec_shapes"][p]
+                b8 = N * (K // 32) * 34
+                comp[f"gemv_q80_{p}_M{M}_GBps"] = round(b8 / t8 / 1e9, 1)
+                comp[f"gemv_q80_{p}_M{M}_us"] = round(t8 * 1e6, 2)
     Wt, Xt, N, K = W["pre"]
     for M in (512, 4096):
         t = T[f"gemm:M{M}"]
@@ -438,6 +454,8 @@ def summarize(tm, W, peaks):
             n = len(W["dec_copies"][k.split(":")[1]])
         elif k.startswith("gemv_q5:"):
             n = len(W["dec_q5_copies"][k.split(":")[1]])
+        elif k.startswith("gemv_q80:"):
+            n = len(W["dec_q80_copies"][k.split(":")[1]])
         elif k.startswith("gemm:"):
             n = len(W["pre_copies"])
         per_step[k] = v * n

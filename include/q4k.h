@@ -109,6 +109,17 @@ q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
 q4k_status q5k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* Decode GEMV over Q8_0 weights (the same tensor-family table lists Q8_0).
+ * W [N][K/32] blocks of 34 bytes: fp16 d (little-endian), then 32 two's-
+ * complement bytes q; w = d*q. K % 256 == 0 (the GEMV reads eight blocks per
+ * 256-wide column). Everything else -- X, Y, ws (q4k_workspace_bytes(
+ * Q4K_OP_GEMV, ...)), shapes, errors, the activation pre-pass -- as q4k_gemv;
+ * each block's 32 products enter exactly (q + 128 as an fp16 subnormal, the
+ * -128 offset through the block's activation sum) and accumulate in fp32.
+ * Row m of the result does not depend on the other rows of X at any M. */
+q4k_status q80_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
+                    void* ws, size_t ws_bytes, void* stream);
+
 /* Load-time repack of Q4_K weights for the decode GEMV (hipEngine 0.3.0
  * README, "GGUF Support": the decode-repacked layouts). A byte permutation:
  * the same 144 bytes per super-block, so the same HBM traffic.

@@ -196,6 +196,12 @@ constexpr int kGemvPitch = 160;
 constexpr int kQ5BlockBytes = 176;
 constexpr int kQ5QhOff = 16;   // qh[32]: bit 2c+h of qh[l] is the fifth bit of weight 64c+32h+l
 constexpr int kQ5QsOff = 48;   // the 128 nibble bytes, ordered as in Q4_K
+// Q8_0: blocks of 32 weights in 34 bytes (fp16 d, then 32 signed bytes); the
+// GEMV reads them eight at a time (one 256-wide column of the matrix, 272 bytes
+// per row), and block j of a group plays the part of Q4_K's sub-block j
+constexpr int kQ80GroupBytes = 272;
+// weight formats of the GEMV kernel
+constexpr int kQtQ4K = 0, kQtQ5K = 1, kQtQ80 = 2;
 
 // Shared memory layout (dynamic):
 //   wring [wstages][WARPS][16*TILES rows][160 B]   weight tiles (TMA destination)
@@ -207,17 +213,24 @@ constexpr int kQ5QsOff = 48;   // the 128 nibble bytes, ordered as in Q4_K
 // the stage is one bulk copy and the smem pitch the block size itself.
 constexpr int kRepackRows = 128;
 
-template <int MT, int WARPS, int TILES, bool REPACK = false, bool Q5 = false>
+template <int MT, int WARPS, int TILES, bool REPACK = false, int QT = kQtQ4K>
 struct GemvSmem {
   static constexpr int TOK = 8 * MT;
-  static constexpr int pitch = Q5 ? kQ5BlockBytes : (REPACK ? BLOCK_BYTES : kGemvPitch);
+  static constexpr int pitch =
+      QT == kQtQ80 ? kQ80GroupBytes : (QT == kQtQ5K ? kQ5BlockBytes : (REPACK ? BLOCK_BYTES : kGemvPitch));
+  // Q8_0 (272-byte rows): the reduction buffer lies in the weight ring, which is
+  // free once every stage has been consumed, so 32 tokens still fit two CTAs per SM
+  static constexpr bool red_in_ring = QT == kQtQ80;
+  static constexpr size_t red_bytes = (size_t)16 * TILES * WARPS * TOK * 4;
   static constexpr int warp_tile = 16 * TILES * pitch;
   static constexpr size_t wstage = (size_t)WARPS * warp_tile;
   static constexpr size_t xstage = (size_t)TOK * kXRec;
   static constexpr __host__ __device__ size_t xring_off(int ws) { return (size_t)ws * wstage; }
-  static constexpr __host__ __device__ size_t red_off(int ws, int xsn) { return xring_off(ws) + (size_t)xsn * xstage; }
+  static constexpr __host__ __device__ size_t red_off(int ws, int xsn) {
+    return red_in_ring ? 0 : xring_off(ws) + (size_t)xsn * xstage;
+  }
   static constexpr __host__ __device__ size_t bar_off(int ws, int xsn) {
-    return red_off(ws, xsn) + (size_t)16 * TILES * WARPS * TOK * 4;
+    return xring_off(ws) + (size_t)xsn * xstage + (red_in_ring ? 0 : red_bytes);
   }
   static constexpr __host__ __device__ size_t total(int ws, int xsn) { return bar_off(ws, xsn) + 16 * (ws + xsn) + 16; }
 };
@@ -244,22 +257,28 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
 // GROUPED: blockIdx.y enumerates non-empty experts (the y-th expert with a
 // non-zero row count); SWIGLU: the first WARPS/2 consumer warps hold gate rows
 // and the last WARPS/2 the matching up rows (at +N/2).
-// Q5: Q5_K weights (176-byte super-blocks; the fifth bit of each quant is ORed
-// into the nibble field before either A form is built, so q runs to 31 and the
-// arithmetic stays exact: q*sc <= 1953 and 1024+16q <= 1520 in fp16).
-template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false, bool Q5 = false>
+// QT: the weight format.
+//  * Q5_K (176-byte super-blocks): the fifth bit of each quant is ORed into the
+//    nibble field before either A form is built, so q runs to 31 and the
+//    arithmetic stays exact (q*sc <= 1953 and 1024+16q <= 1520 in fp16).
+//  * Q8_0 (eight 34-byte blocks per 256-wide column): the subnormal form at
+//    every token count with A = q + 128 (0..255, the byte with its sign bit
+//    flipped), the block's d as the sub-block scale, and the -128 offset taken
+//    by the min-term MMA (A = d_j, against the sub-block sums, times 128).
+template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false, int QT = kQtQ4K>
 __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                                    GemvParams p) {
-  using L = GemvSmem<MT, WARPS, TILES, REPACK, Q5>;
+  using L = GemvSmem<MT, WARPS, TILES, REPACK, QT>;
   static_assert(!REPACK || (!GROUPED && 16 * TILES * WARPS == kRepackRows), "repacked: dense, 128-row tiles");
-  static_assert(!Q5 || (!GROUPED && !REPACK), "Q5_K: dense raw layout");
-  constexpr int BB = Q5 ? kQ5BlockBytes : BLOCK_BYTES;  // bytes per super-block
-  constexpr int QO = Q5 ? kQ5QsOff : 16;                 // offset of the nibble bytes
+  static_assert(QT == kQtQ4K || (!GROUPED && !REPACK), "Q5_K, Q8_0: dense raw layout");
+  constexpr bool Q5 = QT == kQtQ5K, Q80 = QT == kQtQ80;
+  constexpr int BB = Q80 ? kQ80GroupBytes : (Q5 ? kQ5BlockBytes : BLOCK_BYTES);  // bytes per 256-wide column
+  constexpr int QO = Q5 ? kQ5QsOff : 16;                                         // offset of the nibble bytes
   constexpr int TOK = 8 * MT;
   // 1..16 tokens: the subnormal-nibble A operand with per-sub-block scaling after the
   // MMA (fewer instructions per weight); 17..32: fp16 sc*q built before the MMA
   // (the per-result scaling would grow with the token groups).
-  constexpr bool SUBN = MT <= 2;
+  constexpr bool SUBN = Q80 || MT <= 2;
   constexpr int WROWS = 16 * TILES;    // weight rows per consumer warp
   constexpr int ROWS = WROWS * WARPS;  // weight rows per CTA
   extern __shared__ __align__(128) uint8_t smem[];
@@ -350,7 +369,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         if (*abort_flag) break;
         mbar_arrive_expect_tx(wfull(s), (uint32_t)(WARPS * L::warp_tile));
         const uint32_t dst = smem_u32(smem) + (uint32_t)(s * L::wstage);
-        const int x = (kb0 + ks) * BB;
+        const int x = (kb0 + ks) * BB / (Q80 ? 2 : 1);  // Q8_0: 16-bit elements (272 bytes = 136)
         if (REPACK) {  // the tile's super-block column is one contiguous 18 KB run
           const uint8_t* src = p.W + ((size_t)tile * p.nkb + (kb0 + ks)) * (size_t)L::wstage;
           bulk_copy_g2s(dst, src, (uint32_t)L::wstage, wfull(s));
@@ -416,6 +435,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     uint32_t pw = 0, px = 0;  // ring stage indices and phase parities (no divisions)
     for (int ks = 0; ks < nk; ++ks) {
       mbar_wait(wfull(sw), pw, abort_flag);
+      const int sw_cur = sw;
       const uint8_t* wt = smem + sw * L::wstage + warp * L::warp_tile;
       // rows g, g+8 (tile 0), g+16, g+24 (tile 1), ... of this warp's rows
       constexpr int R = 2 * TILES;
@@ -424,7 +444,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
       uint2 qv[R][4];  // [row][chunk]
       uint2 qhv[R];    // Q5: this thread's fifth-bit bytes qh[8t .. 8t+7] of each row
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
+      for (int r = 0; r < (Q80 ? 0 : R); ++r) {  // Q8_0 reads its blocks sub-block by sub-block below
         const uint8_t* rp = wt + (g + 8 * r) * L::pitch;
         const uint4 hd = *reinterpret_cast<const uint4*>(rp);
         hdx[r] = hd.x;
@@ -442,8 +462,10 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         }
         if (Q5) qhv[r] = *reinterpret_cast<const uint2*>(rp + kQ5QhOff + 8 * t);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(wempty(sw));  // the weight tile is in registers: release it
+      if (!Q80) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(wempty(sw));  // the weight tile is in registers: release it
+      }
       if (++sw == SW) {
         sw = 0;
         pw ^= 1u;
@@ -484,22 +506,59 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
               // sub-block's two k-steps accumulate on their own; its scale, sc (sc/16 for
               // high nibbles) as an exact fp32, is applied to the per-row results.
               float fs[R];
-#pragma unroll
-              for (int r = 0; r < R; ++r) {  // 0x4B0000sc = 2^23 + sc; 0x490000sc = 2^19 + sc/16
-                const uint32_t bits = __byte_perm(scw[r][j >> 2], h ? 0x49000000u : 0x4B000000u,
-                                                  0x7650u | (uint32_t)(j & 3));
-                fs[r] = __uint_as_float(bits) - (h ? 524288.f : 8388608.f);
-              }
               uint32_t A[TILES][2][4];
+              if (Q80) {
+                // block j of this 256-wide column: fp16 d at byte 34j, q[8t .. 8t+7] at
+                // 34j + 2 + 8t (4-byte aligned for odd j; for even j two funnel shifts
+                // realign three aligned words), each byte's sign bit flipped: q + 128
+                uint32_t xw[R][2];
 #pragma unroll
-              for (int tt = 0; tt < TILES; ++tt) {
-                const int ra = 2 * tt, rb = 2 * tt + 1;
+                for (int r = 0; r < R; ++r) {
+                  const uint8_t* rp = wt + (g + 8 * r) * L::pitch;
+                  const uint32_t dw = *reinterpret_cast<const uint32_t*>(rp + ((34 * j) & ~3));
+                  fs[r] = half_bits_to_float((j & 1) ? (dw >> 16) : (dw & 0xFFFFu));
+                  const int base = 34 * j + 2 + 8 * t;
+                  if (j & 1) {
+                    xw[r][0] = *reinterpret_cast<const uint32_t*>(rp + base);
+                    xw[r][1] = *reinterpret_cast<const uint32_t*>(rp + base + 4);
+                  } else {
+                    const uint32_t w0 = *reinterpret_cast<const uint32_t*>(rp + base - 2);
+                    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(rp + base + 2);
+                    const uint32_t w2 = *reinterpret_cast<const uint32_t*>(rp + base + 6);
+                    xw[r][0] = __funnelshift_r(w0, w1, 16);
+                    xw[r][1] = __funnelshift_r(w1, w2, 16);
+                  }
+                  xw[r][0] ^= 0x80808080u;
+                  xw[r][1] ^= 0x80808080u;
+                }
 #pragma unroll
-                for (int st = 0; st < 2; ++st) {
-                  A[tt][st][0] = and_or((st ? qv[ra][c].y : qv[ra][c].x), msk, hb[ra][st][0]);
-                  A[tt][st][1] = and_or((st ? qv[rb][c].y : qv[rb][c].x), msk, hb[rb][st][0]);
-                  A[tt][st][2] = and_or(qs8[ra][st], msk, hb[ra][st][1]);
-                  A[tt][st][3] = and_or(qs8[rb][st], msk, hb[rb][st][1]);
+                for (int tt = 0; tt < TILES; ++tt) {
+                  const int ra = 2 * tt, rb = 2 * tt + 1;
+#pragma unroll
+                  for (int st = 0; st < 2; ++st) {  // bytes {0,2} and {1,3} into the low byte of each half
+                    A[tt][st][0] = __byte_perm(xw[ra][st], 0u, 0x4240u);
+                    A[tt][st][1] = __byte_perm(xw[rb][st], 0u, 0x4240u);
+                    A[tt][st][2] = __byte_perm(xw[ra][st], 0u, 0x4341u);
+                    A[tt][st][3] = __byte_perm(xw[rb][st], 0u, 0x4341u);
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {  // 0x4B0000sc = 2^23 + sc; 0x490000sc = 2^19 + sc/16
+                  const uint32_t bits = __byte_perm(scw[r][j >> 2], h ? 0x49000000u : 0x4B000000u,
+                                                    0x7650u | (uint32_t)(j & 3));
+                  fs[r] = __uint_as_float(bits) - (h ? 524288.f : 8388608.f);
+                }
+#pragma unroll
+                for (int tt = 0; tt < TILES; ++tt) {
+                  const int ra = 2 * tt, rb = 2 * tt + 1;
+#pragma unroll
+                  for (int st = 0; st < 2; ++st) {
+                    A[tt][st][0] = and_or((st ? qv[ra][c].y : qv[ra][c].x), msk, hb[ra][st][0]);
+                    A[tt][st][1] = and_or((st ? qv[rb][c].y : qv[rb][c].x), msk, hb[rb][st][0]);
+                    A[tt][st][2] = and_or(qs8[ra][st], msk, hb[ra][st][1]);
+                    A[tt][st][3] = and_or(qs8[rb][st], msk, hb[rb][st][1]);
+                  }
                 }
               }
 #pragma unroll
@@ -567,15 +626,23 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         uint32_t am[R];
         const uint32_t mb = 2u * (t & 1);
 #pragma unroll
-        for (int r = 0; r < R; ++r)
-          am[r] = h2_bits(__hadd2(bits_h2(bytes_1024((t >> 1) ? mnw[r][1] : mnw[r][0], mb, mb + 1)),
-                                  neg1024));
+        for (int r = 0; r < R; ++r) {
+          if (Q80) {  // A = (d_2t, d_2t+1): the fp16 scales at bytes 68t and 68t + 34
+            const uint8_t* rp = wt + (g + 8 * r) * L::pitch;
+            const uint32_t wlo = *reinterpret_cast<const uint32_t*>(rp + 68 * t);
+            const uint32_t whi = *reinterpret_cast<const uint32_t*>(rp + 68 * t + 32);
+            am[r] = __byte_perm(wlo, whi, 0x7610u);
+          } else {
+            am[r] = h2_bits(__hadd2(bits_h2(bytes_1024((t >> 1) ? mnw[r][1] : mnw[r][0], mb, mb + 1)),
+                                    neg1024));
+          }
+        }
         float dd[R], dn[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           // the subnormal form's products carry 2^-24: fold 2^24 into d
-          dd[r] = (SUBN ? 16777216.f : 1.f) * half_bits_to_float(hdx[r]);
-          dn[r] = 64.f * half_bits_to_float(hdx[r] >> 16);
+          dd[r] = Q80 ? 16777216.f : (SUBN ? 16777216.f : 1.f) * half_bits_to_float(hdx[r]);
+          dn[r] = Q80 ? 64.f * 128.f : 64.f * half_bits_to_float(hdx[r] >> 16);
         }
 #pragma unroll
         for (int f = 0; f < MT; ++f) {
@@ -598,6 +665,10 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           }
         }
       }
+      if (Q80) {  // the weight stage was read until here
+        __syncwarp();
+        if (lane == 0) mbar_arrive(wempty(sw_cur));
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(xempty(sx));
       if (++sx == SX) {
@@ -607,6 +678,8 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     }
 
     // ---- CTA partial -> shared memory, token-major: red[token][local row] ----
+    // (in the weight ring for Q8_0: wait until every consumer warp is past its last stage)
+    if (L::red_in_ring) asm volatile("bar.sync 1, %0;" ::"n"(32 * WARPS) : "memory");
 #pragma unroll
     for (int tt = 0; tt < TILES; ++tt)
 #pragma unroll
@@ -697,15 +770,19 @@ inline int64_t repacked_bytes(int N, int K) {
 
 // Raw Q4_K rows as bytes [rows][row_bytes], box 160 bytes x box_rows rows (one super-block
 // per row plus 16 bytes of the next; past the end of a row the box reads zeros).
+// elem_bytes 2 views the bytes as 16-bit elements, for boxes wider than the 256
+// elements a box dimension may hold (the Q8_0 272-byte column); the kernel's x
+// coordinates are then in those elements.
 inline bool make_tmap_w_rowgroup(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes,
-                                 int box_rows, int box_bytes = kGemvPitch) {
+                                 int box_rows, int box_bytes = kGemvPitch, int elem_bytes = 1) {
   auto enc = get_encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / elem_bytes), (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {(cuuint32_t)(box_bytes / elem_bytes), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return enc(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+             const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

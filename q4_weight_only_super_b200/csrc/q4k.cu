@@ -83,9 +83,16 @@ static_assert(GemvSmem<2, 4, 2>::total(kGemvStages[1][0], kGemvStages[1][1]) <= 
 static_assert(GemvSmem<4, 4, 2>::total(kGemvStages[2][0], kGemvStages[2][1]) <= kGemvTwoPerSm, "mt 4");
 // Q5_K: 176-byte rows take a shallower weight ring at the same two CTAs per SM
 constexpr int kGemvStagesQ5[3][2] = {{3, 6}, {3, 2}, {2, 2}};
-static_assert(GemvSmem<1, 4, 2, false, true>::total(kGemvStagesQ5[0][0], kGemvStagesQ5[0][1]) <= kGemvTwoPerSm, "q5 mt 1");
-static_assert(GemvSmem<2, 4, 2, false, true>::total(kGemvStagesQ5[1][0], kGemvStagesQ5[1][1]) <= kGemvTwoPerSm, "q5 mt 2");
-static_assert(GemvSmem<4, 4, 2, false, true>::total(kGemvStagesQ5[2][0], kGemvStagesQ5[2][1]) <= kGemvTwoPerSm, "q5 mt 4");
+static_assert(GemvSmem<1, 4, 2, false, kQtQ5K>::total(kGemvStagesQ5[0][0], kGemvStagesQ5[0][1]) <= kGemvTwoPerSm, "q5 mt 1");
+static_assert(GemvSmem<2, 4, 2, false, kQtQ5K>::total(kGemvStagesQ5[1][0], kGemvStagesQ5[1][1]) <= kGemvTwoPerSm, "q5 mt 2");
+static_assert(GemvSmem<4, 4, 2, false, kQtQ5K>::total(kGemvStagesQ5[2][0], kGemvStagesQ5[2][1]) <= kGemvTwoPerSm, "q5 mt 4");
+// Q8_0: 272-byte rows, two weight stages (the reduction buffer shares the ring)
+constexpr int kGemvStagesQ80[3][2] = {{2, 6}, {2, 2}, {2, 2}};
+static_assert(GemvSmem<1, 4, 2, false, kQtQ80>::total(kGemvStagesQ80[0][0], kGemvStagesQ80[0][1]) <= kGemvTwoPerSm, "q8 mt 1");
+static_assert(GemvSmem<2, 4, 2, false, kQtQ80>::total(kGemvStagesQ80[1][0], kGemvStagesQ80[1][1]) <= kGemvTwoPerSm, "q8 mt 2");
+static_assert(GemvSmem<4, 4, 2, false, kQtQ80>::total(kGemvStagesQ80[2][0], kGemvStagesQ80[2][1]) <= kGemvTwoPerSm, "q8 mt 4");
+static_assert(GemvSmem<4, 4, 2, false, kQtQ80>::red_bytes <= 2 * GemvSmem<4, 4, 2, false, kQtQ80>::wstage,
+              "q8: reduction buffer inside the weight ring");
 
 // fit[d][ks]: clusters of ks GEMV CTAs that can be resident at once on device d
 // (a cluster must sit inside one GPC, so this is below 2 * SMs / ks).
@@ -151,16 +158,17 @@ q4k_status pick_gemv(int tokens, int rows_out, int nkb, int groups, GemvCfg* out
   return Q4K_OK;
 }
 
-template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false, bool Q5 = false>
+template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false, int QT = kQtQ4K>
 q4k_status launch_gemv_t(const GemvParams& p, int rows_total, int tiles, int groups, cudaStream_t s) {
-  auto* k = gemv_kernel<MT, WARPS, TILES, GROUPED, SWIGLU, REPACK, Q5>;
+  auto* k = gemv_kernel<MT, WARPS, TILES, GROUPED, SWIGLU, REPACK, QT>;
   static std::atomic<size_t> smem_set[kMaxDevices];  // one per instantiation
   CUtensorMap tmap = {};  // repacked weights stream by plain bulk copies: no tensor map
-  const int bb = Q5 ? kQ5BlockBytes : BLOCK_BYTES;
-  if (!REPACK && !make_tmap_w_rowgroup(&tmap, p.W, rows_total, (int64_t)p.nkb * bb, 16 * TILES,
-                                       Q5 ? kQ5BlockBytes : kGemvPitch))
+  using LS = GemvSmem<MT, WARPS, TILES, REPACK, QT>;
+  const int bb = QT == kQtQ80 ? kQ80GroupBytes : (QT == kQtQ5K ? kQ5BlockBytes : BLOCK_BYTES);
+  if (!REPACK && !make_tmap_w_rowgroup(&tmap, p.W, rows_total, (int64_t)p.nkb * bb, 16 * TILES, LS::pitch,
+                                       QT == kQtQ80 ? 2 : 1))
     return Q4K_ERR_CUDA;
-  const size_t smem = GemvSmem<MT, WARPS, TILES, REPACK, Q5>::total(p.wstages, p.xstages);
+  const size_t smem = GemvSmem<MT, WARPS, TILES, REPACK, QT>::total(p.wstages, p.xstages);
   if (ensure_smem(k, smem, smem_set) != cudaSuccess) return Q4K_ERR_LAUNCH;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * p.ksplit), (unsigned)groups, 1);
@@ -182,7 +190,7 @@ q4k_status launch_gemv_t(const GemvParams& p, int rows_total, int tiles, int gro
 }
 
 // Activation pre-pass (rows of X, gathered when `gather` is set) then the GEMV.
-template <bool GROUPED, bool SWIGLU, bool REPACK = false, bool Q5 = false>
+template <bool GROUPED, bool SWIGLU, bool REPACK = false, int QT = kQtQ4K>
 q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const int32_t* gather,
                        int rows, int K, void* ws, int rows_out, int groups, cudaStream_t s) {
   p.ksplit = c.ksplit;
@@ -196,9 +204,9 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
                                    rows, p.rows_pad, K, p.nkb, static_cast<uint8_t*>(ws));
   if (st != Q4K_OK) return st;
   const int tiles = (rows_out + 128 - 1) / 128;
-  if (c.mt == 1) return launch_gemv_t<1, 4, 2, GROUPED, SWIGLU, REPACK, Q5>(p, total_rows, tiles, groups, s);
-  if (c.mt == 2) return launch_gemv_t<2, 4, 2, GROUPED, SWIGLU, REPACK, Q5>(p, total_rows, tiles, groups, s);
-  return launch_gemv_t<4, 4, 2, GROUPED, SWIGLU, REPACK, Q5>(p, total_rows, tiles, groups, s);
+  if (c.mt == 1) return launch_gemv_t<1, 4, 2, GROUPED, SWIGLU, REPACK, QT>(p, total_rows, tiles, groups, s);
+  if (c.mt == 2) return launch_gemv_t<2, 4, 2, GROUPED, SWIGLU, REPACK, QT>(p, total_rows, tiles, groups, s);
+  return launch_gemv_t<4, 4, 2, GROUPED, SWIGLU, REPACK, QT>(p, total_rows, tiles, groups, s);
 }
 
 // Routing kernels keep each lane's share of a logit row in registers: pick the
@@ -303,6 +311,29 @@ int64_t q4k_repacked_bytes(int N, int K) {
   return repacked_bytes(N, K);
 }
 
+q4k_status q80_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws, size_t ws_bytes,
+                    void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (M == 0 || N == 0) return Q4K_OK;
+  if (!W || !X || !Y || !ws) return Q4K_ERR_NULL;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(Y) || !aligned16(ws)) return Q4K_ERR_ALIGN;
+  if (M > 32 || N % 16) return Q4K_ERR_UNSUPPORTED;
+  if (ws_bytes < gemv_ws_bytes(M, K)) return Q4K_ERR_WORKSPACE;
+  GemvParams p = {};
+  p.W = static_cast<const uint8_t*>(W);
+  p.out = Y;
+  p.M = M;
+  p.N = N;
+  p.nkb = K / QK;
+  GemvCfg c;
+  const q4k_status st = pick_gemv(M, N, p.nkb, 1, &c);  // the Q4_K K split: same cluster fit
+  if (st != Q4K_OK) return st;
+  const int cls = c.mt == 1 ? 0 : (c.mt == 2 ? 1 : 2);
+  c.wstages = kGemvStagesQ80[cls][0];
+  c.xstages = kGemvStagesQ80[cls][1];
+  return launch_gemv<false, false, false, kQtQ80>(c, p, X, nullptr, M, K, ws, N, 1, static_cast<cudaStream_t>(stream));
+}
+
 q4k_status q5k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws, size_t ws_bytes,
                     void* stream) {
   if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
@@ -323,7 +354,7 @@ q4k_status q5k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
   const int cls = c.mt == 1 ? 0 : (c.mt == 2 ? 1 : 2);
   c.wstages = kGemvStagesQ5[cls][0];
   c.xstages = kGemvStagesQ5[cls][1];
-  return launch_gemv<false, false, false, true>(c, p, X, nullptr, M, K, ws, N, 1, static_cast<cudaStream_t>(stream));
+  return launch_gemv<false, false, false, kQtQ5K>(c, p, X, nullptr, M, K, ws, N, 1, static_cast<cudaStream_t>(stream));
 }
 
 q4k_status q4k_repack(const void* W, int N, int K, void* Wr, void* stream) {

@@ -159,6 +159,47 @@ def test_q5k_gemv_dense_decode_sampled(decode_inputs_q5, proj, M):
     _assert_tol(y[:, rows], Y, S, f"Q5_K {proj} M={M}")
 
 
+# ---------------------------------------------------------------- Q8_0 GEMV --
+
+@pytest.mark.parametrize("N,K", [(16, 256), (48, 512), (272, 4096), (1040, 256 * 69)])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 17, 32])
+def test_q80_gemv_shapes(N, K, M):
+    W, X = synth.gemv_small_q80(500 + M, N=N, K=K, M=M)
+    y = host(q.q80_gemv(dev(W), dev(X), N, K))
+    Y, S = O.matmul_ref_q80(W, X)
+    _assert_tol(y, Y, S, f"Q8_0 N={N} K={K} M={M}")
+
+
+@pytest.fixture(scope="module")
+def decode_inputs_q80():
+    inp = synth.dense_decode_q80(6)
+    d = {k: dev(v) for k, v in inp.items()}
+    return inp, d
+
+
+@pytest.mark.parametrize("proj", ["gate_up", "down"])
+@pytest.mark.parametrize("M", [1, 8, 16, 32])
+def test_q80_gemv_dense_decode_sampled(decode_inputs_q80, proj, M):
+    inp, d = decode_inputs_q80
+    W, X = inp[f"W_{proj}"], inp[f"X_{proj}"][:M]
+    N, K = W.shape[0], W.shape[1] * 32
+    y = host(q.q80_gemv(d[f"W_{proj}"], d[f"X_{proj}"][:M], N, K))
+    rows = sample_rows(N, 384, seed=60 + M)
+    Y, S = O.matmul_rows_ref_q80(W, X, rows)
+    _assert_tol(y[:, rows], Y, S, f"Q8_0 {proj} M={M}")
+
+
+def test_q80_gemv_batch_invariance():
+    """Q8_0 takes the same per-token arithmetic at every token count: row m of any
+    call equals that token's row in a 32-token call; repeated calls are identical."""
+    W, X = synth.gemv_small_q80(520, N=1040, K=256 * 69, M=32)
+    Wd, Xd = dev(W), dev(X)
+    y32 = q.q80_gemv(Wd, Xd, 1040, 256 * 69)
+    assert torch.equal(y32, q.q80_gemv(Wd, Xd, 1040, 256 * 69))
+    for lo, hi in ((0, 1), (0, 8), (3, 12), (0, 16), (5, 22), (0, 17)):
+        assert torch.equal(q.q80_gemv(Wd, Xd[lo:hi], 1040, 256 * 69), y32[lo:hi]), (lo, hi)
+
+
 # ------------------------------------------------------------ decode repack --
 
 @pytest.mark.parametrize("N,K", [(16, 256), (200, 512), (1040, 256 * 69)])

@@ -577,12 +577,16 @@ def only(args):
         return roof(torch, tm)
     if args.only == "gemv":
         M = args.m or 1
-        dd = synth.dense_decode(1)
+        # weight format: Q4_K (default), Q5_K or Q8_0 at the same decode shapes
+        gen, call, wpb = {"q4k": (lambda: synth.dense_decode(1), q.q4k_gemv, BLOCK),
+                          "q5k": (lambda: synth.dense_decode_q5(5), q.q5k_gemv, 176),
+                          "q80": (lambda: synth.dense_decode_q80(6), q.q80_gemv, 272)}[args.quant]
+        dd = gen()
         Wt, Xt = dev(dd[f"W_{args.proj}"]), dev(dd[f"X_{args.proj}"][:M])
-        N, K = dd[f"W_{args.proj}"].shape[0], dd[f"W_{args.proj}"].shape[1] * 256
+        N, K = dd[f"W_{args.proj}"].shape[0], dd["X_" + args.proj].shape[1]
         ws = torch.empty(q.q4k_workspace_bytes(q.OP_GEMV, M, N, K), dtype=torch.uint8, device="cuda")
-        fn = lambda: q.q4k_gemv(Wt, Xt, N, K, ws=ws)
-        units = N * (K // 256) * BLOCK / 1e9
+        fn = lambda: call(Wt, Xt, N, K, ws=ws)
+        units = N * (K // 256) * wpb / 1e9
         unit = "GB/s"
     elif args.only == "gemm":
         M = args.m or 4096
@@ -632,6 +636,7 @@ def main():
                     help="run one kernel family a few times (for profiler captures), print times")
     ap.add_argument("--m", type=int, default=None, help="tokens for --only")
     ap.add_argument("--proj", default="gate_up", choices=["gate_up", "down"], help="GEMV matrix for --only")
+    ap.add_argument("--quant", default="q4k", choices=["q4k", "q5k", "q80"], help="GEMV weight format for --only")
     ap.add_argument("--iters", type=int, default=3, help="launches for --only")
     args = ap.parse_args()
     if args.only:

@@ -243,6 +243,19 @@ q4k_status moe_combine_residual(const float* O, const int32_t* inv_perm, const f
                                 const float* residual, int M, int topk, int H, float* Y,
                                 void* stream);
 
+/* The router product in front of moe_route_permute (the routing front of the
+ * fused MoE layer; hipEngine 0.3.0 README, "Architecture at a glance": moe
+ * kernels).
+ *   logits[t][e] = sum_k X[t][k] * W_router[e][k]: X bf16 [M][H], W_router
+ *   bf16 [E][H], logits fp32 [M][E] (caller-owned, written), the bf16
+ *   products exact in fp32, summed in fp32 in a fixed order.
+ * Then exactly moe_route_permute(logits, ...): the remaining arguments, the
+ * workspace and the errors are that call's. H % 8 == 0; M <= 65535. */
+q4k_status moe_route_permute_hidden(const uint16_t* X, const uint16_t* W_router, int M, int E, int H,
+                                    int topk, float* logits, int32_t* topk_ids, float* topk_w,
+                                    int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm,
+                                    int32_t* row_token, void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace an entry point needs for these sizes
  * (Q4K_OP_ROUTE: moe_route_permute with M tokens and E experts;
  *  Q4K_OP_GEMV: q4k_gemv with M tokens and K inputs;

@@ -269,6 +269,16 @@ def route_topk(logits: np.ndarray, topk: int):
     return ids, w
 
 
+def router_logits_ref(X_bits: np.ndarray, Wr_bits: np.ndarray):
+    """Router logits of the routing front (hipEngine 0.3.0 README, "Architecture at a
+    glance": moe kernels): ``(L, S)`` with ``L = X @ Wr^T`` and ``S = |X| @ |Wr|^T``
+    in fp64, X bf16 [M][H], Wr bf16 [E][H]. Reading R21: the router weights are bf16
+    like the activations; the pages do not give their type."""
+    X = bf16_to_f64(X_bits)
+    W = bf16_to_f64(Wr_bits)
+    return X @ W.T, np.abs(X) @ np.abs(W).T
+
+
 def permute(ids: np.ndarray, E: int):
     """Stable counting sort of the (token, slot) pairs by expert (Reading R6).
 

@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q5k_gemv", "q80_gemv", "q4k_repack", "q4k_gemv_repacked", "q4k_gemm",
     "moe_route_permute",
-    "moe_route_permute_noalloc",
+    "moe_route_permute_noalloc", "moe_route_permute_hidden",
     "moe_q4k_grouped", "moe_combine", "moe_combine_residual", "q4k_workspace_bytes", "q4k_last_device_status",
     "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "OP_GEMV", "EXPORTS",
 ]
@@ -39,6 +39,7 @@ EXPORTS = {
     "q4k_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "moe_route_permute": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_route_permute_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
+    "moe_route_permute_hidden": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_q4k_grouped": (_i, [_p, _i, _i, _i, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
     "moe_combine": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_combine_residual": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
@@ -181,6 +182,30 @@ def q4k_gemm(W, X, N: int, K: int, Y=None, stream=None):
 
 def q4k_workspace_bytes(op: int, M: int, N: int = 0, K: int = 0, E: int = 0, topk: int = 0) -> int:
     return lib().q4k_workspace_bytes(op, M, N, K, E, topk)
+
+
+def moe_route_permute_hidden(X, W_router, topk: int, out=None, ws=None, stream=None):
+    """Router logits X @ W_router^T (bf16 in, fp32 out) then moe_route_permute. Returns
+    the routing dict plus "logits"."""
+    M, H = X.shape
+    E = W_router.shape[0]
+    dev = X.device
+    if out is None:
+        rows = M * topk
+        out = {"logits": torch.empty(M, E, dtype=torch.float32, device=dev),
+               "topk_ids": torch.empty(M, topk, dtype=torch.int32, device=dev),
+               "topk_w": torch.empty(M, topk, dtype=torch.float32, device=dev),
+               "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+               "perm": torch.empty(rows, dtype=torch.int32, device=dev),
+               "inv_perm": torch.empty(rows, dtype=torch.int32, device=dev),
+               "row_token": torch.empty(rows, dtype=torch.int32, device=dev)}
+    ws = _scratch(q4k_workspace_bytes(OP_ROUTE, M, 0, 0, E, topk), dev, ws)
+    st = lib().moe_route_permute_hidden(
+        _ptr(_bits16(X)), _ptr(_bits16(W_router)), M, E, H, topk, _ptr(out["logits"]), _ptr(out["topk_ids"]),
+        _ptr(out["topk_w"]), _ptr(out["expert_offsets"]), _ptr(out["perm"]), _ptr(out["inv_perm"]),
+        _ptr(out["row_token"]), _ptr(ws), ws.numel(), _stream(stream))
+    _check("moe_route_permute_hidden", st)
+    return out
 
 
 def moe_route_permute(logits, topk: int, out=None, ws=None, stream=None):

@@ -351,4 +351,35 @@ combine_kernel(const float* __restrict__ O, const int32_t* __restrict__ inv_perm
   *reinterpret_cast<float4*>(Y + (int64_t)t * H + 4 * h4) = acc;
 }
 
+// Router logits: logits[t][e] = sum_k X[t][k] * Wr[e][k] (bf16 x bf16, fp32
+// accumulation; the products are exact in fp32). CTA (t, eb) computes experts
+// 32*eb .. 32*eb+31 of token t, four per warp: each lane sums its 8-wide slices
+// in increasing k, then the warp adds the lanes in a fixed tree.
+__global__ void __launch_bounds__(256)
+router_logits_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wr, int M, int E, int H,
+                     float* __restrict__ logits) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // X may come from the previous kernel
+  const int t = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* x = X + (int64_t)t * H;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = blockIdx.y * 32 + warp * 4 + i;
+    if (e >= E) break;  // uniform per warp
+    const uint16_t* w = Wr + (int64_t)e * H;
+    float acc = 0.f;
+    for (int k8 = lane * 8; k8 < H; k8 += 256) {
+      const uint4 xv = ldg_u4(x + k8), wv = ldg_u4(w + k8);
+      const uint32_t xa[4] = {xv.x, xv.y, xv.z, xv.w}, wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc = fmaf(bf16_bits_to_float(xa[j] & 0xFFFFu), bf16_bits_to_float(wa[j] & 0xFFFFu), acc);
+        acc = fmaf(bf16_bits_to_float(xa[j] >> 16), bf16_bits_to_float(wa[j] >> 16), acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) logits[(int64_t)t * E + e] = acc;
+  }
+}
+
 }  // namespace q4k

@@ -576,6 +576,29 @@ q4k_status moe_combine_residual(const float* O, const int32_t* inv_perm, const f
                     M, topk, H, residual, Y);
 }
 
+q4k_status moe_route_permute_hidden(const uint16_t* X, const uint16_t* W_router, int M, int E, int H, int topk,
+                                    float* logits, int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                                    int32_t* perm, int32_t* inv_perm, int32_t* row_token, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  if (M < 0 || E <= 0 || topk <= 0 || H <= 0 || H % 8) return Q4K_ERR_SHAPE;
+  if (E > kMaxE || topk > kMaxTopk || topk > E || M > 65535) return Q4K_ERR_UNSUPPORTED;
+  if (M > 0) {
+    if (!X || !W_router || !logits) return Q4K_ERR_NULL;
+    if (!aligned16(X) || !aligned16(W_router) || !aligned16(logits)) return Q4K_ERR_ALIGN;
+    // the routing call's own checks run before anything is launched
+    if (!topk_ids || !topk_w || !expert_offsets || !perm || !inv_perm || !row_token || !ws) return Q4K_ERR_NULL;
+    if (!aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(expert_offsets) || !aligned16(perm) ||
+        !aligned16(inv_perm) || !aligned16(row_token) || !aligned16(ws))
+      return Q4K_ERR_ALIGN;
+    if (ws_bytes < q4k_workspace_bytes(Q4K_OP_ROUTE, M, 0, 0, E, topk)) return Q4K_ERR_WORKSPACE;
+    const q4k_status st = launch_pdl(router_logits_kernel, dim3((unsigned)M, (unsigned)((E + 31) / 32)), dim3(256),
+                                     static_cast<cudaStream_t>(stream), X, W_router, M, E, H, logits);
+    if (st != Q4K_OK) return st;
+  }
+  return moe_route_permute(logits, M, E, topk, topk_ids, topk_w, expert_offsets, perm, inv_perm, row_token, ws,
+                           ws_bytes, stream);
+}
+
 q4k_status q4k_last_device_status(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return Q4K_ERR_CUDA;

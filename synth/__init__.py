@@ -214,6 +214,14 @@ def moe_layer(seed: int, M: int, E: int = 128, H: int = 2048, F: int = 768,
                 E=E, H=H, F=F)
 
 
+def router_weights(seed: int, E: int = 128, H: int = 2048, sigma: float = MOE_LOGIT_SIGMA):
+    """bf16 router weights [E][H] drawn N(0, sigma^2 / H), so that with N(0,1)
+    activations the logits are about N(0, sigma^2) (the logit distribution of the
+    MoE workloads)."""
+    rng = np.random.default_rng(seed)
+    return f32_to_bf16_bits((rng.standard_normal((E, H)) * (sigma / np.sqrt(H))).astype(np.float32))
+
+
 def moe_decode(seed: int = 3, M: int = 32):
     return moe_layer(seed, M)
 

@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     names = _declared()
     for n in ("q4k_gemv", "q4k_gemm", "moe_route_permute", "moe_q4k_grouped", "moe_combine",
               "q4k_repack", "q4k_repacked_bytes", "q4k_gemv_repacked", "moe_combine_residual", "q5k_gemv",
-              "q80_gemv"):
+              "q80_gemv", "moe_route_permute_hidden"):
         assert n in names
 
 
@@ -69,6 +69,11 @@ def test_argument_errors_return_before_launch(L):
     assert L.q80_gemv(fake, fake, fake, 1, 16, 96, fake, 1 << 20, None) == 3
     assert L.q80_gemv(fake, fake, fake, 1, 16, 256, fake, 64, None) == 5
     assert L.q80_gemv(None, None, None, 0, 16, 256, None, 0, None) == 0
+    # router front: H not a multiple of 8; too many experts; M == 0 writes zero offsets only
+    assert L.moe_route_permute_hidden(fake, fake, 1, 128, 100, 8, fake, fake, fake, fake, fake, fake, fake,
+                                      fake, big, None) == 3
+    assert L.moe_route_permute_hidden(fake, fake, 1, 2048, 256, 8, fake, fake, fake, fake, fake, fake, fake,
+                                      fake, big, None) == 4
     # GEMM N not a multiple of 256
     assert L.q4k_gemm(fake, fake, fake, 4, 128, 256, None, 0, None) == 4
     # routing: too many experts / top-k

@@ -277,6 +277,25 @@ def test_route_zero_tokens():
     assert st == 0 and torch.count_nonzero(offs).item() == 0
 
 
+@pytest.mark.parametrize("M", [1, 8, 32, 300])
+def test_route_from_hidden(M):
+    """Router logits within the fp32 summation bound of the oracle ((H-1) * 2^-24 * sum|x*w|);
+    then routing and permutation bit-exact against the oracle run on those logits."""
+    E, H, topk = 128, 2048, 8
+    X = synth.bf16_normal(np.random.default_rng(700 + M), (M, H))
+    Wr = synth.router_weights(22, E, H)
+    r = q.moe_route_permute_hidden(dev(X), dev(Wr), topk)
+    L, S = O.router_logits_ref(X, Wr)
+    lg = host(r["logits"]).astype(np.float64)
+    assert np.all(np.abs(lg - L) <= (H - 1) * 2.0 ** -24 * S)
+    ids, w = O.route_topk(host(r["logits"]), topk)
+    assert np.array_equal(host(r["topk_ids"]), ids)
+    assert np.abs(host(r["topk_w"]).astype(np.float64) - w).max() <= 1e-6
+    offs, perm, inv, rt = O.permute(ids, E)
+    for name, ref in (("expert_offsets", offs), ("perm", perm), ("inv_perm", inv), ("row_token", rt)):
+        assert np.array_equal(host(r[name]), ref), name
+
+
 # -------------------------------------------------------------- MoE combine --
 
 def test_combine():

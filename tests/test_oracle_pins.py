@@ -564,3 +564,31 @@ def test_q80_encode_closed_form_and_brute_force():
     Wq, _ = synth.gemv_small_q80(17, N=64, K=512, M=1)
     qv = Wq[..., 2:34].view(np.int8)
     assert qv.min() == -128 and qv.max() == 127
+
+
+# --------------------------------------------------------------- router --
+
+def test_router_logits_brute_force_and_one_hot():
+    """Every logit enumerated for a tiny case; a one-hot activation row selects a
+    column of the router weights."""
+    rng = np.random.default_rng(19)
+    X = synth.bf16_normal(rng, (3, 16))
+    Wr = synth.bf16_normal(rng, (5, 16))
+    L, S = O.router_logits_ref(X, Wr)
+    xf, wf = O.bf16_to_f64(X), O.bf16_to_f64(Wr)
+    for t in range(3):
+        for e in range(5):
+            prods = [xf[t, k] * wf[e, k] for k in range(16)]
+            assert abs(L[t, e] - math.fsum(prods)) <= 1e-14 * math.fsum(abs(p) for p in prods)
+            assert abs(S[t, e] - math.fsum(abs(p) for p in prods)) <= 1e-14 * S[t, e]
+    onehot = np.zeros((1, 16), np.uint16)
+    onehot[0, 7] = 0x3F80  # bf16 1.0
+    L1, _ = O.router_logits_ref(onehot, Wr)
+    np.testing.assert_array_equal(L1[0], wf[:, 7])
+
+
+def test_router_weights_give_the_workload_logit_spread():
+    rng = np.random.default_rng(20)
+    X = synth.bf16_normal(rng, (64, 2048))
+    L, _ = O.router_logits_ref(X, synth.router_weights(21))
+    assert 1.8 < L.std() < 2.2

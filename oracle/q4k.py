@@ -213,6 +213,41 @@ def make_block_q80(d: float, q) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Q8 activation lane (the pages' "fast" GEMV lane policy, dp4a route, accuracy
+# traded). Reading R22: the pages give no format; the one taken is int8
+# activations with one fp32 scale per 256-wide column of X (the super-block
+# width of the weights, so that the integer dot products of a whole super-block
+# can be summed with the six-bit scales exactly). Per token row and column kb:
+#   amax = max |x_k|;  d_x = RN_fp32(amax / 127);  inv = RN_fp32(127 / amax);
+#   q_k = clamp(rint_even(RN_fp32(x_k * inv)), -127, 127)   (amax = 0: all zero)
+# and the lane's product is y = sum_kb d_x * sum_k w_k * q_k (w exact).
+# --------------------------------------------------------------------------
+
+def quantize_x_q8(X_bits: np.ndarray):
+    """Int8 activations of the Q8 lane: ``(q int64 [M][K], d_x float32 [M][K/256])``,
+    every decision taken in fp32 exactly as written above."""
+    x = bf16_to_f64(X_bits).astype(np.float32)  # exact: bf16 values are fp32 values
+    M, K = x.shape
+    xb = x.reshape(M, K // QK, QK)
+    amax = np.abs(xb).max(axis=2)
+    with np.errstate(divide="ignore"):
+        d_x = np.where(amax > 0, np.float32(amax / np.float32(127)), np.float32(0)).astype(np.float32)
+        inv = np.where(amax > 0, np.float32(np.float32(127) / amax), np.float32(0)).astype(np.float32)
+    prod = (xb * inv[..., None]).astype(np.float32)  # one fp32 rounding per product
+    q = np.clip(np.rint(prod), -127, 127).astype(np.int64)
+    return q.reshape(M, K), d_x
+
+
+def matmul_ref_q8lane(W_blocks: np.ndarray, X_bits: np.ndarray):
+    """The Q8 lane's product in fp64: ``(Y, S)`` with Y = sum_kb d_x * w . q over the
+    quantised activations, S = sum |w| * |d_x * q| (the lane's own scale)."""
+    W = dequant_exact(W_blocks)
+    q, d_x = quantize_x_q8(X_bits)
+    xh = q.astype(np.float64) * np.repeat(d_x.astype(np.float64), QK, axis=1)
+    return xh @ W.T, np.abs(xh) @ np.abs(W).T
+
+
+# --------------------------------------------------------------------------
 # Dense matmul: Y[m, n] = sum_k W[n, k] * X[m, k]
 # --------------------------------------------------------------------------
 

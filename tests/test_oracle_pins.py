@@ -592,3 +592,56 @@ def test_router_weights_give_the_workload_logit_spread():
     X = synth.bf16_normal(rng, (64, 2048))
     L, _ = O.router_logits_ref(X, synth.router_weights(21))
     assert 1.8 < L.std() < 2.2
+
+
+# -------------------------------------------------------------- Q8 lane --
+
+def test_q8lane_quantizer_codes_and_error():
+    """Codes lie in -127..127; each column's largest magnitude maps to +-127; a zero
+    column gives zero codes and scale; every value is recovered within half a step
+    (plus the fp32 rounding of the scale and of its reciprocal)."""
+    rng = np.random.default_rng(23)
+    X = synth.bf16_normal(rng, (4, 1024))
+    X[1, 256:512] = 0
+    q, d_x = O.quantize_x_q8(X)
+    assert q.min() >= -127 and q.max() <= 127
+    x = O.bf16_to_f64(X)
+    for t in range(4):
+        for kb in range(4):
+            seg = x[t, 256 * kb: 256 * kb + 256]
+            qs = q[t, 256 * kb: 256 * kb + 256]
+            if not seg.any():
+                assert d_x[t, kb] == 0 and not qs.any()
+                continue
+            i = np.argmax(np.abs(seg))
+            assert abs(qs[i]) == 127 and np.sign(qs[i]) == np.sign(seg[i])
+            # half a step, plus |q| <= 127 times the gap between d_x = RN(amax/127) and
+            # 1/RN(127/amax) (a few fp32 ulps): d_x * (0.5 + 2e-5)
+            err = np.abs(seg - qs * float(d_x[t, kb]))
+            assert err.max() <= float(d_x[t, kb]) * (0.5 + 2e-5) + 1e-30
+
+
+def test_q8lane_integer_form_and_accuracy_bound():
+    """The lane's product equals the integer form used on the GPU -- per super-block
+    d * sum_j sc_j * (q_w . q_x) - dmin * sum_j m_j * bsum_j, times d_x -- and stays
+    within sum |w| * |x - d_x q| of the exact product."""
+    W, X = synth.gemv_small(24, N=3, K=512, M=2)
+    Y, S = O.matmul_ref_q8lane(W, X)
+    q, d_x = O.quantize_x_q8(X)
+    d, dmin = O.block_d_dmin(W)
+    sc, m = O.scale_min_pairs(W)
+    qw = O.quants(W)
+    for t in range(2):
+        for n in range(3):
+            tot = 0.0
+            for kb in range(2):
+                qx = q[t, 256 * kb: 256 * kb + 256]
+                I = sum(int(sc[n, kb, j]) * int(np.dot(qw[n, kb, 32 * j: 32 * j + 32], qx[32 * j: 32 * j + 32]))
+                        for j in range(8))
+                Im = sum(int(m[n, kb, j]) * int(qx[32 * j: 32 * j + 32].sum()) for j in range(8))
+                tot += float(d_x[t, kb]) * (d[n, kb] * I - dmin[n, kb] * Im)
+            assert abs(Y[t, n] - tot) <= 1e-12 * S[t, n]
+    Ye, _ = O.matmul_ref(W, X)
+    xq = q * np.repeat(d_x.astype(np.float64), 256, axis=1)
+    bound = np.abs(O.dequant_exact(W)) @ np.abs(O.bf16_to_f64(X) - xq).T
+    assert np.all(np.abs(Y - Ye) <= bound.T * (1 + 1e-9) + 1e-30)

@@ -332,6 +332,9 @@ def run_step(q, tm, W):
                 fns = [lambda Wt=Wt: q.q5k_gemv(Wt, X5, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_q5_copies"][p]]
                 tm.run_seq(f"gemv_q5:{p}:M{M}", fns)
                 launches += 2 * len(fns)
+                fns = [lambda Wt=Wt: q.q4k_gemv_q8(Wt, Xt, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_copies"][p]]
+                tm.run_seq(f"gemv_q8x:{p}:M{M}", fns)
+                launches += 2 * len(fns)
                 X8 = W["dec_q80"][f"X_{p}"][:M]
                 fns = [lambda Wt=Wt: q.q80_gemv(Wt, X8, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_q80_copies"][p]]
                 tm.run_seq(f"gemv_q80:{p}:M{M}", fns)
@@ -420,6 +423,12 @@ def summarize(tm, W, peaks):
                 b5 = N * (K // 256) * 176
                 comp[f"gemv_q5k_{p}_M{M}_GBps"] = round(b5 / t5 / 1e9, 1)
                 comp[f"gemv_q5k_{p}_M{M}_us"] = round(t5 * 1e6, 2)
+            tq = T.get(f"gemv_q8x:{p}:M{M}")
+            if tq:  # the Q8 activation lane over the same Q4_K weights
+                N, K = W["dec_shapes"][p]
+                bq = N * (K // 256) * BLOCK
+                comp[f"gemv_q8lane_{p}_M{M}_GBps"] = round(bq / tq / 1e9, 1)
+                comp[f"gemv_q8lane_{p}_M{M}_us"] = round(tq * 1e6, 2)
             t8 = T.get(f"gemv_q80:{p}:M{M}")
             if t8:  # Q8_0: 34 bytes per 32 weights
                 N, K = W["dec_shapes"][p]
@@ -450,7 +459,7 @@ def summarize(tm, W, peaks):
         if k.endswith((":layer", ":graph")):
             continue
         n = 1
-        if k.startswith(("gemv:", "gemv_rep:")):
+        if k.startswith(("gemv:", "gemv_rep:", "gemv_q8x:")):
             n = len(W["dec_copies"][k.split(":")[1]])
         elif k.startswith("gemv_q5:"):
             n = len(W["dec_q5_copies"][k.split(":")[1]])

@@ -109,6 +109,21 @@ q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
 q4k_status q5k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* The Q8 activation lane of the decode GEMV: an opt-in, accuracy-traded form of
+ * q4k_gemv (hipster/hipEngine READMEs: the "fast" GEMV lane policy, dp4a route,
+ * accuracy traded). Same arguments, workspace, shapes and errors as q4k_gemv.
+ * Each token's activations are quantised per 256-wide column: amax = max|x|,
+ * d_x = amax/127, q = rint(x * (127/amax)) clamped to +-127 (every step one
+ * fp32 operation, round to nearest even); the result is
+ *   Y[m][n] = sum_kb d_x[m][kb] * sum_k w[n][k] * q[m][k]
+ * with the 4-bit x 8-bit products and their six-bit scaling summed exactly in
+ * int32 per super-block (integer tensor-core MMA), the rest in fp32. Its error
+ * against q4k_gemv's product is bounded by sum_k |w[n][k]| * |x - d_x*q| (at
+ * most half a step d_x/2 per value). Row m does not depend on the other rows of
+ * X at any M. */
+q4k_status q4k_gemv_q8(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
+                       void* ws, size_t ws_bytes, void* stream);
+
 /* Decode GEMV over Q8_0 weights (the same tensor-family table lists Q8_0).
  * W [N][K/32] blocks of 34 bytes: fp16 d (little-endian), then 32 two's-
  * complement bytes q; w = d*q. K % 256 == 0 (the GEMV reads eight blocks per

@@ -169,6 +169,75 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const uint16_t* __restri
   if (lane == 0) *reinterpret_cast<float*>(rec + 544) = __uint_as_float((uint32_t)(127 - k) << 23);
 }
 
+// Q8 activation lane: the same records (one warp each, rows >= `rows` zero), holding
+// the 256 values of the column as int8 codes in natural order (bytes 0..255), the
+// eight sub-block sums of the codes times 2^-6 as fp16 hi + lo (exact: |sum| <=
+// 4064), and the column scale d_x at byte 544. amax = max |x|, d_x = amax / 127,
+// inv = 127 / amax, q = rint(x * inv) clamped to +-127, each step one IEEE fp32
+// operation in round-to-nearest-even.
+__global__ void __launch_bounds__(256) gemv_prep_q8_kernel(const uint16_t* __restrict__ X,
+                                                           const int32_t* __restrict__ gather, int rows,
+                                                           int rows_pad, int K, int nkb,
+                                                           uint8_t* __restrict__ ws) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // as gemv_prep_kernel
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= (int64_t)rows_pad * nkb) return;  // uniform per warp
+  const int kb = (int)(w / rows_pad), r = (int)(w % rows_pad);
+  uint8_t* rec = ws + w * kXRec;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (r < rows) {
+    const int64_t src = gather ? gather[r] : r;
+    v = ldg_u4(X + src * K + (int64_t)kb * QK + lane * 8);  // values 8*lane .. 8*lane+7
+  }
+  const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+  float x[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    x[2 * e] = bf16_bits_to_float(wv[e] & 0xFFFFu);
+    x[2 * e + 1] = bf16_bits_to_float(wv[e] >> 16);
+  }
+  uint32_t amax = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) amax = max(amax, __float_as_uint(x[e]) & 0x7FFFFFFFu);
+  amax = __reduce_max_sync(0xffffffffu, amax);
+  float dx = 0.f, inv = 0.f;
+  if (amax != 0) {
+    dx = __fdiv_rn(__uint_as_float(amax), 127.f);
+    inv = __fdiv_rn(127.f, __uint_as_float(amax));
+  }
+  uint32_t packed[2] = {0u, 0u};
+  int isum = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int qv = max(-127, min(127, __float2int_rn(__fmul_rn(x[e], inv))));
+    isum += qv;
+    packed[e >> 2] |= ((uint32_t)qv & 0xFFu) << (8 * (e & 3));
+  }
+  *reinterpret_cast<uint2*>(rec + 8 * lane) = make_uint2(packed[0], packed[1]);
+  isum += __shfl_xor_sync(0xffffffffu, isum, 1);  // the four lanes of sub-block lane / 4
+  isum += __shfl_xor_sync(0xffffffffu, isum, 2);
+  const float s2 = (float)isum * 0.015625f;
+  const __half hi = __float2half_rn(s2);
+  const __half lo = __float2half_rn(s2 - __half2float(hi));
+  if ((lane & 3) == 0) {
+    reinterpret_cast<__half*>(rec + 512)[lane >> 2] = hi;
+    reinterpret_cast<__half*>(rec + 528)[lane >> 2] = lo;
+  }
+  if (lane == 0) *reinterpret_cast<float*>(rec + 544) = dx;
+}
+
+// m16n8k32 integer MMA, u8 A x s8 B -> s32, zero accumulator in.
+__device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
 // ---------------------------------------------------------------------- GEMV ---
 
 struct GemvParams {
@@ -202,6 +271,7 @@ constexpr int kQ5QsOff = 48;   // the 128 nibble bytes, ordered as in Q4_K
 constexpr int kQ80GroupBytes = 272;
 // weight formats of the GEMV kernel
 constexpr int kQtQ4K = 0, kQtQ5K = 1, kQtQ80 = 2;
+constexpr int kQtQ4KxQ8 = 3;  // Q4_K weights, int8 activations (the Q8 lane)
 
 // Shared memory layout (dynamic):
 //   wring [wstages][WARPS][16*TILES rows][160 B]   weight tiles (TMA destination)
@@ -271,14 +341,14 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
   using L = GemvSmem<MT, WARPS, TILES, REPACK, QT>;
   static_assert(!REPACK || (!GROUPED && 16 * TILES * WARPS == kRepackRows), "repacked: dense, 128-row tiles");
   static_assert(QT == kQtQ4K || (!GROUPED && !REPACK), "Q5_K, Q8_0: dense raw layout");
-  constexpr bool Q5 = QT == kQtQ5K, Q80 = QT == kQtQ80;
+  constexpr bool Q5 = QT == kQtQ5K, Q80 = QT == kQtQ80, Q8X = QT == kQtQ4KxQ8;
   constexpr int BB = Q80 ? kQ80GroupBytes : (Q5 ? kQ5BlockBytes : BLOCK_BYTES);  // bytes per 256-wide column
   constexpr int QO = Q5 ? kQ5QsOff : 16;                                         // offset of the nibble bytes
   constexpr int TOK = 8 * MT;
   // 1..16 tokens: the subnormal-nibble A operand with per-sub-block scaling after the
   // MMA (fewer instructions per weight); 17..32: fp16 sc*q built before the MMA
   // (the per-result scaling would grow with the token groups).
-  constexpr bool SUBN = Q80 || MT <= 2;
+  constexpr bool SUBN = !Q8X && (Q80 || MT <= 2);
   constexpr int WROWS = 16 * TILES;    // weight rows per consumer warp
   constexpr int ROWS = WROWS * WARPS;  // weight rows per CTA
   extern __shared__ __align__(128) uint8_t smem[];
@@ -474,6 +544,13 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
       const uint8_t* xb = xring + (size_t)sx * L::xstage;
       if (valid) {
         float C[TILES][MT][4];
+        int IA[TILES][MT][4];  // Q8 lane: sum_j sc_j * (q_w . q_x) of the super-block, exact
+#pragma unroll
+        for (int tt = 0; tt < TILES; ++tt)
+#pragma unroll
+          for (int f = 0; f < MT; ++f)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) IA[tt][f][e] = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t qs8[R][2];  // words shifted by 8: bytes 1,3 in the positions of bytes 0,2
@@ -486,6 +563,39 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           for (int h = 0; h < 2; ++h) {
             const int j = 2 * c + h;  // sub-block
             const uint32_t msk = h ? 0x00F000F0u : 0x000F000Fu;
+            if (Q8X) {
+              // Q8 lane: A = the sub-block's nibbles as bytes (k slots 4t.. from word x, 16+4t..
+              // from word y, so B is the codes in natural order: eight bytes at 32j + 8t); one
+              // integer MMA per token group, the six-bit scale applied in int32
+              uint32_t A8[TILES][4];
+              int sci[R];
+#pragma unroll
+              for (int r = 0; r < R; ++r) sci[r] = (int)((scw[r][j >> 2] >> (8 * (j & 3))) & 0xFFu);
+#pragma unroll
+              for (int tt = 0; tt < TILES; ++tt) {
+                const int ra = 2 * tt, rb = 2 * tt + 1;
+                const uint32_t sh = 4 * h;
+                A8[tt][0] = (qv[ra][c].x >> sh) & 0x0F0F0F0Fu;
+                A8[tt][1] = (qv[rb][c].x >> sh) & 0x0F0F0F0Fu;
+                A8[tt][2] = (qv[ra][c].y >> sh) & 0x0F0F0F0Fu;
+                A8[tt][3] = (qv[rb][c].y >> sh) & 0x0F0F0F0Fu;
+              }
+#pragma unroll
+              for (int f = 0; f < MT; ++f) {
+                if (GROUPED && 8 * f >= count) break;
+                const uint2 bq = *reinterpret_cast<const uint2*>(xb + (8 * f + g) * kXRec + 32 * j + 8 * t);
+#pragma unroll
+                for (int tt = 0; tt < TILES; ++tt) {
+                  int ci[4];
+                  imma_16832(ci, A8[tt][0], A8[tt][1], A8[tt][2], A8[tt][3], bq.x, bq.y);
+                  IA[tt][f][0] += sci[2 * tt] * ci[0];
+                  IA[tt][f][1] += sci[2 * tt] * ci[1];
+                  IA[tt][f][2] += sci[2 * tt + 1] * ci[2];
+                  IA[tt][f][3] += sci[2 * tt + 1] * ci[3];
+                }
+              }
+              continue;
+            }
             // Q5: fifth bits of the four weights in bytes {0,2} (e = 0) and {1,3} (e = 1) of
             // each quant word, at bit 4 (low nibbles: q + 16*bit) or 8 (high: 16q + 256*bit)
             uint32_t hb[R][2][2];  // [row][k-step][byte pair]
@@ -621,6 +731,14 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
               }
             }
           }
+        }
+        if (Q8X) {  // the super-block's exact integer sums (|IA| < 2^31) as fp32
+#pragma unroll
+          for (int tt = 0; tt < TILES; ++tt)
+#pragma unroll
+            for (int f = 0; f < MT; ++f)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) C[tt][f][e] = (float)IA[tt][f][e];
         }
         // min term: Cm = sum_j m_j * X_j (k = sub-block index; k >= 8 is zero)
         uint32_t am[R];

@@ -200,8 +200,9 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
   p.xprep = static_cast<const uint8_t*>(ws);
   const int total_rows = (int)(GROUPED ? (int64_t)p.E * p.N : p.N);
   const int64_t recs = (int64_t)p.rows_pad * p.nkb;
-  const q4k_status st = launch_pdl(gemv_prep_kernel, dim3((unsigned)((recs + 7) / 8)), dim3(256), s, X, gather,
-                                   rows, p.rows_pad, K, p.nkb, static_cast<uint8_t*>(ws));
+  const q4k_status st = launch_pdl(QT == kQtQ4KxQ8 ? gemv_prep_q8_kernel : gemv_prep_kernel,
+                                   dim3((unsigned)((recs + 7) / 8)), dim3(256), s, X, gather, rows, p.rows_pad, K,
+                                   p.nkb, static_cast<uint8_t*>(ws));
   if (st != Q4K_OK) return st;
   const int tiles = (rows_out + 128 - 1) / 128;
   if (c.mt == 1) return launch_gemv_t<1, 4, 2, GROUPED, SWIGLU, REPACK, QT>(p, total_rows, tiles, groups, s);
@@ -309,6 +310,27 @@ q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
 int64_t q4k_repacked_bytes(int N, int K) {
   if (N <= 0 || K <= 0 || K % QK) return 0;
   return repacked_bytes(N, K);
+}
+
+q4k_status q4k_gemv_q8(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws,
+                       size_t ws_bytes, void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (M == 0 || N == 0) return Q4K_OK;
+  if (!W || !X || !Y || !ws) return Q4K_ERR_NULL;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(Y) || !aligned16(ws)) return Q4K_ERR_ALIGN;
+  if (M > 32 || N % 16) return Q4K_ERR_UNSUPPORTED;
+  if (ws_bytes < gemv_ws_bytes(M, K)) return Q4K_ERR_WORKSPACE;
+  GemvParams p = {};
+  p.W = static_cast<const uint8_t*>(W);
+  p.out = Y;
+  p.M = M;
+  p.N = N;
+  p.nkb = K / QK;
+  GemvCfg c;
+  const q4k_status st = pick_gemv(M, N, p.nkb, 1, &c);  // Q4_K rows: the Q4_K ring depths and K split
+  if (st != Q4K_OK) return st;
+  return launch_gemv<false, false, false, kQtQ4KxQ8>(c, p, X, nullptr, M, K, ws, N, 1,
+                                                      static_cast<cudaStream_t>(stream));
 }
 
 q4k_status q80_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws, size_t ws_bytes,

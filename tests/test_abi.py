@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     names = _declared()
     for n in ("q4k_gemv", "q4k_gemm", "moe_route_permute", "moe_q4k_grouped", "moe_combine",
               "q4k_repack", "q4k_repacked_bytes", "q4k_gemv_repacked", "moe_combine_residual", "q5k_gemv",
-              "q80_gemv", "moe_route_permute_hidden"):
+              "q80_gemv", "moe_route_permute_hidden", "q4k_gemv_q8"):
         assert n in names
 
 
@@ -65,6 +65,10 @@ def test_argument_errors_return_before_launch(L):
     assert L.q5k_gemv(fake, fake, fake, 1, 16, 300, fake, 1 << 20, None) == 3
     assert L.q5k_gemv(fake, fake, fake, 33, 16, 256, fake, 1 << 20, None) == 4
     assert L.q5k_gemv(fake, fake, fake, 1, 24, 256, fake, 1 << 20, None) == 4
+    # Q8 lane: the q4k_gemv checks
+    assert L.q4k_gemv_q8(fake, fake, fake, 1, 16, 100, fake, big, None) == 3
+    assert L.q4k_gemv_q8(fake, fake, fake, 33, 16, 256, fake, big, None) == 4
+    assert L.q4k_gemv_q8(fake, fake, fake, 1, 16, 256, fake, 64, None) == 5
     # Q8_0 GEMV: K must be a multiple of 256 (eight 32-weight blocks per column)
     assert L.q80_gemv(fake, fake, fake, 1, 16, 96, fake, 1 << 20, None) == 3
     assert L.q80_gemv(fake, fake, fake, 1, 16, 256, fake, 64, None) == 5

@@ -159,6 +159,50 @@ def test_q5k_gemv_dense_decode_sampled(decode_inputs_q5, proj, M):
     _assert_tol(y[:, rows], Y, S, f"Q5_K {proj} M={M}")
 
 
+# ------------------------------------------------------------------ Q8 lane --
+
+def _q8lane_check(W, X, y, what):
+    """Tight parity with the lane's own product (int32-exact super-block sums, fp32 for
+    the rest: 3e-5 of its absolute scale), and the accuracy bound against the exact one."""
+    Yl, Sl = O.matmul_ref_q8lane(W, X)
+    err = np.abs(y.astype(np.float64) - Yl)
+    assert np.all(err <= 3e-5 * Sl + 1e-30), f"{what}: lane parity, worst {float((err / np.maximum(Sl, 1e-300)).max()):.2e}"
+    Ye, _ = O.matmul_ref(W, X)
+    q, d_x = O.quantize_x_q8(X)
+    xq = q * np.repeat(d_x.astype(np.float64), 256, axis=1)
+    bound = (np.abs(O.bf16_to_f64(X) - xq) @ np.abs(O.dequant_exact(W)).T)
+    assert np.all(np.abs(y - Ye) <= bound + 3e-5 * Sl + 1e-30), f"{what}: accuracy bound"
+
+
+@pytest.mark.parametrize("N,K", [(16, 256), (48, 512), (272, 4096), (1040, 256 * 69)])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 17, 32])
+def test_q8lane_gemv_shapes(N, K, M):
+    W, X = synth.gemv_small(600 + M, N=N, K=K, M=M)
+    y = host(q.q4k_gemv_q8(dev(W), dev(X), N, K))
+    _q8lane_check(W, X, y, f"Q8 lane N={N} K={K} M={M}")
+
+
+@pytest.mark.parametrize("proj", ["gate_up", "down"])
+@pytest.mark.parametrize("M", [1, 32])
+def test_q8lane_gemv_dense_decode_sampled(decode_inputs, proj, M):
+    inp, d = decode_inputs
+    W, X = inp[f"W_{proj}"], inp[f"X_{proj}"][:M]
+    N, K = W.shape[0], W.shape[1] * 256
+    y = host(q.q4k_gemv_q8(d[f"W_{proj}"], d[f"X_{proj}"][:M], N, K))
+    rows = sample_rows(N, 256, seed=70 + M)
+    _q8lane_check(W[rows], X, y[:, rows], f"Q8 lane {proj} M={M}")
+
+
+def test_q8lane_batch_invariance():
+    """Integer super-block sums and the same fp32 epilogue per token at every token
+    count: row m of any call equals that token's row of a 32-token call."""
+    W, X = synth.gemv_small(620, N=1040, K=256 * 69, M=32)
+    Wd, Xd = dev(W), dev(X)
+    y32 = q.q4k_gemv_q8(Wd, Xd, 1040, 256 * 69)
+    for lo, hi in ((0, 1), (0, 8), (3, 12), (0, 16), (5, 22)):
+        assert torch.equal(q.q4k_gemv_q8(Wd, Xd[lo:hi], 1040, 256 * 69), y32[lo:hi]), (lo, hi)
+
+
 # ---------------------------------------------------------------- Q8_0 GEMV --
 
 @pytest.mark.parametrize("N,K", [(16, 256), (48, 512), (272, 4096), (1040, 256 * 69)])

@@ -213,6 +213,69 @@ def make_block_q80(d: float, q) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Q6_K super-block (the remaining sibling of the tensor-family table). Reading
+# R23: the llama.cpp-style block of 256 weights in 210 bytes -- ql[128] (bytes
+# 0..127, low four bits), qh[64] (bytes 128..191, high two bits), 16 signed
+# byte scales (bytes 192..207), fp16 d (bytes 208..209). Weight i = 128n + 32u
+# + l (half n, quarter u, lane l) takes nibble u // 2 of ql[64n + 32(u % 2) + l]
+# and bits 2u, 2u+1 of qh[32n + l]; q = those six bits - 32 in -32..31 and
+# w = d * scale[i // 16] * q.
+# --------------------------------------------------------------------------
+
+Q6_BLOCK_BYTES = 210
+
+
+def quants_q6(blocks: np.ndarray) -> np.ndarray:
+    """The 256 six-bit quants (-32..31) of each Q6_K block, in weight order."""
+    b = np.asarray(blocks, dtype=np.uint8)
+    ql = b[..., 0:128].astype(np.int64)
+    qh = b[..., 128:192].astype(np.int64)
+    q = np.empty(b.shape[:-1] + (QK,), dtype=np.int64)
+    for n in range(2):
+        for u in range(4):
+            low = (ql[..., 64 * n + 32 * (u % 2): 64 * n + 32 * (u % 2) + 32] >> (4 * (u // 2))) & 15
+            high = (qh[..., 32 * n: 32 * n + 32] >> (2 * u)) & 3
+            q[..., 128 * n + 32 * u: 128 * n + 32 * u + 32] = (low | (high << 4)) - 32
+    return q
+
+
+def dequant_exact_q6(blocks: np.ndarray) -> np.ndarray:
+    """Exact Q6_K weights in fp64 (``[..., nb, 210]`` -> ``[..., nb*256]``)."""
+    b = np.ascontiguousarray(blocks, dtype=np.uint8)
+    d = b[..., 208:210].copy().view("<f2")[..., 0].astype(np.float64)
+    sc = b[..., 192:208].view(np.int8).astype(np.float64)
+    q = quants_q6(b)
+    w = d[..., None] * sc[..., np.arange(QK) // 16] * q
+    return w.reshape(w.shape[:-2] + (w.shape[-2] * QK,))
+
+
+def matmul_ref_q6(W_blocks: np.ndarray, X_bits: np.ndarray):
+    """``matmul_ref`` for Q6_K weights ``[N][K/256][210]``: ``(Y, S)`` in fp64."""
+    W = dequant_exact_q6(W_blocks)
+    X = bf16_to_f64(X_bits)
+    return X @ W.T, np.abs(X) @ np.abs(W).T
+
+
+def make_block_q6(d: float, scales, q) -> np.ndarray:
+    """One 210-byte Q6_K block from d (rounded to binary16), 16 scales in -128..127
+    and 256 quants in -32..31 (Reading R23)."""
+    q6 = np.asarray(q, dtype=np.int64) + 32
+    b = np.zeros(Q6_BLOCK_BYTES, dtype=np.uint8)
+    ql = np.zeros(128, dtype=np.int64)
+    qh = np.zeros(64, dtype=np.int64)
+    for n in range(2):
+        for u in range(4):
+            v = q6[128 * n + 32 * u: 128 * n + 32 * u + 32]
+            ql[64 * n + 32 * (u % 2): 64 * n + 32 * (u % 2) + 32] |= (v & 15) << (4 * (u // 2))
+            qh[32 * n: 32 * n + 32] |= (v >> 4) << (2 * u)
+    b[0:128] = ql.astype(np.uint8)
+    b[128:192] = qh.astype(np.uint8)
+    b[192:208] = np.asarray(scales, dtype=np.int64).astype(np.int8).view(np.uint8)
+    b[208:210] = np.array([d], dtype="<f2").view(np.uint8)
+    return b
+
+
+# --------------------------------------------------------------------------
 # Q8 activation lane (the pages' "fast" GEMV lane policy, dp4a route, accuracy
 # traded). Reading R22: the pages give no format; the one taken is int8
 # activations with one fp32 scale per 256-wide column of X (the super-block

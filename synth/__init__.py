@@ -101,6 +101,26 @@ def q80_random_blocks(rng: np.random.Generator, nrows: int, K: int) -> np.ndarra
     return out.reshape(nrows, K // 32, Q80_BLOCK_BYTES)
 
 
+Q6_BLOCK_BYTES = 210  # bytes per Q6_K super-block
+
+
+def q6k_random_blocks(rng: np.random.Generator, nrows: int, K: int) -> np.ndarray:
+    """Random Q6_K matrix: uint8 ``[nrows][K/256][210]``. Draw order: the 192 quant
+    bytes (ql then qh, uniform: every six-bit quant uniform), the 16 scale bytes
+    (uniform: signed scales uniform on -128..127), then d as for Q4_K blocks."""
+    if K % BLOCK_WEIGHTS:
+        raise ValueError("K must be a multiple of 256")
+    nb = nrows * (K // BLOCK_WEIGHTS)
+    qb = rng.integers(0, 256, size=(nb, 192), dtype=np.uint8)
+    sc = rng.integers(0, 256, size=(nb, 16), dtype=np.uint8)
+    d = (np.abs(rng.standard_normal(nb)) * 1e-3).astype(np.float16)
+    out = np.empty((nb, Q6_BLOCK_BYTES), dtype=np.uint8)
+    out[:, 0:192] = qb
+    out[:, 192:208] = sc
+    out[:, 208:210] = d.astype("<f2").view(np.uint8).reshape(nb, 2)
+    return out.reshape(nrows, K // BLOCK_WEIGHTS, Q6_BLOCK_BYTES)
+
+
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """fp32 array -> bf16 bit patterns (uint16), round to nearest even (torch CPU cast)."""
     import torch

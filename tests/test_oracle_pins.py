@@ -645,3 +645,53 @@ def test_q8lane_integer_form_and_accuracy_bound():
     xq = q * np.repeat(d_x.astype(np.float64), 256, axis=1)
     bound = np.abs(O.dequant_exact(W)) @ np.abs(O.bf16_to_f64(X) - xq).T
     assert np.all(np.abs(Y - Ye) <= bound.T * (1 + 1e-9) + 1e-30)
+
+
+# ------------------------------------------------------------------ Q6_K --
+
+def test_q6_one_hot_bits():
+    """Setting one bit of ql or qh changes exactly one weight, by d*scale*(bit value):
+    nibble u//2 of ql[64n+32(u%2)+l] and bits 2u, 2u+1 of qh[32n+l] belong to weight
+    128n+32u+l, whose scale is scale[i // 16]."""
+    scales = np.arange(1, 17)
+    base = O.make_block_q6(1.0, scales, np.full(256, -32))  # all six-bit fields zero
+    assert not base[0:192].any()
+    w0 = O.dequant_exact_q6(base[None])
+    assert np.array_equal(w0, -32.0 * scales[np.arange(256) // 16])
+    for n in range(2):
+        for u in range(4):
+            for l in (0, 5, 31):
+                i = 128 * n + 32 * u + l
+                for bit in range(6):
+                    b = base.copy()
+                    if bit < 4:
+                        b[64 * n + 32 * (u % 2) + l] = np.uint8(1 << (bit + 4 * (u // 2)))
+                    else:
+                        b[128 + 32 * n + l] = np.uint8(1 << (2 * u + bit - 4))
+                    diff = O.dequant_exact_q6(b[None]) - w0
+                    expect = np.zeros(256)
+                    expect[i] = float(1 << bit) * scales[i // 16]
+                    assert np.array_equal(diff, expect), (n, u, l, bit)
+
+
+def test_q6_round_trip_signs_and_brute_force():
+    rng = np.random.default_rng(25)
+    q = rng.integers(-32, 32, 256)
+    sc = rng.integers(-128, 128, 16)
+    blk = O.make_block_q6(2e-3, sc, q)
+    np.testing.assert_array_equal(O.quants_q6(blk[None])[0], q)
+    dh = float(np.float16(2e-3))
+    np.testing.assert_array_equal(O.dequant_exact_q6(blk[None]), dh * sc[np.arange(256) // 16] * q)
+    W = synth.q6k_random_blocks(rng, 2, 256)
+    X = synth.bf16_normal(rng, (2, 256))
+    Y, S = O.matmul_ref_q6(W, X)
+    xf = O.bf16_to_f64(X)
+    wq = O.quants_q6(W)
+    for n in range(2):
+        d = float(np.frombuffer(bytes(W[n, 0, 208:210]), "<f2")[0])
+        s = W[n, 0, 192:208].view(np.int8)
+        for t in range(2):
+            prods = [d * int(s[i // 16]) * int(wq[n, 0, i]) * xf[t, i] for i in range(256)]
+            assert abs(Y[t, n] - math.fsum(prods)) <= 1e-12 * math.fsum(abs(p) for p in prods)
+    allq = O.quants_q6(synth.q6k_random_blocks(rng, 64, 512))
+    assert allq.min() == -32 and allq.max() == 31

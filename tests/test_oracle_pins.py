@@ -695,3 +695,149 @@ def test_q6_round_trip_signs_and_brute_force():
             assert abs(Y[t, n] - math.fsum(prods)) <= 1e-12 * math.fsum(abs(p) for p in prods)
     allq = O.quants_q6(synth.q6k_random_blocks(rng, 64, 512))
     assert allq.min() == -32 and allq.max() == 31
+
+
+# ---------------------------------------------------------------- SiLU / SwiGLU --
+# silu_mul and swiglu_bf16_ref (Reading R16: SiLU(g) = g * sigma(g), the gate of
+# the SwiGLU expert FFN; Reading R8: gate columns first, then up) pinned by values
+# the mathematics fixes, not by a restatement of the formula:
+#   silu(0) = 0;  silu(1) = 1 / (1 + e^-1) = 0.7310585786300049;
+#   silu(-1) = -1 / (1 + e) = -0.2689414213699951;
+#   silu(g) - silu(-g) = g (sigma(g) + sigma(-g) = 1);
+#   silu(g) > g / 2 for g > 0 (sigma(g) > 1/2 there);
+#   silu(g) -> g as g -> +inf, silu(g) -> 0 from below as g -> -inf;
+# and the logistic function of an independent library (scipy.special.expit).
+
+SILU_1 = 0.7310585786300049    # 1 / (1 + 1/e), e = 2.718281828459045
+SILU_M1 = -0.2689414213699951  # -1 / (1 + e)
+
+
+def _silu_pins_hold(silu_mul) -> bool:
+    from scipy.special import expit
+
+    one = np.ones(1)
+    if silu_mul(np.zeros(1), one)[0] != 0.0:
+        return False
+    if abs(silu_mul(one, one)[0] - SILU_1) > 1e-15 or abs(silu_mul(-one, one)[0] - SILU_M1) > 1e-15:
+        return False
+    g = np.linspace(-12.0, 12.0, 241)
+    s, s_neg = silu_mul(g, np.ones_like(g)), silu_mul(-g, np.ones_like(g))
+    if np.max(np.abs((s - s_neg) - g)) > 1e-13:
+        return False
+    pos = g > 0
+    if not np.all(s[pos] > g[pos] / 2):
+        return False
+    if np.max(np.abs(s - g * expit(g))) > 1e-14:
+        return False
+    big = np.array([40.0, 100.0])
+    if not np.all(silu_mul(big, np.ones(2)) == big):           # sigma(40) = 1 - 4e-18 -> 1.0
+        return False
+    tail = silu_mul(-big, np.ones(2))
+    if not (np.all(tail < 0) and np.all(tail > -1e-15)):        # -40 e^-40 ~ -1.7e-16
+        return False
+    u = np.array([3.0, -0.5])                                   # linear in u
+    return bool(np.all(np.abs(silu_mul(np.array([1.0, 1.0]), u) - SILU_1 * u) <= 1e-15))
+
+
+def test_silu_pinned():
+    assert _silu_pins_hold(O.silu_mul)
+
+
+@pytest.mark.parametrize("mutant", [
+    lambda g, u: g / (1.0 + np.exp(g)) * u,            # sigma(-g) in place of sigma(g)
+    lambda g, u: 1.0 / (1.0 + np.exp(-g)) * u,         # sigmoid without the factor g
+    lambda g, u: g / (1.0 + np.exp(-2.0 * g)) * u,     # a different slope
+    lambda g, u: g * np.tanh(g) * u,                   # a different gate
+])
+def test_silu_mutants_are_caught(mutant):
+    assert not _silu_pins_hold(mutant)
+
+
+def test_swiglu_bf16_hand_values():
+    """h = RN_bf16(RN_fp32(silu(gate) * up)) on hand-worked rows, gate columns first.
+
+    gate 1, up 2: 2 * 0.7310585786300049 = 1.4621171572600098; bf16 spacing in [1, 2) is 2^-7,
+    1.46211.../2^-7 = 187.15 -> 187 -> 1.4609375 = 0x3FBB.
+    gate 2, up 1: 2 / (1 + e^-2) = 1.7615941559557646 -> 225.48 * 2^-7 -> 225 -> 1.7578125 = 0x3FE1
+    (the same row read up-first would give 0x3FBB: the column order is pinned).
+    gate 0, up 5: 0 -> 0x0000.  gate -1, up -4: 4 * 0.2689414213699951 = 1.0757656854799804
+    -> 137.70 * 2^-7 -> 138 -> 1.078125 = 0x3F8A.
+    """
+    GU = np.array([[1.0, 2.0, 0.0, -1.0, 2.0, 1.0, 5.0, -4.0]])
+    h = O.swiglu_bf16_ref(GU, 4)
+    assert h.dtype == np.uint16
+    assert [int(v) for v in h[0]] == [0x3FBB, 0x3FE1, 0x0000, 0x3F8A]
+
+
+# ---------------------------------------------------- bf16 round to nearest even --
+# Reading R2 (bf16 weights = RN_bf16(RN_fp32(w))) and the h rounding of Reading R7
+# both rest on round-to-nearest-EVEN. Ties are built by hand: 1 + 2^-8 lies exactly
+# halfway between the bf16 neighbours 1.0 (0x3F80, even) and 1 + 2^-7 (0x3F81, odd);
+# 1 + 3*2^-8 halfway between 0x3F81 and 1 + 2^-6 (0x3F82, even). Round-half-away,
+# round-half-up and truncation each get at least one of these wrong.
+
+def _f32(v):
+    return np.array([v], dtype=np.float64)
+
+
+_RNE_CASES = [
+    (1.0 + 2.0 ** -8, 0x3F80),                    # tie -> even (down)
+    (1.0 + 3 * 2.0 ** -8, 0x3F82),                # tie -> even (up)
+    (-(1.0 + 2.0 ** -8), 0xBF80),                 # sign symmetric
+    (-(1.0 + 3 * 2.0 ** -8), 0xBF82),
+    (1.0 + 2.0 ** -8 - 2.0 ** -23, 0x3F80),       # largest fp32 below the tie
+    (1.0 + 2.0 ** -8 + 2.0 ** -23, 0x3F81),       # smallest fp32 above it
+    # bf16 subnormals are k * 2^-133 (k < 128); fp32 holds these ties exactly
+    (2.0 ** -133 * 1.5, 0x0002),                  # tie between k = 1 and 2 -> even (2)
+    (2.0 ** -133 * 2.5, 0x0002),                  # tie between k = 2 and 3 -> even (2)
+]
+
+
+def _rne_pins_hold(to_bf16) -> bool:
+    return all(int(to_bf16(_f32(v))[0]) == bits for v, bits in _RNE_CASES)
+
+
+def test_bf16_rne_ties_and_neighbours():
+    assert _rne_pins_hold(O.f64_to_bf16_bits)
+
+
+def _f32_bits(a):
+    return np.ascontiguousarray(a, dtype=np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+
+
+@pytest.mark.parametrize("mutant", [
+    lambda a: ((_f32_bits(a) + 0x8000) >> 16).astype(np.uint16),             # ties away from zero
+    lambda a: (_f32_bits(a) >> 16).astype(np.uint16),                         # truncation
+    lambda a: ((_f32_bits(a) + 0x7FFF) >> 16).astype(np.uint16),             # ties toward zero
+])
+def test_bf16_rounding_mutants_are_caught(mutant):
+    assert not _rne_pins_hold(mutant)
+
+
+def test_bf16_double_rounding_through_fp32():
+    """RN_bf16(RN_fp32(w)): 1 + 2^-8 + 2^-30 rounds to the tie 1 + 2^-8 in fp32 (2^-30 is
+    below half an fp32 ulp of 1, 2^-24), then to the even 0x3F80 -- a direct rounding
+    of the fp64 value would give 0x3F81."""
+    assert int(O.f64_to_bf16_bits(_f32(1.0 + 2.0 ** -8 + 2.0 ** -30))[0]) == 0x3F80
+    assert int(O.f64_to_bf16_bits(_f32(1.0 + 2.0 ** -8 + 2.0 ** -23))[0]) == 0x3F81
+
+
+def test_dequant_bf16_ties_on_blocks():
+    """Blocks whose weights are exact bf16 ties: d = 1 + 2^-8 and 1 + 3*2^-8 are fp16 values
+    (10 mantissa bits), sc = q = 1, dmin = m = 0, so w = d exactly; bf16 must be the even
+    neighbour. With q = 2 the weight 2d = 2 + 2^-7 is again a tie (spacing 2^-6 in [2, 4)):
+    0x4000 (even). A min term reaching a tie from below: d = 1, sc = q = 1, dmin = 2^-8,
+    m = 1 gives 1 - 2^-8, exactly representable in bf16 (spacing 2^-8 in [0.5, 1)): 0x3F7F."""
+    blocks = np.stack([
+        O.make_block(1.0 + 2.0 ** -8, 0.0, [1] * 8, [0] * 8, [1] * 256),
+        O.make_block(1.0 + 3 * 2.0 ** -8, 0.0, [1] * 8, [0] * 8, [1] * 256),
+        O.make_block(1.0 + 2.0 ** -8, 0.0, [1] * 8, [0] * 8, [2] * 256),
+        O.make_block(1.0, 2.0 ** -8, [1] * 8, [1] * 8, [1] * 256),
+    ])[:, None, :]                                    # four rows of one block each
+    bits = O.dequant_bf16_bits(blocks)
+    assert np.all(bits[0] == 0x3F80)
+    assert np.all(bits[1] == 0x3F82)
+    assert np.all(bits[2] == 0x4000)
+    assert np.all(bits[3] == 0x3F7F)
+    f32 = O.dequant_f32(blocks)
+    assert np.all(f32[0] == np.float32(1.0 + 2.0 ** -8))

@@ -62,8 +62,10 @@ typedef enum {
   Q4K_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up                */
   Q4K_ERR_DEVICE_BOUNDS = 8,  /* a device-side index check failed                  */
   Q4K_ERR_CUDA = 9,           /* a CUDA runtime call returned an error             */
-  Q4K_ERR_DEVICE_RANGE = 10,  /* a value does not fit the fp16 operands of the
-                                 tensor-core grouped path (|x| or |w| > 65504)     */
+  Q4K_ERR_DEVICE_RANGE = 10,  /* a value may not fit the fp16 operands of the
+                                 tensor-core grouped path: |x| > 65504, or a
+                                 sub-block whose bound 15*|d*sc| + |dmin*m|
+                                 exceeds 65504                                     */
   Q4K_ERR_TOO_LARGE = 11      /* the problem needs more than the fixed scratch of
                                  the no-allocation entry point                     */
 } q4k_status;
@@ -85,13 +87,15 @@ q4k_status q4k_dequant(const void* W, int64_t nblocks, int out_bf16, void* out, 
  *   Y[m][n] = sum_k w[n][k] * X[m][k],  W [N][K/256] blocks, X bf16 [M][K],
  *   Y fp32 [M][N].  N % 16 == 0.  M == 0 or N == 0 is a no-op.
  *   ws/ws_bytes: device scratch of q4k_workspace_bytes(Q4K_OP_GEMV, M, N, K,
- *   0, 0) bytes; a pre-pass writes each token's activations there, per
- *   256-wide block scaled by a power of two and rounded to fp16 (an
- *   activation is represented to 11 significant bits relative to the largest
- *   magnitude of its 256-block). The 4-bit weights and their six-bit scales
- *   enter exactly; products accumulate in fp32. Calls sharing `ws` must be
- *   ordered on one stream.
- * Within a token class (M = 1..16, M = 17..32) row m of the result does not
+ *   0, 0) bytes (required; some launch shapes leave it untouched). Each
+ *   token's activations are taken per 256-wide block, scaled by a power of two
+ *   so the block's largest magnitude lands in [2^14, 2^15), and converted to
+ *   fp16: exact for every bf16 value within a factor 2^31 of that largest
+ *   magnitude (smaller ones keep fp16 subnormal resolution, 2^-24 of the
+ *   scaled unit). The 4-bit weights and their six-bit scales enter exactly;
+ *   products accumulate in fp32. Calls sharing `ws` must be ordered on one
+ *   stream.
+ * Within a token class (M = 1..8, 9..16, 17..32) row m of the result does not
  * depend on the other rows of X (bit-identical to any other call of the same
  * class on that row). */
 q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
@@ -281,6 +285,22 @@ size_t q4k_workspace_bytes(int op, int M, int N, int K, int E, int topk);
 /* Synchronises `stream`, returns the device status word (Q4K_OK if no
  * device-side error was latched since the last call) and clears it. */
 q4k_status q4k_last_device_status(void* stream);
+
+/* Test hook for the bounded device-side waits (failure detection without a GPU
+ * fault; hipEngine 0.3.0 README, "Core principles": fail closed instead of
+ * hanging or falling back). Sets, for every later launch on the current device:
+ *   drop_stage     >= 0: the weight producer of every CTA of q4k_gemm and of the
+ *                  decode GEMVs skips its stage with this index (no copy, no
+ *                  arrival), so the roles waiting for it reach the wait limit;
+ *                  < 0: off (the default).
+ *   wait_limit_ns  the limit of every bounded wait, in ns; 0 restores the
+ *                  default (2 s).
+ * A kernel whose wait expires latches Q4K_ERR_DEVICE_TIMEOUT, stops every role,
+ * waits (bounded) for its own copies in flight, releases its tensor memory and
+ * returns; its outputs are then undefined. Synchronous with the host (a copy to
+ * device symbols); not for use while kernels of this library are in flight.
+ * Returns Q4K_ERR_CUDA if the copy fails. */
+q4k_status q4k_test_wait_fault(int drop_stage, uint64_t wait_limit_ns);
 
 /* Static description of a status code. */
 const char* q4k_status_string(int status);

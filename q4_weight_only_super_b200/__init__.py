@@ -18,6 +18,7 @@ __all__ = [
     "moe_route_permute",
     "moe_route_permute_noalloc", "moe_route_permute_hidden",
     "moe_q4k_grouped", "moe_combine", "moe_combine_residual", "q4k_workspace_bytes", "q4k_last_device_status",
+    "q4k_test_wait_fault",
     "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "OP_GEMV", "EXPORTS",
 ]
 
@@ -46,6 +47,7 @@ EXPORTS = {
     "moe_combine_residual": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "q4k_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "q4k_last_device_status": (_i, [_p]),
+    "q4k_test_wait_fault": (_i, [_i, ctypes.c_uint64]),
     "q4k_status_string": (ctypes.c_char_p, [_i]),
 }
 
@@ -306,3 +308,9 @@ def moe_combine_residual(O, inv_perm, topk_w, residual, M: int, topk: int, H: in
 def q4k_last_device_status(stream=None) -> int:
     """Synchronise the stream, return and clear the device status word (0 = ok)."""
     return lib().q4k_last_device_status(_stream(stream))
+
+
+def q4k_test_wait_fault(drop_stage: int = -1, wait_limit_ns: int = 0) -> None:
+    """Test hook: make the weight producers skip stage `drop_stage` (-1: off) and set the
+    bounded-wait limit (0: the 2 s default). Synchronous; see include/q4k.h."""
+    _check("q4k_test_wait_fault", lib().q4k_test_wait_fault(int(drop_stage), int(wait_limit_ns)))

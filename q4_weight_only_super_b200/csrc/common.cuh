@@ -16,6 +16,15 @@ constexpr int BLOCK_BYTES = 144;  // bytes per super-block
 // Device status word: 0 = no error latched. Kernels latch the first error.
 __device__ int g_status;
 
+// Limit of every bounded device-side wait, in ns of %globaltimer: 2 s by default,
+// far beyond any legal wait. A test may shorten it (q4k_test_wait_fault).
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+// Test hook (q4k_test_wait_fault): when >= 0, the weight producer of every CTA of the
+// prefill GEMM and the decode GEMVs skips its stage with this index -- neither the
+// copy nor the arrival happens -- so the roles waiting for that stage run into the
+// wait limit. -1 (the default) disables it.
+__device__ int g_test_drop_stage = -1;
+
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
 
 // ---- loads ---------------------------------------------------------------

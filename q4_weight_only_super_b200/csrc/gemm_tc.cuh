@@ -120,19 +120,50 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
-
 // Bounded wait; returns false (after latching a timeout) if the phase never
-// completes or another role has already aborted.
+// completes within g_wait_limit_ns or another role has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = *const_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > limit) {
+      latch_status(Q4K_ERR_DEVICE_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// As mbar_wait, with the limit passed in (read once per thread by the caller).
+__device__ __forceinline__ bool mbar_wait_l(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            uint64_t limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit) {
       latch_status(Q4K_ERR_DEVICE_TIMEOUT);
       *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// Wait for copies this CTA issued itself to land before it exits, whatever the
+// abort flag says (shared memory must not be released under an asynchronous
+// write); bounded by the same limit, after which it latches a timeout.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = *const_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (global_timer_ns() - t0 > limit) {
+      latch_status(Q4K_ERR_DEVICE_TIMEOUT);
       return false;
     }
   }
@@ -368,6 +399,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     if (warp == 0) {
       // ---------------- TMA producer ----------------
       if (lane == 0) {
+        const int drop = g_test_drop_stage;  // test hook; -1 in normal use
         int issued = 0;
         // weight rows of this tile in the [rows][row_bytes] view of W
         int wy0, wy1;
@@ -384,6 +416,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         for (int ks = 0; ks < nks; ++ks) {
           const int s = ks % kStagesAW, u = ks / kStagesAW;
           if (u >= 1 && !mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag)) break;
+          ++issued;
+          if (ks == drop) continue;  // test hook: this stage never arrives
           const uint32_t bytes = (GROUPED ? 0u : kATileBytes) + kWRawBytes;
           mbar_arrive_expect_tx(bar_full_aw(s), bytes);
           const uint32_t a_dst = sbase + kSmemA + s * kATileBytes;
@@ -400,17 +434,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
           tma_load_2d(w_dst + kWRawPart + 2048, &tmap_w, xq, wy1, bar_full_aw(s));
           tma_load_2d(w_dst + 2 * kWRawPart, &tmap_w, xq + 16, wy0, bar_full_aw(s));
           tma_load_2d(w_dst + 2 * kWRawPart + 2048, &tmap_w, xq + 16, wy1, bar_full_aw(s));
-          ++issued;
         }
         // Drain: every issued stage must have landed before this CTA may exit. On the
         // normal path the consumers have waited for all of them already.
         if (*abort_flag) {
-          for (int ks = (issued > kStagesAW ? issued - kStagesAW : 0); ks < issued; ++ks) {
-            const int s = ks % kStagesAW, u = ks / kStagesAW;
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(bar_full_aw(s), u & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
-            }
-          }
+          for (int ks = (issued > kStagesAW ? issued - kStagesAW : 0); ks < issued; ++ks)
+            if (ks != drop) mbar_wait_drain(bar_full_aw(ks % kStagesAW), (ks / kStagesAW) & 1);
         }
       }
     } else if (warp == 1) {

@@ -331,10 +331,10 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
 //  * Q5_K (176-byte super-blocks): the fifth bit of each quant is ORed into the
 //    nibble field before either A form is built, so q runs to 31 and the
 //    arithmetic stays exact (q*sc <= 1953 and 1024+16q <= 1520 in fp16).
-//  * Q8_0 (eight 34-byte blocks per 256-wide column): the subnormal form at
-//    every token count with A = q + 128 (0..255, the byte with its sign bit
-//    flipped), the block's d as the sub-block scale, and the -128 offset taken
-//    by the min-term MMA (A = d_j, against the sub-block sums, times 128).
+//  * Q8_0 (eight 34-byte blocks per 256-wide column): the per-sub-block scaling
+//    of the subnormal form at every token count, with A = the signed q itself as
+//    an fp16 integer (-128..127, exact) and the block's d as the sub-block scale;
+//    no min term.
 template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false, int QT = kQtQ4K>
 __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                                    GemvParams p) {
@@ -431,12 +431,21 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     // ---------------- weight producer: TMA ----------------
     if (lane == 0) {
       const int lim = SWIGLU ? p.N / 2 : p.N;
+      const int drop = g_test_drop_stage;  // test hook; -1 in normal use
       int issued = 0;
       int s = 0;
       uint32_t ph = 0;  // stage index and the parity of its current use (no divisions)
       for (int ks = 0; ks < nk; ++ks) {
         if (ks >= SW) mbar_wait(wempty(s), ph ^ 1u, abort_flag);
         if (*abort_flag) break;
+        if (ks == drop) {  // test hook: this stage never arrives
+          ++issued;
+          if (++s == SW) {
+            s = 0;
+            ph ^= 1u;
+          }
+          continue;
+        }
         mbar_arrive_expect_tx(wfull(s), (uint32_t)(WARPS * L::warp_tile));
         const uint32_t dst = smem_u32(smem) + (uint32_t)(s * L::wstage);
         const int x = (kb0 + ks) * BB / (Q80 ? 2 : 1);  // Q8_0: 16-bit elements (272 bytes = 136)
@@ -457,10 +466,10 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           ph ^= 1u;
         }
       }
-      // Every issued stage must land before the CTA exits (normally the
-      // consumers have already waited for all of them).
+      // Every issued stage must land before the CTA exits, abort or not (normally
+      // the consumers have already waited for all of them).
       for (int ks = (issued > SW ? issued - SW : 0); ks < issued; ++ks)
-        mbar_wait(wfull(ks % SW), (ks / SW) & 1, abort_flag);
+        if (ks != drop) mbar_wait_drain(wfull(ks % SW), (ks / SW) & 1);
     }
   } else if (warp == WARPS + 1) {
     // ---------------- activation producer: bulk copies of prepared records ----------------
@@ -484,7 +493,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         }
       }
       for (int ks = (issued > SX ? issued - SX : 0); ks < issued; ++ks)
-        mbar_wait(xfull(ks % SX), (ks / SX) & 1, abort_flag);
+        mbar_wait_drain(xfull(ks % SX), (ks / SX) & 1);
     }
   } else {
     // ---------------- consumers ----------------
@@ -620,7 +629,10 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
               if (Q80) {
                 // block j of this 256-wide column: fp16 d at byte 34j, q[8t .. 8t+7] at
                 // 34j + 2 + 8t (4-byte aligned for odd j; for even j two funnel shifts
-                // realign three aligned words), each byte's sign bit flipped: q + 128
+                // realign three aligned words), each byte's sign bit flipped: q + 128 in
+                // 0..255, the low byte of 0x6400 = 1024 + (q + 128); one fp16 add of -1152
+                // then leaves q itself, exact (the weight enters the MMA as the signed
+                // integer: no offset term whose cancellation would cost accuracy)
                 uint32_t xw[R][2];
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
@@ -646,10 +658,11 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
                   const int ra = 2 * tt, rb = 2 * tt + 1;
 #pragma unroll
                   for (int st = 0; st < 2; ++st) {  // bytes {0,2} and {1,3} into the low byte of each half
-                    A[tt][st][0] = __byte_perm(xw[ra][st], 0u, 0x4240u);
-                    A[tt][st][1] = __byte_perm(xw[rb][st], 0u, 0x4240u);
-                    A[tt][st][2] = __byte_perm(xw[ra][st], 0u, 0x4341u);
-                    A[tt][st][3] = __byte_perm(xw[rb][st], 0u, 0x4341u);
+                    const __half2 off = __float2half2_rn(-1152.f);
+                    A[tt][st][0] = h2_bits(__hadd2(bits_h2(__byte_perm(xw[ra][st], 0x64646464u, 0x4240u)), off));
+                    A[tt][st][1] = h2_bits(__hadd2(bits_h2(__byte_perm(xw[rb][st], 0x64646464u, 0x4240u)), off));
+                    A[tt][st][2] = h2_bits(__hadd2(bits_h2(__byte_perm(xw[ra][st], 0x64646464u, 0x4341u)), off));
+                    A[tt][st][3] = h2_bits(__hadd2(bits_h2(__byte_perm(xw[rb][st], 0x64646464u, 0x4341u)), off));
                   }
                 }
               } else {
@@ -745,11 +758,8 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
         const uint32_t mb = 2u * (t & 1);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          if (Q80) {  // A = (d_2t, d_2t+1): the fp16 scales at bytes 68t and 68t + 34
-            const uint8_t* rp = wt + (g + 8 * r) * L::pitch;
-            const uint32_t wlo = *reinterpret_cast<const uint32_t*>(rp + 68 * t);
-            const uint32_t whi = *reinterpret_cast<const uint32_t*>(rp + 68 * t + 32);
-            am[r] = __byte_perm(wlo, whi, 0x7610u);
+          if (Q80) {  // Q8_0 has no min term
+            am[r] = 0u;
           } else {
             am[r] = h2_bits(__hadd2(bits_h2(bytes_1024((t >> 1) ? mnw[r][1] : mnw[r][0], mb, mb + 1)),
                                     neg1024));
@@ -759,8 +769,9 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           // the subnormal form's products carry 2^-24: fold 2^24 into d
-          dd[r] = Q80 ? 16777216.f : (SUBN ? 16777216.f : 1.f) * half_bits_to_float(hdx[r]);
-          dn[r] = Q80 ? 64.f * 128.f : 64.f * half_bits_to_float(hdx[r] >> 16);
+          // (Q8_0: A is q itself and the block scales d_j are already in C)
+          dd[r] = Q80 ? 1.f : (SUBN ? 16777216.f : 1.f) * half_bits_to_float(hdx[r]);
+          dn[r] = Q80 ? 0.f : 64.f * half_bits_to_float(hdx[r] >> 16);
         }
 #pragma unroll
         for (int f = 0; f < MT; ++f) {
@@ -772,9 +783,11 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
           const float s1 = *reinterpret_cast<const float*>(xb + (8 * f + 2 * t + 1) * kXRec + 544);
 #pragma unroll
           for (int tt = 0; tt < TILES; ++tt) {
-            float Cm[4];
-            mma_f16_16816(Cm, am[2 * tt], am[2 * tt + 1], 0u, 0u, bh, 0u, true);
-            mma_f16_16816(Cm, am[2 * tt], am[2 * tt + 1], 0u, 0u, bl, 0u, false);
+            float Cm[4] = {0.f, 0.f, 0.f, 0.f};
+            if (!Q80) {
+              mma_f16_16816(Cm, am[2 * tt], am[2 * tt + 1], 0u, 0u, bh, 0u, true);
+              mma_f16_16816(Cm, am[2 * tt], am[2 * tt + 1], 0u, 0u, bl, 0u, false);
+            }
             const float dA = dd[2 * tt], dB = dd[2 * tt + 1], mA = dn[2 * tt], mB = dn[2 * tt + 1];
             acc[tt][f][0] = fmaf(-mA * s0, Cm[0], fmaf(dA * s0, C[tt][f][0], acc[tt][f][0]));
             acc[tt][f][1] = fmaf(-mA * s1, Cm[1], fmaf(dA * s1, C[tt][f][1], acc[tt][f][1]));

@@ -11,6 +11,7 @@
 #include "dequant.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_sk.cuh"
 #include "moe.cuh"
 
 using namespace q4k;
@@ -210,6 +211,95 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
   return launch_gemv_t<4, 4, 2, GROUPED, SWIGLU, REPACK, QT>(p, total_rows, tiles, groups, s);
 }
 
+// ------------------------------------------------ stationary GEMV (1..8 tokens) ----
+
+// sk_fit[d][tiles-1][P]: clusters of P stationary-GEMV CTAs (one per SM) resident at
+// once on device d.
+std::atomic<int> g_sk_fit[kMaxDevices][2][9];
+std::atomic<size_t> g_sk_smem_set[2][kMaxDevices];
+
+template <int TILES>
+q4k_status sk_cluster_fit_t(int P, int* fit) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices || P < 1 || P > 8) return Q4K_ERR_CUDA;
+  int v = g_sk_fit[dev][TILES - 1][P].load();
+  if (v <= 0) {
+    auto* k = gemv_sk_kernel<TILES>;
+    if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[TILES - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(P * 64), 1, 1);
+    cfg.blockDim = dim3(SkMax<TILES>::threads, 1, 1);
+    cfg.dynamicSmemBytes = kSkSmemBudget;  // one CTA per SM
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)P;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&v, k, &cfg) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      return Q4K_ERR_CUDA;
+    }
+    g_sk_fit[dev][TILES - 1][P].store(v);
+  }
+  *fit = v;
+  return Q4K_OK;
+}
+
+// The stationary GEMV's launch shape for an N x K matrix; *ok = false when the shape
+// is outside what it covers (more than 8 K parts).
+q4k_status pick_sk(int N, int nkb, SkCfg* c, bool* ok) {
+  *ok = false;
+  if (!sk_shape(N, nkb, c)) return Q4K_OK;
+  int fit = 0;
+  const q4k_status st = c->tiles == 2 ? sk_cluster_fit_t<2>(c->P, &fit) : sk_cluster_fit_t<1>(c->P, &fit);
+  if (st != Q4K_OK) return st;
+  *ok = sk_finish(fit, c);
+  return Q4K_OK;
+}
+
+template <int TILES>
+q4k_status launch_sk_t(const SkCfg& c, const void* W, const uint16_t* X, float* Y, int M, int N, int K,
+                       cudaStream_t s) {
+  auto* k = gemv_sk_kernel<TILES>;
+  if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[TILES - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
+  SkParams p = {};
+  p.W = static_cast<const uint8_t*>(W);
+  p.X = X;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nkb = K / QK;
+  p.P = c.P;
+  p.KU = c.KU;
+  p.units = c.units;
+  p.pitch = c.pitch;
+  p.stages = c.stages;
+  p.uslots = c.uslots;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)c.grid, 1, 1);
+  cfg.blockDim = dim3((unsigned)(32 * (c.KU + 2)), 1, 1);
+  cfg.dynamicSmemBytes = c.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)c.P;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = c.P > 1 ? 2 : 1;
+  return launch_status(cudaLaunchKernelEx(&cfg, k, p));
+}
+
+q4k_status launch_sk(const SkCfg& c, const void* W, const uint16_t* X, float* Y, int M, int N, int K,
+                     cudaStream_t s) {
+  return c.tiles == 2 ? launch_sk_t<2>(c, W, X, Y, M, N, K, s) : launch_sk_t<1>(c, W, X, Y, M, N, K, s);
+}
+
 // Routing kernels keep each lane's share of a logit row in registers: pick the
 // instantiation whose per-lane slot count PL covers E (E <= 32 * PL).
 template <typename F>
@@ -294,6 +384,14 @@ q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
   if (!aligned16(W) || !aligned16(X) || !aligned16(Y) || !aligned16(ws)) return Q4K_ERR_ALIGN;
   if (M > 32 || N % 16) return Q4K_ERR_UNSUPPORTED;
   if (ws_bytes < gemv_ws_bytes(M, K)) return Q4K_ERR_WORKSPACE;
+  if (M <= 8) {  // super-block-stationary kernel: no pre-pass, no workspace traffic
+    SkCfg sc;
+    bool ok = false;
+    const q4k_status st = pick_sk(N, K / QK, &sc, &ok);
+    if (st != Q4K_OK) return st;
+    // measured faster than the ring kernel where K is split over a cluster
+    if (ok && sc.tiles == 1 && sc.P > 1) return launch_sk(sc, W, X, Y, M, N, K, static_cast<cudaStream_t>(stream));
+  }
   GemvParams p = {};
   p.W = static_cast<const uint8_t*>(W);
   p.out = Y;
@@ -619,6 +717,17 @@ q4k_status moe_route_permute_hidden(const uint16_t* X, const uint16_t* W_router,
   }
   return moe_route_permute(logits, M, E, topk, topk_ids, topk_w, expert_offsets, perm, inv_perm, row_token, ws,
                            ws_bytes, stream);
+}
+
+q4k_status q4k_test_wait_fault(int drop_stage, uint64_t wait_limit_ns) {
+  const int drop = drop_stage < 0 ? -1 : drop_stage;
+  const unsigned long long lim = wait_limit_ns ? (unsigned long long)wait_limit_ns : 2000000000ull;
+  if (cudaMemcpyToSymbol(g_test_drop_stage, &drop, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_wait_limit_ns, &lim, sizeof(lim)) != cudaSuccess) {
+    cudaGetLastError();
+    return Q4K_ERR_CUDA;
+  }
+  return Q4K_OK;
 }
 
 q4k_status q4k_last_device_status(void* stream) {

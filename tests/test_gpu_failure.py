@@ -1,0 +1,60 @@
+"""Failure detection on the GPU without a fault: a bounded wait is made to expire.
+
+The library's test hook (q4k_test_wait_fault) shortens the wait limit to 200 us and
+makes the weight producer of every CTA skip its first stage -- no copy and no arrival
+-- so the roles waiting for it reach the limit. The kernel must return (no hang, no
+trap), latch Q4K_ERR_DEVICE_TIMEOUT (7) in the status word, leave the context usable,
+and the next normal call must be correct (fail closed: hipEngine 0.3.0 README, "Core
+principles").
+"""
+import numpy as np
+import pytest
+
+import synth
+from oracle import q4k as O
+from tests.gpu_util import dev, host
+
+pytestmark = pytest.mark.gpu
+
+q = pytest.importorskip("q4_weight_only_super_b200")
+
+TIMEOUT = 7  # Q4K_ERR_DEVICE_TIMEOUT
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    q.lib()
+    q.q4k_test_wait_fault(-1, 0)
+    assert q.q4k_last_device_status() == 0
+    yield
+    q.q4k_test_wait_fault(-1, 0)
+    assert q.q4k_last_device_status() == 0
+
+
+def _run(op):
+    if op.startswith("gemv"):
+        M = 1 if op == "gemv_1tok" else 17  # 1..8 tokens: stationary kernel; 17..32: ring kernel
+        N, K = 272, 256 * 69                 # K split over a cluster in both kernels
+        W, X = synth.gemv_small(990 + M, N=N, K=K, M=M)
+        return (lambda: q.q4k_gemv(dev(W), dev(X), N, K)), W, X
+    M, N, K = 300, 256, 1024
+    W, X = synth.gemv_small(995, N=N, K=K, M=M)
+    return (lambda: q.q4k_gemm(dev(W), dev(X), N, K)), W, X
+
+
+@pytest.mark.parametrize("op", ["gemv_1tok", "gemv_17tok", "gemm"])
+def test_bounded_wait_expires_and_recovers(op):
+    call, W, X = _run(op)
+    assert q.q4k_last_device_status() == 0
+    try:
+        q.q4k_test_wait_fault(0, 200_000)  # skip stage 0 everywhere; 200 us limit
+        call()
+        assert q.q4k_last_device_status() == TIMEOUT
+    finally:
+        q.q4k_test_wait_fault(-1, 0)
+    assert q.q4k_last_device_status() == 0
+    y = host(call())
+    assert q.q4k_last_device_status() == 0
+    Y, S = O.matmul_ref(W, X)
+    ok, ratio = O.check_tolerance(y, Y, S)
+    assert ok, f"{op} after a timeout: worst err/S = {ratio:.3e}"

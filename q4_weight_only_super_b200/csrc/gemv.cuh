@@ -64,16 +64,20 @@ namespace cg = cooperative_groups;
 constexpr int kXRec = 576;
 constexpr int kXPadRows = 32;  // zero records appended after the real rows
 
+// The MMA wrappers are plain (not volatile) asm: they have no side effects, so the
+// compiler may schedule independent MMAs (and their operand set-up) around one
+// another instead of keeping every MMA in program order; an MMA whose accumulator
+// comes from the previous one otherwise stalls the warp for its full latency.
 __device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                               uint32_t a3, uint32_t b0, uint32_t b1, bool zero_c) {
   if (zero_c) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%10,%10,%10,%10};"
         : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
   } else {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(256) gemv_prep_q8_kernel(const uint16_t* __res
 // m16n8k32 integer MMA, u8 A x s8 B -> s32, zero accumulator in.
 __device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                            uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%10,%10,%10,%10};"
       : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])

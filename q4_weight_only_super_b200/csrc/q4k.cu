@@ -213,22 +213,22 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
 
 // ------------------------------------------------ stationary GEMV (1..8 tokens) ----
 
-// sk_fit[d][tiles-1][P]: clusters of P stationary-GEMV CTAs (one per SM) resident at
+// sk_fit[d][kpw-1][P]: clusters of P stationary-GEMV CTAs (one per SM) resident at
 // once on device d.
 std::atomic<int> g_sk_fit[kMaxDevices][2][9];
 std::atomic<size_t> g_sk_smem_set[2][kMaxDevices];
 
-template <int TILES>
+template <int KPW>
 q4k_status sk_cluster_fit_t(int P, int* fit) {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices || P < 1 || P > 8) return Q4K_ERR_CUDA;
-  int v = g_sk_fit[dev][TILES - 1][P].load();
+  int v = g_sk_fit[dev][KPW - 1][P].load();
   if (v <= 0) {
-    auto* k = gemv_sk_kernel<TILES>;
-    if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[TILES - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
+    auto* k = gemv_sk_kernel<KPW>;
+    if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[KPW - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(P * 64), 1, 1);
-    cfg.blockDim = dim3(SkMax<TILES>::threads, 1, 1);
+    cfg.blockDim = dim3(SkMax<KPW>::threads, 1, 1);
     cfg.dynamicSmemBytes = kSkSmemBudget;  // one CTA per SM
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -241,7 +241,7 @@ q4k_status sk_cluster_fit_t(int P, int* fit) {
       cudaGetLastError();
       return Q4K_ERR_CUDA;
     }
-    g_sk_fit[dev][TILES - 1][P].store(v);
+    g_sk_fit[dev][KPW - 1][P].store(v);
   }
   *fit = v;
   return Q4K_OK;
@@ -253,17 +253,17 @@ q4k_status pick_sk(int N, int nkb, SkCfg* c, bool* ok) {
   *ok = false;
   if (!sk_shape(N, nkb, c)) return Q4K_OK;
   int fit = 0;
-  const q4k_status st = c->tiles == 2 ? sk_cluster_fit_t<2>(c->P, &fit) : sk_cluster_fit_t<1>(c->P, &fit);
-  if (st != Q4K_OK) return st;
+  const q4k_status st = c->kpw == 2 ? sk_cluster_fit_t<2>(c->P, &fit) : sk_cluster_fit_t<1>(c->P, &fit);
+  if (st != Q4K_OK) return Q4K_OK;  // not resident on this device: the ring kernel takes the shape
   *ok = sk_finish(fit, c);
   return Q4K_OK;
 }
 
-template <int TILES>
+template <int KPW>
 q4k_status launch_sk_t(const SkCfg& c, const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                        cudaStream_t s) {
-  auto* k = gemv_sk_kernel<TILES>;
-  if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[TILES - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
+  auto* k = gemv_sk_kernel<KPW>;
+  if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[KPW - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
   SkParams p = {};
   p.W = static_cast<const uint8_t*>(W);
   p.X = X;
@@ -274,13 +274,14 @@ q4k_status launch_sk_t(const SkCfg& c, const void* W, const uint16_t* X, float* 
   p.nkb = K / QK;
   p.P = c.P;
   p.KU = c.KU;
+  p.CW = c.CW;
   p.units = c.units;
   p.pitch = c.pitch;
   p.stages = c.stages;
   p.uslots = c.uslots;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)c.grid, 1, 1);
-  cfg.blockDim = dim3((unsigned)(32 * (c.KU + 2)), 1, 1);
+  cfg.blockDim = dim3((unsigned)(32 * (c.CW + 2)), 1, 1);
   cfg.dynamicSmemBytes = c.smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -297,7 +298,7 @@ q4k_status launch_sk_t(const SkCfg& c, const void* W, const uint16_t* X, float* 
 
 q4k_status launch_sk(const SkCfg& c, const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                      cudaStream_t s) {
-  return c.tiles == 2 ? launch_sk_t<2>(c, W, X, Y, M, N, K, s) : launch_sk_t<1>(c, W, X, Y, M, N, K, s);
+  return c.kpw == 2 ? launch_sk_t<2>(c, W, X, Y, M, N, K, s) : launch_sk_t<1>(c, W, X, Y, M, N, K, s);
 }
 
 // Routing kernels keep each lane's share of a logit row in registers: pick the
@@ -389,8 +390,7 @@ q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
     bool ok = false;
     const q4k_status st = pick_sk(N, K / QK, &sc, &ok);
     if (st != Q4K_OK) return st;
-    // measured faster than the ring kernel where K is split over a cluster
-    if (ok && sc.tiles == 1 && sc.P > 1) return launch_sk(sc, W, X, Y, M, N, K, static_cast<cudaStream_t>(stream));
+    if (ok) return launch_sk(sc, W, X, Y, M, N, K, static_cast<cudaStream_t>(stream));
   }
   GemvParams p = {};
   p.W = static_cast<const uint8_t*>(W);

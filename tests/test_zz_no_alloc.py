@@ -54,21 +54,42 @@ def _noalloc_via_c_abi(logits, topk):
     return st, out
 
 
+def _compare(logits_np, topk):
+    logits = dev(logits_np)
+    ref = q.moe_route_permute(logits, topk)
+    st, got = _noalloc_via_c_abi(logits, topk)
+    assert st == 0
+    for key in ("topk_ids", "expert_offsets", "perm", "inv_perm", "row_token"):
+        assert torch.equal(got[key], ref[key]), (logits_np.shape, topk, key)
+    dw = np.abs(host(got["topk_w"]).astype(np.float64) - host(ref["topk_w"]).astype(np.float64))
+    assert dw.max() <= ROUTE_W_TOL
+
+
 def test_noalloc_route_matches_workspace_entry_point(cuda_ok):
-    # Two calls in a row on the shared scratch: a large skewed prefill batch,
-    # then a small decode batch that reads the array the first call filled.
-    cases = [synth.moe_layer(4, 4096, E=128, H=256, F=256, hot=16)["logits"],
-             synth.moe_layer(5, 37, E=128, H=256, F=256)["logits"]]
-    for logits_np in cases:
-        logits = dev(logits_np)
-        ref = q.moe_route_permute(logits, 8)
-        st, got = _noalloc_via_c_abi(logits, 8)
-        assert st == 0
-        for key in ("topk_ids", "expert_offsets", "perm", "inv_perm", "row_token"):
-            assert torch.equal(got[key], ref[key]), key
-        dw = np.abs(host(got["topk_w"]).astype(np.float64) - host(ref["topk_w"]).astype(np.float64))
-        assert dw.max() <= ROUTE_W_TOL
+    # Calls back to back on the shared scratch: a large skewed prefill batch, then
+    # smaller batches that read the array the earlier calls filled. Up to 32 tokens
+    # the regular entry point routes in one CTA while this one always runs the
+    # per-tile kernels (one tile there), so those token counts pair the two paths.
+    rng = np.random.default_rng(77)
+    cases = [(synth.moe_layer(4, 4096, E=128, H=256, F=256, hot=16)["logits"], 8),
+             (synth.moe_layer(5, 37, E=128, H=256, F=256)["logits"], 8)]
+    cases += [(synth.moe_layer(3, M, E=128, H=256, F=256)["logits"], 8) for M in (1, 8, 32)]
+    cases += [((rng.standard_normal((70, 40)) * 2).astype(np.float32), 3),     # E = 40, top-3, 3 tiles
+              ((rng.standard_normal((9, 1000))).astype(np.float32), 16),       # E = 1000, top-16, 1 tile
+              (synth.moe_layer(3, 1, E=128, H=256, F=256)["logits"], 8)]       # again after those
+    for logits_np, topk in cases:
+        _compare(logits_np, topk)
     assert q.q4k_last_device_status() == 0
+
+
+def test_noalloc_route_zero_tokens(cuda_ok):
+    """M = 0: only the expert offsets are written, all zero."""
+    L = q.lib()
+    offs = torch.full((129,), -1, dtype=torch.int32, device="cuda")
+    st = L.moe_route_permute_noalloc(None, 0, 128, 8, None, None, ctypes.c_void_p(offs.data_ptr()), None, None,
+                                     None, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    assert torch.count_nonzero(offs).item() == 0
 
 
 def test_noalloc_route_rejects_problems_beyond_its_scratch(cuda_ok):

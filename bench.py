@@ -46,6 +46,8 @@ sys.path.insert(0, ROOT)
 METRIC = "Q4_K GEMV effective HBM GB/s (% of peak); prefill GEMM TFLOPS; MoE layer tokens/s"
 UNIT = "GB/s"
 BLOCK = 144
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e specification (about 8 TB/s), for the spec fraction
+MOE_EXPERT_BYTES = 1536 * 8 * BLOCK + 2048 * 3 * BLOCK  # one expert's Q4_K gate_up + down: 2,654,208 B
 
 
 def _peaks():
@@ -226,6 +228,7 @@ def build_workloads(torch, q, synth):
     Wp, Xp = synth.dense_prefill(2)
     W["pre"] = (dev(Wp), dev(Xp), Wp.shape[0], Wp.shape[1] * 256)
     W["pre_copies"] = [W["pre"][0]] + [W["pre"][0].clone() for _ in range(2)]
+    W["pre_bf16"] = torch.empty(Wp.shape[0] * Wp.shape[1] * 256, dtype=torch.bfloat16, device="cuda")
     del Wp, Xp
     md = synth.moe_decode(3, 32)
     W["moe_dec"] = {k: dev(md[k]) for k in ("logits", "X", "W_gate_up", "W_down")}
@@ -323,7 +326,8 @@ def run_step(q, tm, W):
             Y = W["dec_Y"][:M * N].view(M, N)
             fns = [lambda Wt=Wt: q.q4k_gemv(Wt, Xt, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_copies"][p]]
             tm.run_seq(f"gemv:{p}:M{M}", fns)
-            launches += 2 * len(fns)  # activation pre-pass + GEMV per call
+            # 1..8 tokens: one launch of the stationary GEMV; 9..32: activation pre-pass + ring GEMV
+            launches += (1 if M <= 8 else 2) * len(fns)
             fns = [lambda Wr=Wr: q.q4k_gemv_repacked(Wr, Xt, N, K, Y=Y, ws=W["ws"]) for Wr in W["dec_rep_copies"][p]]
             tm.run_seq(f"gemv_rep:{p}:M{M}", fns)
             launches += 2 * len(fns)
@@ -345,6 +349,12 @@ def run_step(q, tm, W):
         fns = [lambda Wt=Wt: q.q4k_gemm(Wt, Xt[:M], N, K, Y=Y) for Wt in W["pre_copies"]]
         tm.run_seq(f"gemm:M{M}", fns)
         launches += len(fns)
+    # the unfused chain at 4096 tokens: dequantise to bf16 (17408 x 5120), then the same
+    # tcgen05 GEMM reading bf16 weights
+    Y = W["pre_Y"][:4096 * N].view(4096, N)
+    tm.run("gemm_unfused:dequant", lambda: q.q4k_dequant(W["pre"][0], out_bf16=True, out=W["pre_bf16"]))
+    tm.run("gemm_unfused:gemm", lambda: q.bf16w_gemm(W["pre_bf16"], Xt, N, K, Y=Y))
+    launches += 2
     W["moe_dec"]["ws"] = W["ws"]
     import torch
     for staged in (True, False):
@@ -357,6 +367,21 @@ def run_step(q, tm, W):
         moe_layer_graph(torch, q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"])
         launches += 6
     return launches
+
+
+def read_roof(torch, tm, W):
+    """The bench's own read roof: a plain streaming reduction (torch amax over the bytes
+    viewed as fp32) over the same rotating gate+up weight copies, launched back to back
+    exactly like the GEMV."""
+    copies = [Wt.view(-1).view(torch.float32) for Wt in W["dec_copies"]["gate_up"]]
+    for Wt in copies:
+        Wt.amax()
+    tm.times.clear()
+    for _ in range(3):
+        tm.run_seq("roof", [lambda Wt=Wt: Wt.amax() for Wt in copies] * 2)
+    tm.collect()
+    t = min(tm.times.pop("roof"))
+    return copies[0].numel() * 4 / t / 1e9
 
 
 def e2e_gemv(torch, q, W, steps, warmup):
@@ -448,6 +473,18 @@ def summarize(tm, W, peaks):
         if f"{key}:M{M}:graph" in T:
             comp[f"{key}_M{M}_graph_us"] = round(T[f"{key}:M{M}:graph"] * 1e6, 2)
             comp[f"{key}_M{M}_graph_tokens_per_s"] = round(M / T[f"{key}:M{M}:graph"], 1)
+    if "gemm_unfused:gemm" in T:
+        tg, td = T["gemm_unfused:gemm"], T["gemm_unfused:dequant"]
+        comp["gemm_unfused_M4096_us"] = {"dequant_bf16": round(td * 1e6, 1), "bf16w_gemm": round(tg * 1e6, 1),
+                                         "total": round((td + tg) * 1e6, 1)}
+        comp["gemm_unfused_M4096_TFLOPS"] = round(2.0 * 4096 * N * K / (td + tg) / 1e12, 1)
+    for M, nd in W.get("moe_dec_distinct", {}).items():
+        wb = nd * MOE_EXPERT_BYTES
+        t = T[f"moe_dec:M{M}:layer"]
+        comp[f"moe_dec_M{M}_distinct_experts"] = nd
+        comp[f"moe_dec_M{M}_expert_bytes"] = wb
+        comp[f"moe_dec_M{M}_weight_GBps"] = round(wb / t / 1e9, 1)
+        comp[f"moe_dec_M{M}_hbm_bound_us"] = round(wb / (peaks["hbm"] * 1e9) * 1e6, 2)
     gbps = gemv_bytes / gemv_time / 1e9
     if "_rep_time" in comp:
         comp["gemv_repacked_all_GBps"] = round(gemv_bytes / comp.pop("_rep_time") / 1e9, 1)
@@ -499,6 +536,13 @@ def roofline_for(key, T, W, peaks, traffic=None):
         a = N * (K // 256) * BLOCK / t / 1e9
         return {"kernel": key, "bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": round(a / peaks["hbm"], 4), "traffic": traffic, "peak_source": peaks["src"] + " (copy)"}
+    if key.startswith("moe_dec") and key.endswith(":layer"):
+        M = int(key.split(":")[1][1:])
+        nd = W["moe_dec_distinct"][M]
+        a = nd * MOE_EXPERT_BYTES / t / 1e9
+        return {"kernel": key, "bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(a / peaks["hbm"], 4), "traffic": traffic, "peak_source": peaks["src"] + " (copy)",
+                "units": f"{nd} distinct experts x {MOE_EXPERT_BYTES} B (Q4_K gate_up + down)"}
     if key.startswith("moe_pre") and key.endswith(("gate_up", "down")):
         E, H, F = W["moe_dims"]
         rows = 4096 * 8
@@ -536,6 +580,69 @@ def cpu_oracle_gemv_sample(seconds_target=10.0):
         cores = os.cpu_count()
     return {"value": round(gbps, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{done} x (512 rows x 5120 Q4_K gate+up GEMV, M=1, dequant+fp64 matmul) in {dt:.1f} s"}
+
+
+def cpu_oracle_configs(seconds_each=1.5):
+    """The oracle on bounded samples of each workload, timed with one BLAS thread and
+    with all the host's threads (the dequantisation is numpy elementwise work on one
+    core either way; only the fp64 matmuls use the BLAS threads)."""
+    import synth
+    from oracle import q4k as O
+    try:
+        from threadpoolctl import threadpool_limits, threadpool_info
+        all_threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        threadpool_limits, all_threads = None, os.cpu_count()
+
+    def timed(fn):
+        done, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            done += 1
+            dt = time.perf_counter() - t0
+            if dt >= seconds_each:
+                return done, dt
+
+    rng = np.random.default_rng(11)
+    W0, X0 = synth.gemv_small(0)
+    Wg = synth.q4k_random_blocks(rng, 512, 5120)
+    Xg = synth.bf16_normal(rng, (32, 5120))
+    Wd = synth.q4k_random_blocks(rng, 128, 17408)
+    Xd = synth.bf16_normal(rng, (32, 17408))
+    Wp = synth.q4k_random_blocks(rng, 256, 5120)
+    Xp = synth.bf16_normal(rng, (512, 5120))
+    moe = synth.moe_layer(3, 1, E=128, H=2048, F=768)
+    sel = np.unique(O.route_topk(moe["logits"], 8)[0])  # the touched experts only
+    moe_w = (moe["W_gate_up"][sel], moe["W_down"][sel])
+    moe_l = moe["logits"][:, sel]
+    pre = synth.moe_layer(4, 2, E=128, H=2048, F=768, hot=16)  # 2 tokens of the skewed prefill layer
+    psel = np.unique(O.route_topk(pre["logits"], 8)[0])
+    pre_w = (pre["W_gate_up"][psel], pre["W_down"][psel])
+    pre_l = pre["logits"][:, psel]
+    cases = [
+        ("c0 GEMV 256x2048 M=1 (whole)", lambda: O.matmul_ref(W0, X0), 256 * 8 * BLOCK / 1e9, "GB/s"),
+        ("c1 GEMV gate+up 512-row sample of 34816x5120, M=32", lambda: O.matmul_ref(Wg, Xg), 512 * 20 * BLOCK / 1e9, "GB/s"),
+        ("c1 GEMV down 128-row sample of 5120x17408, M=32", lambda: O.matmul_ref(Wd, Xd), 128 * 68 * BLOCK / 1e9, "GB/s"),
+        ("c2 GEMM 512 tokens x 256-row sample of 17408x5120", lambda: O.matmul_ref(Wp, Xp), 2 * 512 * 256 * 5120 / 1e12,
+         "TFLOP/s"),
+        ("c3 MoE decode layer M=1 (routing + the 8 touched experts)",
+         lambda: O.moe_layer_ref(moe_l, moe["X"], moe_w[0], moe_w[1], 8), 1.0, "tokens/s"),
+        ("c4 MoE prefill layer, 2-token sample (routing + the touched experts)",
+         lambda: O.moe_layer_ref(pre_l, pre["X"], pre_w[0], pre_w[1], 8), 2.0, "tokens/s"),
+    ]
+    out = {}
+    for name, fn, units, unit in cases:
+        rec = {}
+        for label, n in (("1_thread", 1), ("all_threads", all_threads)):
+            if threadpool_limits is not None:
+                with threadpool_limits(limits=n):
+                    done, dt = timed(fn)
+            else:
+                done, dt = timed(fn)
+            rec[label] = round(done * units / dt, 6)
+        rec["unit"] = unit
+        out[name] = rec
+    return out, all_threads
 
 
 # ------------------------------------------------------------ read roof ---
@@ -726,7 +833,13 @@ def main():
     step_s = s_ev.elapsed_time(e_ev) * 1e-3 / args.steps
     assert q.q4k_last_device_status() == 0
 
+    # distinct experts each MoE decode batch touches (the routing result is the same every step)
+    W["moe_dec_distinct"] = {}
+    for M, b in W["moe_dec"].get("bufs", {}).items():
+        eo = b["route"]["expert_offsets"].cpu().numpy()
+        W["moe_dec_distinct"][M] = int(np.count_nonzero(np.diff(eo) > 0))
     gbps, comp, T, dom = summarize(tm, W, peaks)
+    roof_gbps = read_roof(torch, tm, W)
     total_bytes, h2d, d2h, e2e_times = e2e_gemv(torch, q, W, max(3, args.steps // 2), 2)
     e2e_gbps = total_bytes / float(np.mean(e2e_times)) / 1e9
 
@@ -753,11 +866,17 @@ def main():
                        "parallelism": "replicas" if world > 1 else "single GPU",
                        "moe_prefill_hot_experts": W["moe_pre_hot"]},
             "frac_of_hbm_peak": round(gbps_all / world / peaks["hbm"], 4),
+            "frac_of_spec_8TBps": round(gbps_all / world / SPEC_HBM_GBS, 4),
+            "read_roof": {"value": round(roof_gbps, 1), "unit": "GB/s",
+                          "how": "torch amax (fp32 view) over the same six rotating 100 MB gate+up copies, back to back"},
+            "frac_of_read_roof": round(gbps_all / world / roof_gbps, 4),
             "components": comp,
             "roofline": roofline_for(dom[0], T, W, peaks),
             "rooflines": [roofline_for(k, T, W, peaks) for k in ("gemv:gate_up:M1", "gemv:down:M1",
-                                                                  "gemv:gate_up:M32", "gemm:M4096",
-                                                                  "moe_pre:M4096:gate_up", "moe_pre:M4096:down")],
+                                                                  "gemv:gate_up:M32", "gemv:down:M32", "gemm:M4096",
+                                                                  "moe_pre:M4096:gate_up", "moe_pre:M4096:down",
+                                                                  "moe_dec:M1:layer", "moe_dec:M8:layer",
+                                                                  "moe_dec:M32:layer")],
             "e2e": {"value": round(e2e_all, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clocks,
@@ -765,7 +884,9 @@ def main():
             "peaks": peaks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_gemv_sample(10.0)
+            cb = cpu_oracle_gemv_sample(6.0)
+            cb["configs"], cb["threads_all"] = cpu_oracle_configs(1.5)
+            line["cpu_baseline"] = cb
         print(json.dumps(line))
     if world > 1:
         torch.distributed.destroy_process_group()

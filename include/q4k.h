@@ -171,6 +171,15 @@ q4k_status q4k_gemv_repacked(const void* Wr, const uint16_t* X, float* Y, int M,
 q4k_status q4k_gemm(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* The GEMM half of the unfused chain that q4k_gemm fuses: with the weights first
+ * dequantised to bf16 by q4k_dequant(out_bf16 = 1), this multiplies them with
+ * exactly q4k_gemm's tiles, tcgen05 MMAs and summation order, so
+ *   bf16w_gemm(q4k_dequant(W, bf16), X) == q4k_gemm(W, X)   bit for bit
+ * (hipEngine 0.3.0 README, "Core principles": every fused composite has a
+ * numerically equivalent unfused chain). Wb bf16 [N][K], X bf16 [M][K], Y fp32
+ * [M][N], all row-major; N % 256 == 0, K % 256 == 0; errors as q4k_gemm. */
+q4k_status bf16w_gemm(const uint16_t* Wb, const uint16_t* X, float* Y, int M, int N, int K, void* stream);
+
 /* Top-k routing and token permutation for a mixture-of-experts layer
  * (hipEngine 0.3.0 README, "Architecture at a glance": moe kernels).
  *   logits     fp32 [M][E] router logits.

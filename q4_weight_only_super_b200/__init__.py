@@ -14,7 +14,7 @@ import os
 import torch
 
 __all__ = [
-    "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemv_q8", "q5k_gemv", "q80_gemv", "q4k_repack", "q4k_gemv_repacked", "q4k_gemm",
+    "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemv_q8", "q5k_gemv", "q80_gemv", "q4k_repack", "q4k_gemv_repacked", "q4k_gemm", "bf16w_gemm",
     "moe_route_permute",
     "moe_route_permute_noalloc", "moe_route_permute_hidden",
     "moe_q4k_grouped", "moe_combine", "moe_combine_residual", "q4k_workspace_bytes", "q4k_last_device_status",
@@ -39,6 +39,7 @@ EXPORTS = {
     "q4k_repack": (_i, [_p, _i, _i, _p, _p]),
     "q4k_gemv_repacked": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "q4k_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
+    "bf16w_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p]),
     "moe_route_permute": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_route_permute_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
     "moe_route_permute_hidden": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
@@ -191,6 +192,15 @@ def q4k_gemm(W, X, N: int, K: int, Y=None, stream=None):
         Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
     _check("q4k_gemm", lib().q4k_gemm(_ptr(W), _ptr(_bits16(X)), _ptr(Y), M, N, K, None, 0,
                                       _stream(stream)))
+    return Y
+
+
+def bf16w_gemm(Wb, X, N: int, K: int, Y=None, stream=None):
+    """Y = X @ Wb^T with bf16 weights Wb [N][K] (the unfused chain's GEMM)."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
+    _check("bf16w_gemm", lib().bf16w_gemm(_ptr(_bits16(Wb)), _ptr(_bits16(X)), _ptr(Y), M, N, K, _stream(stream)))
     return Y
 
 

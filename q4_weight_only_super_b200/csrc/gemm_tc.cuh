@@ -59,7 +59,7 @@ constexpr uint32_t kSmemTotal = kSmemBar + 256;
 constexpr size_t kGemmSmemLaunch = kSmemTotal + 1024;  // + alignment slack
 
 struct GemmParams {
-  const uint8_t* W;        // dense [N][nkb][144]; grouped [E][N][nkb][144]
+  const uint8_t* W;        // dense [N][nkb][144]; grouped [E][N][nkb][144]; bf16-weight form: bf16 [N][K]
   const uint16_t* X;       // activations bf16 (dense [M][K]; grouped: rows of A)
   void* Y;                 // dense fp32 [M][N]; grouped fp32 [rows][N] or bf16 [rows][N/2]
   int M, N, K;
@@ -305,10 +305,16 @@ __device__ __forceinline__ void dequant_row_step(uint8_t* btile, int r, int chun
 
 // ---- the kernel -----------------------------------------------------------------
 
-template <bool GROUPED, bool SWIGLU>
+// BF16W: the weights arrive already dequantised, as bf16 [N][K] (the unfused chain:
+// q4k_dequant to bf16, then this GEMM); the producer loads each K step's weight tile
+// by TMA with the 128-byte swizzle -- the very layout the dequantising warps write --
+// and everything else (tiles, MMAs and their order, epilogue) is the fused GEMM's,
+// so the two give bit-identical results for the same bf16 weights.
+template <bool GROUPED, bool SWIGLU, bool BF16W = false>
 __global__ void __launch_bounds__(32 * (2 + kDqWarps + (GROUPED ? kGatherWarps : 0)), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                GemmParams p) {
+  static_assert(!BF16W || !GROUPED, "bf16-weight form: dense only");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, formed by pointer arithmetic on the shared array so the
   // compiler keeps the shared address space (plain LDS/STS, not generic accesses)
@@ -333,10 +339,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesAW; ++s) {
       mbar_init(bar_full_aw(s), GROUPED ? 1 + kGatherWarps : 1);
-      mbar_init(bar_empty_aw(s), 1 + kDqWarps);
+      mbar_init(bar_empty_aw(s), BF16W ? 1 : 1 + kDqWarps);
     }
     for (int s = 0; s < kStagesB; ++s) {
-      mbar_init(bar_full_b(s), kDqWarps);
+      mbar_init(bar_full_b(s), BF16W ? 1 : kDqWarps);
       mbar_init(bar_empty_b(s), 1);
     }
     mbar_init(bar_tmem_full, 1);
@@ -416,14 +422,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         for (int ks = 0; ks < nks; ++ks) {
           const int s = ks % kStagesAW, u = ks / kStagesAW;
           if (u >= 1 && !mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag)) break;
+          if (BF16W) {  // the weight tile's B stage must be free too
+            const int sb = ks % kStagesB, ub = ks / kStagesB;
+            if (ub >= 1 && !mbar_wait(bar_empty_b(sb), (ub - 1) & 1, abort_flag)) break;
+          }
           ++issued;
           if (ks == drop) continue;  // test hook: this stage never arrives
-          const uint32_t bytes = (GROUPED ? 0u : kATileBytes) + kWRawBytes;
+          const uint32_t bytes = (GROUPED ? 0u : kATileBytes) + (BF16W ? 0u : kWRawBytes);
           mbar_arrive_expect_tx(bar_full_aw(s), bytes);
           const uint32_t a_dst = sbase + kSmemA + s * kATileBytes;
           if (!GROUPED) {
             tma_load_2d(a_dst, &tmap_x, ks * kGemmBK, ay, bar_full_aw(s));
             tma_load_2d(a_dst + kATileBytes / 2, &tmap_x, ks * kGemmBK, ay + 128, bar_full_aw(s));
+          }
+          if (BF16W) {  // 256 weight rows x 64 bf16, 128-byte swizzled, into the B stage
+            const int sb = ks % kStagesB;
+            mbar_arrive_expect_tx(bar_full_b(sb), kBTileBytes);
+            tma_load_2d(sbase + kSmemB + sb * kBTileBytes, &tmap_w, ks * kGemmBK, n_tile * kGemmBN, bar_full_b(sb));
+            continue;
           }
           const int kb = ks >> 2, c = ks & 3;
           const int xh = kb * BLOCK_BYTES, xq = xh + 16 + 32 * c;
@@ -440,6 +456,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         if (*abort_flag) {
           for (int ks = (issued > kStagesAW ? issued - kStagesAW : 0); ks < issued; ++ks)
             if (ks != drop) mbar_wait_drain(bar_full_aw(ks % kStagesAW), (ks / kStagesAW) & 1);
+          if (BF16W)
+            for (int ks = (issued > kStagesB ? issued - kStagesB : 0); ks < issued; ++ks)
+              if (ks != drop) mbar_wait_drain(bar_full_b(ks % kStagesB), (ks / kStagesB) & 1);
         }
       }
     } else if (warp == 1) {
@@ -472,7 +491,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       // ---------------- dequantisation, then epilogue ----------------
       const int r = (warp - 2) * 32 + lane;  // weight row of the B tile (0..255)
       bool ok = true;
-      for (int ks = 0; ks < nks; ++ks) {
+      for (int ks = 0; ks < (BF16W ? 0 : nks); ++ks) {  // (bf16 weights: loaded by TMA)
         const int s = ks % kStagesAW, sb = ks % kStagesB, ub = ks / kStagesB;
         if (!__all_sync(0xffffffffu, mbar_wait(bar_full_aw(s), (ks / kStagesAW) & 1, abort_flag))) {
           ok = false;
@@ -483,13 +502,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
           ok = false;
           break;
         }
-        const uint8_t* wr = smem + kSmemW + s * kWRawBytes;
-        const uint4 hdr = *reinterpret_cast<const uint4*>(wr + r * 16);
-        const uint4 qa = *reinterpret_cast<const uint4*>(wr + kWRawPart + r * 16);
-        const uint4 qb = *reinterpret_cast<const uint4*>(wr + 2 * kWRawPart + r * 16);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty_aw(s));
-        dequant_row_step<GROUPED>(smem + kSmemB + sb * kBTileBytes, r, ks & 3, hdr, qa, qb);
+        {
+          const uint8_t* wr = smem + kSmemW + s * kWRawBytes;
+          const uint4 hdr = *reinterpret_cast<const uint4*>(wr + r * 16);
+          const uint4 qa = *reinterpret_cast<const uint4*>(wr + kWRawPart + r * 16);
+          const uint4 qb = *reinterpret_cast<const uint4*>(wr + 2 * kWRawPart + r * 16);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_empty_aw(s));
+          dequant_row_step<GROUPED>(smem + kSmemB + sb * kBTileBytes, r, ks & 3, hdr, qa, qb);
+        }
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_full_b(sb));
@@ -662,10 +683,10 @@ inline bool make_tmap_w(CUtensorMap* m, const void* base, int64_t rows, int64_t 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GROUPED, bool SWIGLU>
+template <bool GROUPED, bool SWIGLU, bool BF16W = false>
 inline q4k_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
                                 cudaStream_t s) {
-  auto* k = gemm_tc_kernel<GROUPED, SWIGLU>;
+  auto* k = gemm_tc_kernel<GROUPED, SWIGLU, BF16W>;
   static std::atomic<int> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -691,6 +712,29 @@ inline q4k_status launch_gemm_tc(GemmParams p, cudaStream_t s) {
   p.n_tiles = p.N / kGemmBN;
   p.m_tiles = (p.M + kGemmBM - 1) / kGemmBM;
   return launch_gemm_t<false, false>(tx, tw, p, s);
+}
+
+// bf16 weights [N][K], box 64 x 256 (one B stage), 128-byte swizzle.
+inline bool make_tmap_wb(CUtensorMap* m, const void* base, int64_t rows, int K) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, 256};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The GEMM of the unfused chain: bf16 weights [N][K] (e.g. from q4k_dequant), the
+// fused kernel's tiles and MMA order.
+inline q4k_status launch_gemm_tc_bf16w(GemmParams p, cudaStream_t s) {
+  CUtensorMap tx, tw;
+  if (!make_tmap_x(&tx, p.X, p.M, p.K) || !make_tmap_wb(&tw, p.W, p.N, p.K)) return Q4K_ERR_CUDA;
+  p.n_tiles = p.N / kGemmBN;
+  p.m_tiles = (p.M + kGemmBM - 1) / kGemmBM;
+  return launch_gemm_t<false, false, true>(tx, tw, p, s);
 }
 
 // Grouped: tasks are (expert, 256-row tile of that expert's rows); their number

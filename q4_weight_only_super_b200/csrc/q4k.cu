@@ -528,6 +528,22 @@ q4k_status q4k_gemm(const void* W, const uint16_t* X, float* Y, int M, int N, in
   return launch_gemm_tc(p, static_cast<cudaStream_t>(stream));
 }
 
+q4k_status bf16w_gemm(const uint16_t* Wb, const uint16_t* X, float* Y, int M, int N, int K, void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (M == 0 || N == 0) return Q4K_OK;
+  if (!Wb || !X || !Y) return Q4K_ERR_NULL;
+  if (!aligned16(Wb) || !aligned16(X) || !aligned16(Y)) return Q4K_ERR_ALIGN;
+  if (N % kGemmBN) return Q4K_ERR_UNSUPPORTED;
+  GemmParams p = {};
+  p.W = reinterpret_cast<const uint8_t*>(Wb);
+  p.X = X;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  return launch_gemm_tc_bf16w(p, static_cast<cudaStream_t>(stream));
+}
+
 size_t q4k_workspace_bytes(int op, int M, int N, int K, int E, int topk) {
   (void)N;
   (void)topk;

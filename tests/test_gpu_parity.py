@@ -475,6 +475,20 @@ def test_gemm_small(M, N, K):
     _assert_tol(y, Y, S, f"gemm M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (300, 768, 2048), (513, 1024, 5120)])
+def test_gemm_fused_equals_unfused_chain(M, N, K):
+    """q4k_gemm (dequantise into shared memory, then tcgen05) is bit-identical to the
+    unfused chain q4k_dequant(bf16) -> bf16w_gemm over the same tiles and MMA order
+    (hipEngine 0.3.0 README, "Core principles": fused composites have numerically
+    equivalent unfused chains)."""
+    W, X = synth.gemv_small(230 + M, N=N, K=K, M=M)
+    Wd, Xd = dev(W), dev(X)
+    fused = q.q4k_gemm(Wd, Xd, N, K)
+    Wb = q.q4k_dequant(Wd.reshape(-1), out_bf16=True).view(N, K)
+    unfused = q.bf16w_gemm(Wb, Xd, N, K)
+    assert torch.equal(fused, unfused)
+
+
 @pytest.fixture(scope="module")
 def prefill_inputs():
     W, X = synth.dense_prefill(2)

@@ -225,6 +225,12 @@ def build_workloads(torch, q, synth):
     W["dec_q80_copies"] = {"gate_up": [W["dec_q80"]["W_gate_up"], W["dec_q80"]["W_gate_up"].clone()],
                            "down": [W["dec_q80"]["W_down"]] + [W["dec_q80"]["W_down"].clone() for _ in range(2)]}
     del d8
+    # and in Q6_K (210-byte blocks): 4 x 146 MB (gate+up), 6 x 73 MB (down)
+    d6 = synth.dense_decode_q6(7)
+    W["dec_q6"] = {k: dev(v) for k, v in d6.items()}
+    W["dec_q6_copies"] = {"gate_up": [W["dec_q6"]["W_gate_up"]] + [W["dec_q6"]["W_gate_up"].clone() for _ in range(3)],
+                          "down": [W["dec_q6"]["W_down"]] + [W["dec_q6"]["W_down"].clone() for _ in range(5)]}
+    del d6
     Wp, Xp = synth.dense_prefill(2)
     W["pre"] = (dev(Wp), dev(Xp), Wp.shape[0], Wp.shape[1] * 256)
     W["pre_copies"] = [W["pre"][0]] + [W["pre"][0].clone() for _ in range(2)]
@@ -343,6 +349,10 @@ def run_step(q, tm, W):
                 fns = [lambda Wt=Wt: q.q80_gemv(Wt, X8, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_q80_copies"][p]]
                 tm.run_seq(f"gemv_q80:{p}:M{M}", fns)
                 launches += 2 * len(fns)
+                X6 = W["dec_q6"][f"X_{p}"][:M]
+                fns = [lambda Wt=Wt: q.q6k_gemv(Wt, X6, N, K, Y=Y, ws=W["ws"]) for Wt in W["dec_q6_copies"][p]]
+                tm.run_seq(f"gemv_q6:{p}:M{M}", fns)
+                launches += 2 * len(fns)
     _, Xt, N, K = W["pre"]
     for M in (512, 4096):
         Y = W["pre_Y"][:M * N].view(M, N)
@@ -454,6 +464,12 @@ def summarize(tm, W, peaks):
                 bq = N * (K // 256) * BLOCK
                 comp[f"gemv_q8lane_{p}_M{M}_GBps"] = round(bq / tq / 1e9, 1)
                 comp[f"gemv_q8lane_{p}_M{M}_us"] = round(tq * 1e6, 2)
+            t6 = T.get(f"gemv_q6:{p}:M{M}")
+            if t6:  # Q6_K: 210 bytes per super-block
+                N, K = W["dec_shapes"][p]
+                b6 = N * (K // 256) * 210
+                comp[f"gemv_q6k_{p}_M{M}_GBps"] = round(b6 / t6 / 1e9, 1)
+                comp[f"gemv_q6k_{p}_M{M}_us"] = round(t6 * 1e6, 2)
             t8 = T.get(f"gemv_q80:{p}:M{M}")
             if t8:  # Q8_0: 34 bytes per 32 weights
                 N, K = W["dec_shapes"][p]
@@ -502,6 +518,8 @@ def summarize(tm, W, peaks):
             n = len(W["dec_q5_copies"][k.split(":")[1]])
         elif k.startswith("gemv_q80:"):
             n = len(W["dec_q80_copies"][k.split(":")[1]])
+        elif k.startswith("gemv_q6:"):
+            n = len(W["dec_q6_copies"][k.split(":")[1]])
         elif k.startswith("gemm:"):
             n = len(W["pre_copies"])
         per_step[k] = v * n
@@ -696,7 +714,8 @@ def only(args):
         # weight format: Q4_K (default), Q5_K or Q8_0 at the same decode shapes
         gen, call, wpb = {"q4k": (lambda: synth.dense_decode(1), q.q4k_gemv, BLOCK),
                           "q5k": (lambda: synth.dense_decode_q5(5), q.q5k_gemv, 176),
-                          "q80": (lambda: synth.dense_decode_q80(6), q.q80_gemv, 272)}[args.quant]
+                          "q80": (lambda: synth.dense_decode_q80(6), q.q80_gemv, 272),
+                          "q6k": (lambda: synth.dense_decode_q6(7), q.q6k_gemv, 210)}[args.quant]
         dd = gen()
         Wt, Xt = dev(dd[f"W_{args.proj}"]), dev(dd[f"X_{args.proj}"][:M])
         N, K = dd[f"W_{args.proj}"].shape[0], dd["X_" + args.proj].shape[1]
@@ -752,7 +771,7 @@ def main():
                     help="run one kernel family a few times (for profiler captures), print times")
     ap.add_argument("--m", type=int, default=None, help="tokens for --only")
     ap.add_argument("--proj", default="gate_up", choices=["gate_up", "down"], help="GEMV matrix for --only")
-    ap.add_argument("--quant", default="q4k", choices=["q4k", "q5k", "q80"], help="GEMV weight format for --only")
+    ap.add_argument("--quant", default="q4k", choices=["q4k", "q5k", "q80", "q6k"], help="GEMV weight format for --only")
     ap.add_argument("--iters", type=int, default=3, help="launches for --only")
     args = ap.parse_args()
     if args.only:

@@ -113,6 +113,21 @@ q4k_status q4k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
 q4k_status q5k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* Decode GEMV over Q6_K weights, the remaining large tensor family of a Q4_K_M
+ * file (hipEngine 0.3.0 README, "GGUF Support": the tensor-family table lists
+ * Q6_K beside Q4_K, Q5_K and Q8_0). W [N][K/256] Q6_K blocks of 210 bytes:
+ * ql[128] (low four bits), qh[64] (high two bits), 16 signed byte scales, fp16
+ * d; weight i = 128n + 32u + l is nibble u/2 of ql[64n + 32(u%2) + l] plus 16 x
+ * bits 2u, 2u+1 of qh[32n + l], minus 32; w = d * scale[i/16] * q, q in
+ * -32..31. W must be 16-byte aligned (its rows are then 2-byte aligned: 210-byte
+ * blocks). The quants enter the tensor-core MMA exactly (q as an fp16 integer),
+ * the signed scales and d in fp32. Everything else -- X, Y, ws
+ * (q4k_workspace_bytes(Q4K_OP_GEMV, ...)), the shapes, errors and the
+ * activation representation -- as q4k_gemv; results are batch-invariant within
+ * each token class (1..8, 9..16, 17..32). */
+q4k_status q6k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K,
+                    void* ws, size_t ws_bytes, void* stream);
+
 /* The Q8 activation lane of the decode GEMV: an opt-in, accuracy-traded form of
  * q4k_gemv (hipster/hipEngine READMEs: the "fast" GEMV lane policy, dp4a route,
  * accuracy traded). Same arguments, workspace, shapes and errors as q4k_gemv.

@@ -14,7 +14,7 @@ import os
 import torch
 
 __all__ = [
-    "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemv_q8", "q5k_gemv", "q80_gemv", "q4k_repack", "q4k_gemv_repacked", "q4k_gemm", "bf16w_gemm",
+    "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemv_q8", "q5k_gemv", "q80_gemv", "q6k_gemv", "q4k_repack", "q4k_gemv_repacked", "q4k_gemm", "bf16w_gemm",
     "moe_route_permute",
     "moe_route_permute_noalloc", "moe_route_permute_hidden",
     "moe_q4k_grouped", "moe_combine", "moe_combine_residual", "q4k_workspace_bytes", "q4k_last_device_status",
@@ -34,6 +34,7 @@ EXPORTS = {
     "q4k_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "q5k_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "q80_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
+    "q6k_gemv": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "q4k_gemv_q8": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
     "q4k_repacked_bytes": (_i64, [_i, _i]),
     "q4k_repack": (_i, [_p, _i, _i, _p, _p]),
@@ -159,6 +160,18 @@ def q80_gemv(W, X, N: int, K: int, Y=None, ws=None, stream=None):
         Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
     ws = _scratch(q4k_workspace_bytes(OP_GEMV, M, N, K), X.device, ws)
     _check("q80_gemv", lib().q80_gemv(_ptr(W), _ptr(_bits16(X)), _ptr(Y), M, N, K, _ptr(ws), ws.numel(),
+                                      _stream(stream)))
+    return Y
+
+
+def q6k_gemv(W, X, N: int, K: int, Y=None, ws=None, stream=None):
+    """Decode GEMV over Q6_K weights [N][K/256][210]: Y[M][N] = X @ W^T."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
+    need = q4k_workspace_bytes(OP_GEMV, M, N, K)
+    ws = _scratch(need, X.device, ws)
+    _check("q6k_gemv", lib().q6k_gemv(_ptr(W), _ptr(_bits16(X)), _ptr(Y), M, N, K, _ptr(ws), ws.numel(),
                                       _stream(stream)))
     return Y
 

@@ -11,6 +11,7 @@
 #include "dequant.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_q6.cuh"
 #include "gemv_sk.cuh"
 #include "moe.cuh"
 
@@ -475,6 +476,36 @@ q4k_status q5k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
   c.wstages = kGemvStagesQ5[cls][0];
   c.xstages = kGemvStagesQ5[cls][1];
   return launch_gemv<false, false, false, kQtQ5K>(c, p, X, nullptr, M, K, ws, N, 1, static_cast<cudaStream_t>(stream));
+}
+
+q4k_status q6k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, int K, void* ws, size_t ws_bytes,
+                    void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (M == 0 || N == 0) return Q4K_OK;
+  if (!W || !X || !Y || !ws) return Q4K_ERR_NULL;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(Y) || !aligned16(ws)) return Q4K_ERR_ALIGN;
+  if (M > 32 || N % 16) return Q4K_ERR_UNSUPPORTED;
+  if (ws_bytes < gemv_ws_bytes(M, K)) return Q4K_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nkb = K / QK;
+  Q6Params p = {};
+  p.W = static_cast<const uint8_t*>(W);
+  p.xprep = static_cast<const uint8_t*>(ws);
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.nkb = nkb;
+  p.rows_pad = M + kXPadRows;
+  p.P = q6_parts(N, nkb);
+  const int64_t recs = (int64_t)p.rows_pad * nkb;
+  q4k_status st = launch_pdl(gemv_prep_kernel, dim3((unsigned)((recs + 7) / 8)), dim3(256), s, X,
+                             static_cast<const int32_t*>(nullptr), M, p.rows_pad, K, nkb, static_cast<uint8_t*>(ws));
+  if (st != Q4K_OK) return st;
+  const int T = kQ6Warps / p.P;
+  const dim3 grid((unsigned)((N / 16 + T - 1) / T));
+  if (M <= 8) return launch_pdl(q6k_gemv_kernel<1>, grid, dim3(32 * kQ6Warps), s, p);
+  if (M <= 16) return launch_pdl(q6k_gemv_kernel<2>, grid, dim3(32 * kQ6Warps), s, p);
+  return launch_pdl(q6k_gemv_kernel<4>, grid, dim3(32 * kQ6Warps), s, p);
 }
 
 q4k_status q4k_repack(const void* W, int N, int K, void* Wr, void* stream) {

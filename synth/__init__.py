@@ -204,6 +204,25 @@ def dense_decode_q80(seed: int = 6, Mmax: int = 32):
     return dict(W_gate_up=Wgu, W_down=Wdn, X_gate_up=Xgu, X_down=Xdn)
 
 
+def gemv_small_q6(seed: int = 0, N: int = 256, K: int = 2048, M: int = 1):
+    """Single-matrix Q6_K GEMV case. Order: W, X."""
+    rng = np.random.default_rng(seed)
+    W = q6k_random_blocks(rng, N, K)
+    X = bf16_normal(rng, (M, K))
+    return W, X
+
+
+def dense_decode_q6(seed: int = 7, Mmax: int = 32):
+    """The dense decode shapes with Q6_K weights. Order: W_gate_up, W_down, X_gate_up, X_down."""
+    rng = np.random.default_rng(seed)
+    (ngu, kgu), (ndn, kdn) = DENSE_DECODE["gate_up"], DENSE_DECODE["down"]
+    Wgu = q6k_random_blocks(rng, ngu, kgu)
+    Wdn = q6k_random_blocks(rng, ndn, kdn)
+    Xgu = bf16_normal(rng, (Mmax, kgu))
+    Xdn = bf16_normal(rng, (Mmax, kdn))
+    return dict(W_gate_up=Wgu, W_down=Wdn, X_gate_up=Xgu, X_down=Xdn)
+
+
 def dense_prefill(seed: int = 2, M: int = 4096, N: int = 17408, K: int = 5120):
     """Dense prefill GEMM: W [N][K] in Q4_K, X [M][K] bf16. Order: W, X."""
     rng = np.random.default_rng(seed)

@@ -184,6 +184,70 @@ def test_q5k_gemv_dense_decode_sampled(decode_inputs_q5, proj, M):
     _assert_tol(y[:, rows], Y, S, f"Q5_K {proj} M={M}")
 
 
+# ---------------------------------------------------------------- Q6_K GEMV --
+
+@pytest.mark.parametrize("N,K", [(16, 256), (48, 512), (272, 4096), (1040, 256 * 69)])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 17, 32])
+def test_q6k_gemv_shapes(N, K, M):
+    W, X = synth.gemv_small_q6(800 + M, N=N, K=K, M=M)
+    y = host(q.q6k_gemv(dev(W), dev(X), N, K))
+    Y, S = O.matmul_ref_q6(W, X)
+    _assert_tol(y, Y, S, f"Q6_K N={N} K={K} M={M}")
+
+
+def test_q6k_gemv_odd_block_count_rows():
+    """K = 256 * 69 (odd super-block count): every other row starts 2 bytes off a word."""
+    W, X = synth.gemv_small_q6(820, N=64, K=256 * 69, M=5)
+    y = host(q.q6k_gemv(dev(W), dev(X), 64, 256 * 69))
+    Y, S = O.matmul_ref_q6(W, X)
+    _assert_tol(y, Y, S, "Q6_K odd block count")
+
+
+def test_q6k_gemv_edge_blocks():
+    """Extreme Q6_K blocks: d = +-65504, subnormal d, zero; scales -128, 127, 0; q = -32, 31, 0."""
+    rng = np.random.default_rng(830)
+    N, K, M = 272, 256 * 5, 9
+    pool = np.stack([O.make_block_q6(d, sc, qv) for d in (65504.0, -65504.0, 6e-8, 0.0, -1.5)
+                     for sc in ([-128] * 16, [127] * 16, [0] * 16, list(range(-8, 8)))
+                     for qv in ([-32] * 256, [31] * 256, [0] * 256, list(rng.integers(-32, 32, 256)))])
+    W = synth.q6k_random_blocks(rng, N, K)
+    pick = rng.random(W.shape[:2]) < 0.5
+    W[pick] = pool[rng.integers(0, len(pool), W.shape[:2])[pick]]
+    X = synth.bf16_normal(rng, (M, K))
+    Y, S = O.matmul_ref_q6(W, X)
+    _assert_tol(host(q.q6k_gemv(dev(W), dev(X), N, K)), Y, S, "Q6_K edge blocks")
+
+
+@pytest.fixture(scope="module")
+def decode_inputs_q6():
+    inp = synth.dense_decode_q6(7)
+    d = {k: dev(v) for k, v in inp.items()}
+    return inp, d
+
+
+@pytest.mark.parametrize("proj", ["gate_up", "down"])
+@pytest.mark.parametrize("M", [1, 4, 8, 16, 32])
+def test_q6k_gemv_dense_decode_full(decode_inputs_q6, proj, M):
+    """Every output of the decode projections in Q6_K against the oracle, in row chunks."""
+    inp, d = decode_inputs_q6
+    W, X = inp[f"W_{proj}"], inp[f"X_{proj}"][:M]
+    N, K = W.shape[0], W.shape[1] * 256
+    y = host(q.q6k_gemv(d[f"W_{proj}"], d[f"X_{proj}"][:M], N, K))
+    for r0 in range(0, N, 4096):
+        Y, S = O.matmul_ref_q6(W[r0:r0 + 4096], X)
+        _assert_tol(y[:, r0:r0 + 4096], Y, S, f"Q6_K {proj} M={M} rows {r0}..")
+
+
+def test_q6k_gemv_batch_invariance():
+    """Within a token class a token's result does not depend on the rest of the batch."""
+    W, X = synth.gemv_small_q6(840, N=1040, K=256 * 69, M=32)
+    Wd, Xd = dev(W), dev(X)
+    y8 = q.q6k_gemv(Wd, Xd[:8], 1040, 256 * 69)
+    assert torch.equal(q.q6k_gemv(Wd, Xd[3:4], 1040, 256 * 69)[0], y8[3])
+    y32 = q.q6k_gemv(Wd, Xd, 1040, 256 * 69)
+    assert torch.equal(q.q6k_gemv(Wd, Xd[5:27], 1040, 256 * 69), y32[5:27])
+
+
 # ------------------------------------------------------------------ Q8 lane --
 
 def _q8lane_check(W, X, y, what):

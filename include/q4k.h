@@ -247,8 +247,15 @@ q4k_status moe_route_permute_noalloc(const float* logits, int M, int E, int topk
  *   expert_offsets int32 [E+1] (device): rows [off[e], off[e+1]) use expert e.
  *   rows       total rows = off[E] (host value; must match the device array).
  *   max_rows_hint  upper bound on any single expert's row count (for a
- *              top-k layer over M tokens: M). <= 32 selects the GEMV-style
- *              decode kernel (the arithmetic of q4k_gemv);
+ *              top-k layer over M tokens: M). <= 32 selects a decode kernel
+ *              with the arithmetic of q4k_gemv at 1..8 tokens: for K <= 5120
+ *              the grouped stationary GEMV (no activation pre-pass; any row
+ *              count per expert, 8 rows per pass over its weights; each row's
+ *              result bit-identical to q4k_gemv of that expert on up to 8 rows;
+ *              offsets that are not non-decreasing within [0, rows] latch
+ *              Q4K_ERR_DEVICE_BOUNDS and nothing is written), for longer K the
+ *              grouped ring GEMV (at most 32 rows per expert, else
+ *              Q4K_ERR_DEVICE_BOUNDS is latched);
  *              larger selects the tcgen05 grouped GEMM, whose operands are
  *              fp16: weights RN_fp16 of the fp32 dequant, activations
  *              converted from bf16 (|values| must stay below 65504, else
@@ -257,8 +264,8 @@ q4k_status moe_route_permute_noalloc(const float* logits, int M, int E, int topk
  *   act == Q4K_ACT_SWIGLU: out bf16 [rows][N/2], h = SiLU(g) * u with
  *              g = columns 0..N/2-1 (gate rows of W) and u = N/2..N-1 (up rows).
  *   ws/ws_bytes: device scratch of q4k_workspace_bytes(Q4K_OP_GROUPED, rows,
- *              N, K, E, 0) bytes (used by the decode kernel; may be NULL when
- *              max_rows_hint > 32).
+ *              N, K, E, 0) bytes (required when max_rows_hint <= 32, used by the
+ *              ring GEMV; may be NULL when max_rows_hint > 32).
  * N % 32 == 0 (SWIGLU: N/2 % 16 == 0), rows == 0 is a no-op. */
 q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uint16_t* A,
                            const int32_t* row_gather, const int32_t* expert_offsets,

@@ -13,6 +13,7 @@
 #include "gemv.cuh"
 #include "gemv_q6.cuh"
 #include "gemv_sk.cuh"
+#include "gemv_skg.cuh"
 #include "moe.cuh"
 
 using namespace q4k;
@@ -300,6 +301,66 @@ q4k_status launch_sk_t(const SkCfg& c, const void* W, const uint16_t* X, float* 
 q4k_status launch_sk(const SkCfg& c, const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                      cudaStream_t s) {
   return c.kpw == 2 ? launch_sk_t<2>(c, W, X, Y, M, N, K, s) : launch_sk_t<1>(c, W, X, Y, M, N, K, s);
+}
+
+// ------------------------------------ grouped stationary GEMV (MoE decode) ----
+
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  int v = g_sm_count[dev].load();
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) v = 0;
+    g_sm_count[dev].store(v);
+  }
+  return v;
+}
+
+// Shared memory one grouped-GEMV CTA may take: two CTAs per SM with one super-block
+// a warp (at most 20 warps of 96 registers: both fit), one with two.
+size_t skg_budget(int nkb) { return nkb > 10 ? kSkSmemBudget : kGemvTwoPerSm; }
+
+// Every CTA resident at once: the kernel deals the units over the whole grid.
+template <int KPW, bool SWIGLU>
+q4k_status launch_skg_t(const SkgCfg& c, const SkgParams& p, cudaStream_t s) {
+  auto* k = gemv_skg_kernel<KPW, SWIGLU>;
+  static std::atomic<size_t> smem_set[kMaxDevices];
+  // resident CTAs per SM for the last (threads, smem) asked on each device, packed
+  // as (threads << 40) | (smem << 8) | count
+  static std::atomic<uint64_t> occ[kMaxDevices];
+  if (ensure_smem(k, c.smem, smem_set) != cudaSuccess) return Q4K_ERR_LAUNCH;
+  const int dev = current_device();
+  const int threads = 32 * (c.CW + 2);
+  const uint64_t key = ((uint64_t)threads << 40) | ((uint64_t)c.smem << 8);
+  uint64_t o = occ[dev].load();
+  if ((o & ~(uint64_t)0xFF) != key) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, c.smem) != cudaSuccess || per_sm <= 0)
+      return launch_status(cudaErrorUnknown);
+    o = key | (uint64_t)std::min(per_sm, 255);
+    occ[dev].store(o);
+  }
+  const int grid = (int)(o & 0xFF) * sm_count();
+  if (grid <= 0) return Q4K_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = c.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return launch_status(cudaLaunchKernelEx(&cfg, k, p));
+}
+
+q4k_status launch_skg(const SkgCfg& c, const SkgParams& p, bool swiglu, cudaStream_t s) {
+  if (c.kpw == 2)
+    return swiglu ? launch_skg_t<2, true>(c, p, s) : launch_skg_t<2, false>(c, p, s);
+  return swiglu ? launch_skg_t<1, true>(c, p, s) : launch_skg_t<1, false>(c, p, s);
 }
 
 // Routing kernels keep each lane's share of a logit row in registers: pick the
@@ -682,6 +743,26 @@ q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uin
     if (!ws) return Q4K_ERR_NULL;
     if (!aligned16(ws)) return Q4K_ERR_ALIGN;
     if (ws_bytes < gemv_ws_bytes(rows, K)) return Q4K_ERR_WORKSPACE;
+    // K within one CTA's warps: the grouped stationary GEMV (no activation pre-pass,
+    // any number of rows per expert); else the ring kernel below
+    SkgCfg sc;
+    if (skg_shape(nkb, E, skg_budget(nkb), &sc) && ((int64_t)(rows + 7) / 8 + E) * (N / kSkRows) < 0x7fffffffLL) {
+      SkgParams sp = {};
+      sp.W = static_cast<const uint8_t*>(W_experts);
+      sp.A = A;
+      sp.gather = row_gather;
+      sp.offsets = expert_offsets;
+      sp.out = out;
+      sp.E = E;
+      sp.N = N;
+      sp.K = K;
+      sp.nkb = nkb;
+      sp.rows = rows;
+      sp.CW = sc.CW;
+      sp.pitch = sc.pitch;
+      sp.stages = sc.stages;
+      return launch_skg(sc, sp, act == Q4K_ACT_SWIGLU, s);
+    }
     GemvParams p = {};
     p.W = static_cast<const uint8_t*>(W_experts);
     p.out = out;

@@ -32,6 +32,15 @@ def _gpu(cuda_ok):
 
 
 def _run(op):
+    if op == "moe_dec":  # grouped stationary GEMV (MoE decode)
+        rng = np.random.default_rng(996)
+        E, N, K = 4, 256, 2048
+        W = np.stack([synth.q4k_random_blocks(rng, N, K) for _ in range(E)])
+        X = synth.bf16_normal(rng, (12, K))
+        offs = np.array([0, 3, 3, 11, 12], dtype=np.int32)
+        Wd, Xd, od = dev(W), dev(X), dev(offs)
+        call = lambda: q.moe_q4k_grouped(Wd, E, N, K, Xd, od, 12, 8, q.ACT_NONE)
+        return call, (W, offs), X
     if op.startswith("gemv"):
         M = 1 if op == "gemv_1tok" else 17  # 1..8 tokens: stationary kernel; 17..32: ring kernel
         N, K = 272, 256 * 69                 # K split over a cluster in both kernels
@@ -42,7 +51,7 @@ def _run(op):
     return (lambda: q.q4k_gemm(dev(W), dev(X), N, K)), W, X
 
 
-@pytest.mark.parametrize("op", ["gemv_1tok", "gemv_17tok", "gemm"])
+@pytest.mark.parametrize("op", ["gemv_1tok", "gemv_17tok", "gemm", "moe_dec"])
 def test_bounded_wait_expires_and_recovers(op):
     call, W, X = _run(op)
     assert q.q4k_last_device_status() == 0
@@ -55,6 +64,6 @@ def test_bounded_wait_expires_and_recovers(op):
     assert q.q4k_last_device_status() == 0
     y = host(call())
     assert q.q4k_last_device_status() == 0
-    Y, S = O.matmul_ref(W, X)
+    Y, S = O.grouped_ref(W[0], X, W[1]) if op == "moe_dec" else O.matmul_ref(W, X)
     ok, ratio = O.check_tolerance(y, Y, S)
     assert ok, f"{op} after a timeout: worst err/S = {ratio:.3e}"

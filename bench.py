@@ -370,12 +370,12 @@ def run_step(q, tm, W):
     for staged in (True, False):
         for M in (1, 8, 32):
             moe_layer_gpu(q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"], staged=staged)
-            launches += 6  # routing+permutation, 2 x (activation pre-pass + grouped GEMV), combine
+            launches += 4  # routing+permutation, grouped gate_up GEMV (+SwiGLU), grouped down GEMV, combine
         moe_layer_gpu(q, tm, "moe_pre:M4096", W["moe_pre"], 4096, W["moe_dims"], staged=staged)
         launches += 5  # routing, permutation, 2 grouped GEMMs, combine
     for M in (1, 8, 32):
         moe_layer_graph(torch, q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"])
-        launches += 6
+        launches += 4
     return launches
 
 

@@ -58,6 +58,28 @@ constexpr uint32_t kSmemBar = kSmemW + kStagesAW * kWRawBytes;
 constexpr uint32_t kSmemTotal = kSmemBar + 256;
 constexpr size_t kGemmSmemLaunch = kSmemTotal + 1024;  // + alignment slack
 
+// Shared-memory layout of one CTA. PAIR: a CTA pair (a cluster of two) computes a
+// 512-token x 256-weight-row tile with tcgen05.mma.cta_group::2 (M = 256, N = 256):
+// each CTA holds 256 token rows of A (two 128-row halves, one per MMA) and half the
+// weight tile -- 128 rows, which it alone dequantises -- and its TMEM receives its
+// own token rows x all 256 weight rows. Half the dequantisation per SM leaves room
+// for 4-deep rings.
+template <bool PAIR>
+struct GemmLayout {
+  static constexpr int SA = PAIR ? 4 : kStagesAW;                 // A (and raw weight) stages
+  static constexpr int SB = PAIR ? 4 : kStagesB;                  // B stages
+  static constexpr int BROWS = PAIR ? kGemmBN / 2 : kGemmBN;      // weight rows per CTA
+  static constexpr uint32_t BTile = (uint32_t)BROWS * 128;        // bytes per B stage
+  static constexpr uint32_t WPart = (uint32_t)BROWS * 16;         // one 16-byte column of the rows
+  static constexpr uint32_t WRaw = 3 * WPart;                     // header, quants 0-15, quants 16-31
+  static constexpr uint32_t SmemB = kSmemA + SA * kATileBytes;
+  static constexpr uint32_t SmemW = SmemB + SB * BTile;
+  static constexpr uint32_t SmemBar = SmemW + SA * WRaw;
+  static constexpr size_t Launch = SmemBar + 256 + 1024;          // + barriers, + alignment slack
+};
+static_assert(GemmLayout<false>::SmemBar == kSmemBar, "one-CTA layout unchanged");
+static_assert(GemmLayout<true>::Launch <= 232448, "pair layout fits one SM's shared memory");
+
 struct GemmParams {
   const uint8_t* W;        // dense [N][nkb][144]; grouped [E][N][nkb][144]; bf16-weight form: bf16 [N][K]
   const uint16_t* X;       // activations bf16 (dense [M][K]; grouped: rows of A)
@@ -169,6 +191,33 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
+// As mbar_wait, with cluster-scope acquire: for a barrier that a thread of the
+// other CTA of the cluster arrives on (release, cluster scope).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  auto try_once = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (try_once()) return true;
+  const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = *const_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+  for (;;) {
+    if (try_once()) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > limit) {
+      latch_status(Q4K_ERR_DEVICE_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
   asm volatile(
@@ -202,6 +251,9 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
 constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
                                 ((uint32_t)(128 >> 4) << 24);
 constexpr uint32_t kIdescF16 = (1u << 4) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+// bf16 x bf16 -> fp32, K-major, M=256 (a CTA pair, 128 rows each), N=256
+constexpr uint32_t kIdescBf16Pair = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                                    ((uint32_t)(256 >> 4) << 24);
 
 __device__ __forceinline__ void umma_f16kind(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                              uint32_t idesc, uint32_t accumulate) {
@@ -216,6 +268,48 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
       : "memory");
+}
+
+// The CTA-pair MMA (issued by the even CTA of the cluster): A rows 0..127 from
+// this CTA's shared memory and 128..255 from the peer's, at the same offsets; B
+// rows (weight rows) 0..127 from this CTA, 128..255 from the peer; D rows 0..127
+// into this CTA's TMEM and 128..255 into the peer's, at the same address.
+__device__ __forceinline__ void umma2_f16kind(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Completion of the pair's MMAs issued so far, signalled on the barrier at this
+// offset in both CTAs of the pair.
+__device__ __forceinline__ void umma2_commit_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+// Arrive (release, cluster scope) on the barrier at this offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, uint32_t rank) {
+  asm volatile(
+      "{\n .reg .b32 ra;\n mapa.shared::cluster.u32 ra, %0, %1;\n"
+      " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}" ::"r"(bar),
+      "r"(rank)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of both CTAs of the cluster (release / acquire).
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
@@ -271,36 +365,41 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return F16 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
 }
 
-// Dequantise weight row `r` for K step `ks` (super-block ks/4, chunk ks%4)
-// from its raw header (16 B) and 32 quant bytes into the swizzled B tile.
+// Dequantise half H of weight row `r`'s K step (super-block ks/4, chunk ks%4: the
+// 32 weights of sub-block 2*chunk + H) from its raw header (16 B) and 32 quant
+// bytes into the swizzled B tile.
+template <bool F16, int H>
+__device__ __forceinline__ void dequant_row_half(uint8_t* btile, int r, int chunk, uint4 hdr, uint4 qa, uint4 qb) {
+  const float d = half_bits_to_float(hdr.x), dmin = half_bits_to_float(hdr.x >> 16);
+  const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};  // bytes l = 4i..4i+3
+  uint32_t sc, m;
+  scale_min(hdr.y, hdr.z, hdr.w, 2 * chunk + H, sc, m);
+  const float ds = d * (float)sc;   // exact
+  const float dm = dmin * (float)m; // exact
+  const float cA = -ds * __uint_as_float((uint32_t)(127 + 23 - 4 * H) << 23);
+  const float cB = -ds * __uint_as_float((uint32_t)(127 + 15 - 4 * H) << 23);
+  if (F16 && fmaf(15.f, fabsf(ds), fabsf(dm)) > 65504.f) latch_status(Q4K_ERR_DEVICE_RANGE);
+#pragma unroll
+  for (int c8 = 0; c8 < 4; ++c8) {  // 8 weights: l = 8*c8 .. 8*c8+7 of the sub-block
+    float w0[4], w1[4];
+    dq4(qw[2 * c8], H, ds, dm, cA, cB, w0);
+    dq4(qw[2 * c8 + 1], H, ds, dm, cA, cB, w1);
+    // dq4 returns weights in byte order (b0, b1, b2, b3)
+    uint4 o;
+    o.x = pack2<F16>(w0[0], w0[1]);
+    o.y = pack2<F16>(w0[2], w0[3]);
+    o.z = pack2<F16>(w1[0], w1[1]);
+    o.w = pack2<F16>(w1[2], w1[3]);
+    *reinterpret_cast<uint4*>(btile + sw128_offset(r, 4 * H + c8)) = o;
+  }
+}
+
+// Both halves of weight row `r`'s K step.
 template <bool F16>
 __device__ __forceinline__ void dequant_row_step(uint8_t* btile, int r, int chunk, uint4 hdr, uint4 qa,
                                                  uint4 qb) {
-  const float d = half_bits_to_float(hdr.x), dmin = half_bits_to_float(hdr.x >> 16);
-  const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};  // bytes l = 4i..4i+3
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t sc, m;
-    scale_min(hdr.y, hdr.z, hdr.w, 2 * chunk + h, sc, m);
-    const float ds = d * (float)sc;   // exact
-    const float dm = dmin * (float)m; // exact
-    const float cA = -ds * __uint_as_float((uint32_t)(127 + 23 - 4 * h) << 23);
-    const float cB = -ds * __uint_as_float((uint32_t)(127 + 15 - 4 * h) << 23);
-    if (F16 && fmaf(15.f, fabsf(ds), fabsf(dm)) > 65504.f) latch_status(Q4K_ERR_DEVICE_RANGE);
-#pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8) {  // 8 weights: l = 8*c8 .. 8*c8+7 of sub-block 2*chunk+h
-      float w0[4], w1[4];
-      dq4(qw[2 * c8], h, ds, dm, cA, cB, w0);
-      dq4(qw[2 * c8 + 1], h, ds, dm, cA, cB, w1);
-      // dq4 returns weights in byte order (b0, b1, b2, b3)
-      uint4 o;
-      o.x = pack2<F16>(w0[0], w0[1]);
-      o.y = pack2<F16>(w0[2], w0[3]);
-      o.z = pack2<F16>(w1[0], w1[1]);
-      o.w = pack2<F16>(w1[2], w1[3]);
-      *reinterpret_cast<uint4*>(btile + sw128_offset(r, 4 * h + c8)) = o;
-    }
-  }
+  dequant_row_half<F16, 0>(btile, r, chunk, hdr, qa, qb);
+  dequant_row_half<F16, 1>(btile, r, chunk, hdr, qa, qb);
 }
 
 // ---- the kernel -----------------------------------------------------------------
@@ -310,11 +409,14 @@ __device__ __forceinline__ void dequant_row_step(uint8_t* btile, int r, int chun
 // by TMA with the 128-byte swizzle -- the very layout the dequantising warps write --
 // and everything else (tiles, MMAs and their order, epilogue) is the fused GEMM's,
 // so the two give bit-identical results for the same bf16 weights.
-template <bool GROUPED, bool SWIGLU, bool BF16W = false>
+template <bool GROUPED, bool SWIGLU, bool BF16W = false, bool PAIR = false>
 __global__ void __launch_bounds__(32 * (2 + kDqWarps + (GROUPED ? kGatherWarps : 0)), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                GemmParams p) {
   static_assert(!BF16W || !GROUPED, "bf16-weight form: dense only");
+  static_assert(!PAIR || !GROUPED, "CTA pairs: dense only");
+  using LY = GemmLayout<PAIR>;
+  constexpr int SA = LY::SA, SB = LY::SB;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, formed by pointer arithmetic on the shared array so the
   // compiler keeps the shared address space (plain LDS/STS, not generic accesses)
@@ -322,36 +424,45 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // barriers (8 bytes each) at kSmemBar: [0..2] full_aw, [3..5] empty_aw, [6..7] fullB,
-  // [8..9] emptyB, [10] tmem_full
-  auto bar_full_aw = [&](int s) { return sbase + kSmemBar + 8u * s; };
-  auto bar_empty_aw = [&](int s) { return sbase + kSmemBar + 8u * (3 + s); };
-  auto bar_full_b = [&](int s) { return sbase + kSmemBar + 8u * (6 + s); };
-  auto bar_empty_b = [&](int s) { return sbase + kSmemBar + 8u * (8 + s); };
-  const uint32_t bar_tmem_full = sbase + kSmemBar + 8u * 10;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kSmemBar + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemBar + 132);
-  int* task_info = reinterpret_cast<int*>(smem + kSmemBar + 136);  // expert, row_base, count, m0
+  // barriers (8 bytes each) at SmemBar: [0..3] full_aw, [4..7] empty_aw, [8..11] full_b,
+  // [12..15] empty_b, [16] tmem_full, [17..20] pair_full (PAIR, bf16 weights: the odd
+  // CTA's stage is ready, arrived on in the even CTA)
+  auto bar_full_aw = [&](int s) { return sbase + LY::SmemBar + 8u * s; };
+  auto bar_empty_aw = [&](int s) { return sbase + LY::SmemBar + 8u * (4 + s); };
+  auto bar_full_b = [&](int s) { return sbase + LY::SmemBar + 8u * (8 + s); };
+  auto bar_empty_b = [&](int s) { return sbase + LY::SmemBar + 8u * (12 + s); };
+  const uint32_t bar_tmem_full = sbase + LY::SmemBar + 8u * 16;
+  auto bar_pair_full = [&](int s) { return sbase + LY::SmemBar + 8u * (17 + s); };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + LY::SmemBar + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::SmemBar + 196);
+  int* task_info = reinterpret_cast<int*>(smem + LY::SmemBar + 200);  // expert, row_base, count, m0
 
   // ---- tile coordinates ----
-  const int n_tile = (int)(blockIdx.x % (unsigned)p.n_tiles);
-  const int task = (int)(blockIdx.x / (unsigned)p.n_tiles);
+  // PAIR: CTAs 2i and 2i+1 form cluster i (rank = blockIdx.x % 2) and share its tile
+  const int rank = PAIR ? (int)(blockIdx.x & 1u) : 0;
+  const unsigned tile_id = PAIR ? blockIdx.x >> 1 : blockIdx.x;
+  const int n_tile = (int)(tile_id % (unsigned)p.n_tiles);
+  const int task = (int)(tile_id / (unsigned)p.n_tiles);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStagesAW; ++s) {
+    for (int s = 0; s < SA; ++s) {
       mbar_init(bar_full_aw(s), GROUPED ? 1 + kGatherWarps : 1);
       mbar_init(bar_empty_aw(s), BF16W ? 1 : 1 + kDqWarps);
     }
-    for (int s = 0; s < kStagesB; ++s) {
+    // PAIR: the even CTA's full_b also takes the odd CTA's dequantising warps (remote
+    // arrivals, made after they have seen their own stage's copies land)
+    for (int s = 0; s < SB; ++s) {
       mbar_init(bar_full_b(s), BF16W ? 1 : kDqWarps);
       mbar_init(bar_empty_b(s), 1);
     }
+    if (PAIR)
+      for (int s = 0; s < SA; ++s) mbar_init(bar_pair_full(s), 1);
     mbar_init(bar_tmem_full, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    // Resolve the task: dense -> m tile; grouped -> (expert, m tile within expert).
-    int expert = 0, row_base = 0, count = p.M, m0 = task * kGemmBM;
+    // Resolve the task: dense -> m tile (PAIR: 512 tokens); grouped -> (expert, m tile within expert).
+    int expert = 0, row_base = 0, count = p.M, m0 = task * (PAIR ? 2 * kGemmBM : kGemmBM);
     if (GROUPED) {
       int seen = 0;
       expert = -1;
@@ -388,13 +499,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     }
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
-                     smem_u32(const_cast<uint32_t*>(tmem_slot)))
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (PAIR) {  // warp 1 of both CTAs, the same slot offset: the same TMEM address in each
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                       smem_u32(const_cast<uint32_t*>(tmem_slot)))
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                       smem_u32(const_cast<uint32_t*>(tmem_slot)))
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_barrier();  // both CTAs' barriers initialised and TMEM allocated
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int expert = task_info[0], row_base = task_info[1], count = task_info[2], m0 = task_info[3];
@@ -415,35 +536,45 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
           wy0 = (GROUPED ? expert * p.N : 0) + g0;
           wy1 = wy0 + half;
         } else {
-          wy0 = (GROUPED ? expert * p.N : 0) + n_tile * kGemmBN;
+          // PAIR: this CTA's 128 of the tile's 256 weight rows
+          wy0 = (GROUPED ? expert * p.N : 0) + n_tile * kGemmBN + (PAIR ? 128 * rank : 0);
           wy1 = wy0 + kGemmBN / 2;
         }
-        const int ay = GROUPED ? row_base + m0 : m0;
+        // token rows of the two A halves (PAIR: MMA h takes tokens m0 + 256h + 128 rank ..)
+        const int ay = GROUPED ? row_base + m0 : m0 + (PAIR ? 128 * rank : 0);
+        const int ay1 = ay + (PAIR ? 256 : 128);
         for (int ks = 0; ks < nks; ++ks) {
-          const int s = ks % kStagesAW, u = ks / kStagesAW;
+          const int s = ks % SA, u = ks / SA;
           if (u >= 1 && !mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag)) break;
           if (BF16W) {  // the weight tile's B stage must be free too
-            const int sb = ks % kStagesB, ub = ks / kStagesB;
+            const int sb = ks % SB, ub = ks / SB;
             if (ub >= 1 && !mbar_wait(bar_empty_b(sb), (ub - 1) & 1, abort_flag)) break;
           }
           ++issued;
           if (ks == drop) continue;  // test hook: this stage never arrives
-          const uint32_t bytes = (GROUPED ? 0u : kATileBytes) + (BF16W ? 0u : kWRawBytes);
+          const uint32_t bytes = (GROUPED ? 0u : kATileBytes) + (BF16W ? 0u : LY::WRaw);
           mbar_arrive_expect_tx(bar_full_aw(s), bytes);
           const uint32_t a_dst = sbase + kSmemA + s * kATileBytes;
           if (!GROUPED) {
             tma_load_2d(a_dst, &tmap_x, ks * kGemmBK, ay, bar_full_aw(s));
-            tma_load_2d(a_dst + kATileBytes / 2, &tmap_x, ks * kGemmBK, ay + 128, bar_full_aw(s));
+            tma_load_2d(a_dst + kATileBytes / 2, &tmap_x, ks * kGemmBK, ay1, bar_full_aw(s));
           }
-          if (BF16W) {  // 256 weight rows x 64 bf16, 128-byte swizzled, into the B stage
-            const int sb = ks % kStagesB;
-            mbar_arrive_expect_tx(bar_full_b(sb), kBTileBytes);
-            tma_load_2d(sbase + kSmemB + sb * kBTileBytes, &tmap_w, ks * kGemmBK, n_tile * kGemmBN, bar_full_b(sb));
+          if (BF16W) {  // the CTA's weight rows x 64 bf16, 128-byte swizzled, into the B stage
+            const int sb = ks % SB;
+            mbar_arrive_expect_tx(bar_full_b(sb), LY::BTile);
+            tma_load_2d(sbase + LY::SmemB + sb * LY::BTile, &tmap_w, ks * kGemmBK,
+                        n_tile * kGemmBN + (PAIR ? 128 * rank : 0), bar_full_b(sb));
             continue;
           }
           const int kb = ks >> 2, c = ks & 3;
           const int xh = kb * BLOCK_BYTES, xq = xh + 16 + 32 * c;
-          const uint32_t w_dst = sbase + kSmemW + s * kWRawBytes;
+          const uint32_t w_dst = sbase + LY::SmemW + s * LY::WRaw;
+          if (PAIR) {  // 128 rows: one box per 16-byte column
+            tma_load_2d(w_dst, &tmap_w, xh, wy0, bar_full_aw(s));
+            tma_load_2d(w_dst + LY::WPart, &tmap_w, xq, wy0, bar_full_aw(s));
+            tma_load_2d(w_dst + 2 * LY::WPart, &tmap_w, xq + 16, wy0, bar_full_aw(s));
+            continue;
+          }
           tma_load_2d(w_dst, &tmap_w, xh, wy0, bar_full_aw(s));
           tma_load_2d(w_dst + 2048, &tmap_w, xh, wy1, bar_full_aw(s));
           tma_load_2d(w_dst + kWRawPart, &tmap_w, xq, wy0, bar_full_aw(s));
@@ -454,46 +585,68 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         // Drain: every issued stage must have landed before this CTA may exit. On the
         // normal path the consumers have waited for all of them already.
         if (*abort_flag) {
-          for (int ks = (issued > kStagesAW ? issued - kStagesAW : 0); ks < issued; ++ks)
-            if (ks != drop) mbar_wait_drain(bar_full_aw(ks % kStagesAW), (ks / kStagesAW) & 1);
+          for (int ks = (issued > SA ? issued - SA : 0); ks < issued; ++ks)
+            if (ks != drop) mbar_wait_drain(bar_full_aw(ks % SA), (ks / SA) & 1);
           if (BF16W)
-            for (int ks = (issued > kStagesB ? issued - kStagesB : 0); ks < issued; ++ks)
-              if (ks != drop) mbar_wait_drain(bar_full_b(ks % kStagesB), (ks / kStagesB) & 1);
+            for (int ks = (issued > SB ? issued - SB : 0); ks < issued; ++ks)
+              if (ks != drop) mbar_wait_drain(bar_full_b(ks % SB), (ks / SB) & 1);
         }
       }
     } else if (warp == 1) {
       // ---------------- MMA issuer ----------------
+      // PAIR: the even CTA issues the pair's MMAs. Its full_b also counts the odd CTA's
+      // dequantising warps, which arrive once their own stage's copies (A included) have
+      // landed and their B half is written. With bf16 weights (no dequantising warps) the
+      // odd CTA's lane relays "my stage is ready" instead (a remote arrive on pair_full).
       if (lane == 0) {
         bool ok = true;
         for (int ks = 0; ks < nks && ok; ++ks) {
-          const int s = ks % kStagesAW, sb = ks % kStagesB;
-          ok = mbar_wait(bar_full_aw(s), (ks / kStagesAW) & 1, abort_flag) &&
-               mbar_wait(bar_full_b(sb), (ks / kStagesB) & 1, abort_flag);
+          const int s = ks % SA, sb = ks % SB;
+          ok = mbar_wait(bar_full_aw(s), (ks / SA) & 1, abort_flag) &&
+               mbar_wait(bar_full_b(sb), (ks / SB) & 1, abort_flag);
           if (!ok) break;
+          if (PAIR && rank == 1) {
+            mbar_arrive_remote(bar_pair_full(s), 0);
+            continue;
+          }
+          if (PAIR && !(ok = mbar_wait_cluster(bar_pair_full(s), (ks / SA) & 1, abort_flag))) break;
           tc_fence_after();
           const uint32_t a0 = sbase + kSmemA + s * kATileBytes;
-          const uint32_t b0 = sbase + kSmemB + sb * kBTileBytes;
+          const uint32_t b0 = sbase + LY::SmemB + sb * LY::BTile;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
 #pragma unroll
             for (int kk = 0; kk < kGemmBK / 16; ++kk) {
-              umma_f16kind(tmem + h * 256, umma_desc_sw128(a0 + h * (kATileBytes / 2) + kk * 32),
-                           umma_desc_sw128(b0 + kk * 32), GROUPED ? kIdescF16 : kIdescBf16,
-                           (ks | kk) != 0);
+              if (PAIR)
+                umma2_f16kind(tmem + h * 256, umma_desc_sw128(a0 + h * (kATileBytes / 2) + kk * 32),
+                              umma_desc_sw128(b0 + kk * 32), kIdescBf16Pair, (ks | kk) != 0);
+              else
+                umma_f16kind(tmem + h * 256, umma_desc_sw128(a0 + h * (kATileBytes / 2) + kk * 32),
+                             umma_desc_sw128(b0 + kk * 32), GROUPED ? kIdescF16 : kIdescBf16,
+                             (ks | kk) != 0);
             }
           }
-          umma_commit(bar_empty_aw(s));
-          umma_commit(bar_empty_b(sb));
+          if (PAIR) {
+            umma2_commit_both(bar_empty_aw(s));
+            umma2_commit_both(bar_empty_b(sb));
+          } else {
+            umma_commit(bar_empty_aw(s));
+            umma_commit(bar_empty_b(sb));
+          }
         }
-        if (ok) umma_commit(bar_tmem_full);
+        if (ok && PAIR && rank == 0) umma2_commit_both(bar_tmem_full);
+        if (ok && !PAIR) umma_commit(bar_tmem_full);
       }
     } else if (warp < 2 + kDqWarps) {
       // ---------------- dequantisation, then epilogue ----------------
-      const int r = (warp - 2) * 32 + lane;  // weight row of the B tile (0..255)
+      // weight row of the B tile (0..255); PAIR: row 0..127 of the CTA's half, and the
+      // 32-weight half of the K step (warps 2-5: the first, 6-9: the second)
+      const int r = PAIR ? ((warp - 2) & 3) * 32 + lane : (warp - 2) * 32 + lane;
+      const int hh = (warp - 2) >> 2;
       bool ok = true;
       for (int ks = 0; ks < (BF16W ? 0 : nks); ++ks) {  // (bf16 weights: loaded by TMA)
-        const int s = ks % kStagesAW, sb = ks % kStagesB, ub = ks / kStagesB;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_full_aw(s), (ks / kStagesAW) & 1, abort_flag))) {
+        const int s = ks % SA, sb = ks % SB, ub = ks / SB;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_full_aw(s), (ks / SA) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -503,13 +656,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
           break;
         }
         {
-          const uint8_t* wr = smem + kSmemW + s * kWRawBytes;
+          const uint8_t* wr = smem + LY::SmemW + s * LY::WRaw;
           const uint4 hdr = *reinterpret_cast<const uint4*>(wr + r * 16);
-          const uint4 qa = *reinterpret_cast<const uint4*>(wr + kWRawPart + r * 16);
-          const uint4 qb = *reinterpret_cast<const uint4*>(wr + 2 * kWRawPart + r * 16);
+          const uint4 qa = *reinterpret_cast<const uint4*>(wr + LY::WPart + r * 16);
+          const uint4 qb = *reinterpret_cast<const uint4*>(wr + 2 * LY::WPart + r * 16);
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_empty_aw(s));
-          dequant_row_step<GROUPED>(smem + kSmemB + sb * kBTileBytes, r, ks & 3, hdr, qa, qb);
+          uint8_t* bt = smem + LY::SmemB + sb * LY::BTile;
+          if (!PAIR)
+            dequant_row_step<GROUPED>(bt, r, ks & 3, hdr, qa, qb);
+          else if (hh == 0)
+            dequant_row_half<GROUPED, 0>(bt, r, ks & 3, hdr, qa, qb);
+          else
+            dequant_row_half<GROUPED, 1>(bt, r, ks & 3, hdr, qa, qb);
         }
         fence_async_smem();
         __syncwarp();
@@ -519,7 +678,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       if (ok && __all_sync(0xffffffffu, mbar_wait(bar_tmem_full, 0, abort_flag))) {
         tc_fence_after();
         const int q = warp & 3, hm = (warp - 2) >> 2;
-        const int mbase = m0 + hm * 128 + q * 32;  // first of this warp's 32 token rows
+        // first of this warp's 32 token rows (PAIR: MMA hm's rows of this CTA)
+        const int mbase = PAIR ? m0 + hm * 256 + rank * 128 + q * 32 : m0 + hm * 128 + q * 32;
         const int limit = GROUPED ? count : p.M;
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(hm * 256);
         // Coalesced stores through a per-warp staging tile (the activation stages are
@@ -605,7 +765,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       uint32_t amax = 0;  // largest |bf16| bit pattern seen, per 16-bit half
       if (nks > 0) load(0);
       for (int ks = 0; ks < nks; ++ks) {
-        const int s = ks % kStagesAW, u = ks / kStagesAW;
+        const int s = ks % SA, u = ks / SA;
         if (u >= 1 &&
             !__all_sync(0xffffffffu, mbar_wait(bar_empty_aw(s), (u - 1) & 1, abort_flag)))
           break;
@@ -634,11 +794,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 
   // ---- teardown ----
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_barrier();  // neither CTA leaves while the pair's MMAs or arrivals may touch it
+  else
+    __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    if (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
   }
 }
 
@@ -683,26 +849,49 @@ inline bool make_tmap_w(CUtensorMap* m, const void* base, int64_t rows, int64_t 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GROUPED, bool SWIGLU, bool BF16W = false>
+// PAIR: clusters of two CTAs, m_tiles counting 512-token tiles.
+template <bool GROUPED, bool SWIGLU, bool BF16W = false, bool PAIR = false>
 inline q4k_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
                                 cudaStream_t s) {
-  auto* k = gemm_tc_kernel<GROUPED, SWIGLU, BF16W>;
+  auto* k = gemm_tc_kernel<GROUPED, SWIGLU, BF16W, PAIR>;
+  constexpr size_t smem = GemmLayout<PAIR>::Launch;
   static std::atomic<int> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return Q4K_ERR_CUDA;
   if (!attr_set[dev].load()) {
     if (cudaFuncSetAttribute(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kGemmSmemLaunch) != cudaSuccess)
+                             (int)smem) != cudaSuccess)
       return Q4K_ERR_LAUNCH;
     attr_set[dev].store(1);
   }
-  const dim3 grid((unsigned)(p.n_tiles * p.m_tiles));
   const dim3 block(32 * (2 + kDqWarps + (GROUPED ? kGatherWarps : 0)));
-  k<<<grid, block, kGemmSmemLaunch, s>>>(tx, tw, p);
-  const cudaError_t e = cudaGetLastError();
+  if (!PAIR) {
+    const dim3 grid((unsigned)(p.n_tiles * p.m_tiles));
+    k<<<grid, block, smem, s>>>(tx, tw, p);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? Q4K_OK : Q4K_ERR_LAUNCH;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * p.n_tiles * p.m_tiles), 1, 1);
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, tx, tw, p);
+  if (e != cudaSuccess) cudaGetLastError();
   return e == cudaSuccess ? Q4K_OK : Q4K_ERR_LAUNCH;
 }
+
+// More than 256 tokens: CTA pairs on 512-token tiles (tcgen05.mma.cta_group::2);
+// up to 256: one CTA per 256-token tile.
+constexpr int kGemmPairMinM = 257;
 
 inline q4k_status launch_gemm_tc(GemmParams p, cudaStream_t s) {
   CUtensorMap tx, tw;
@@ -710,17 +899,21 @@ inline q4k_status launch_gemm_tc(GemmParams p, cudaStream_t s) {
   if (!make_tmap_x(&tx, p.X, p.M, p.K) || !make_tmap_w(&tw, p.W, p.N, row_bytes))
     return Q4K_ERR_CUDA;
   p.n_tiles = p.N / kGemmBN;
+  if (p.M >= kGemmPairMinM) {
+    p.m_tiles = (p.M + 2 * kGemmBM - 1) / (2 * kGemmBM);
+    return launch_gemm_t<false, false, false, true>(tx, tw, p, s);
+  }
   p.m_tiles = (p.M + kGemmBM - 1) / kGemmBM;
   return launch_gemm_t<false, false>(tx, tw, p, s);
 }
 
-// bf16 weights [N][K], box 64 x 256 (one B stage), 128-byte swizzle.
-inline bool make_tmap_wb(CUtensorMap* m, const void* base, int64_t rows, int K) {
+// bf16 weights [N][K], box 64 x box_rows (one B stage), 128-byte swizzle.
+inline bool make_tmap_wb(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  cuuint32_t box[2] = {64, 256};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -731,8 +924,14 @@ inline bool make_tmap_wb(CUtensorMap* m, const void* base, int64_t rows, int K) 
 // fused kernel's tiles and MMA order.
 inline q4k_status launch_gemm_tc_bf16w(GemmParams p, cudaStream_t s) {
   CUtensorMap tx, tw;
-  if (!make_tmap_x(&tx, p.X, p.M, p.K) || !make_tmap_wb(&tw, p.W, p.N, p.K)) return Q4K_ERR_CUDA;
+  const bool pair = p.M >= kGemmPairMinM;
+  if (!make_tmap_x(&tx, p.X, p.M, p.K) || !make_tmap_wb(&tw, p.W, p.N, p.K, pair ? kGemmBN / 2 : kGemmBN))
+    return Q4K_ERR_CUDA;
   p.n_tiles = p.N / kGemmBN;
+  if (pair) {
+    p.m_tiles = (p.M + 2 * kGemmBM - 1) / (2 * kGemmBM);
+    return launch_gemm_t<false, false, true, true>(tx, tw, p, s);
+  }
   p.m_tiles = (p.M + kGemmBM - 1) / kGemmBM;
   return launch_gemm_t<false, false, true>(tx, tw, p, s);
 }

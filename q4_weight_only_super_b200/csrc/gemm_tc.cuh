@@ -18,6 +18,14 @@
 //   warps 10-13 (grouped variant) load activation rows by index (gathered or
 //               contiguous), convert bf16 -> fp16 in registers and store them
 //               in the same swizzled layout.
+// Dense GEMM above 256 tokens (PAIR): a cluster of two CTAs on two SMs computes a
+// 512-token x 256-weight-row tile with tcgen05.mma.cta_group::2 (M=256, N=256,
+// issued by the even CTA): each CTA holds 256 token rows of A (128 per MMA, one
+// MMA per 256-token half) and dequantises 128 of the 256 weight rows -- half the
+// per-SM dequantisation -- into 4-deep rings; its TMEM receives its own token rows
+// x all 256 weight rows. The odd CTA's MMA lane relays "stage ready" to the even
+// CTA by one remote mbarrier arrive per K step; the MMA completions are committed
+// to the barriers of both CTAs (multicast commit).
 // The dense GEMM multiplies bf16 x bf16. The grouped (mixture-of-experts) GEMM
 // multiplies fp16 x fp16: its activations can be heavy-tailed (SwiGLU outputs),
 // where bf16-rounded weights (unit roundoff 2^-8) would not keep the

@@ -531,9 +531,9 @@ def summarize(tm, W, peaks):
 # same kernel code (dram__bytes_read.sum + dram__bytes_write.sum); the captures
 # and their commands are summarised in profiles/. None where not captured.
 TRAFFIC = {
-    "gemv:gate_up:M1": 103.005952e6 + 4.032256e6,    # profiles/gemv_gate_up_34816x5120_M1.md
-    "gemm:M512": 55.41e6 + 3.38e6,                  # profiles/gemm_prefill_17408x5120.md
-    "gemm:M4096": 410.91e6 + 243.23e6,              # profiles/gemm_prefill_17408x5120.md
+    "gemv:gate_up:M1": 100.35e6 + 4.54e6,           # profiles/gemv_sk_gate_up_34816x5120_M1.md
+    "gemm:M512": 55.41e6 + 3.43e6,                  # profiles/gemm_prefill_17408x5120.md
+    "gemm:M4096": 368.32e6 + 237.22e6,              # profiles/gemm_prefill_17408x5120.md
 }
 
 

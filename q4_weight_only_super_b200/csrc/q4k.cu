@@ -318,9 +318,12 @@ int sm_count() {
   return v;
 }
 
-// Shared memory one grouped-GEMV CTA may take: two CTAs per SM with one super-block
-// a warp (at most 20 warps of 96 registers: both fit), one with two.
-size_t skg_budget(int nkb) { return nkb > 10 ? kSkSmemBudget : kGemvTwoPerSm; }
+// Shared memory one grouped-GEMV CTA may take: one CTA per SM with two super-blocks a
+// warp; with one, two CTAs per SM, or four when K has at most four super-blocks (at
+// most six warps a CTA: four fit the registers too).
+size_t skg_budget(int nkb) {
+  return nkb > 10 ? kSkSmemBudget : (nkb <= 4 ? 233472 / 4 - 1024 : kGemvTwoPerSm);
+}
 
 // Every CTA resident at once: the kernel deals the units over the whole grid.
 template <int KPW, bool SWIGLU>

@@ -532,8 +532,13 @@ def summarize(tm, W, peaks):
 # and their commands are summarised in profiles/. None where not captured.
 TRAFFIC = {
     "gemv:gate_up:M1": 100.35e6 + 4.54e6,           # profiles/gemv_sk_gate_up_34816x5120_M1.md
+    "gemv:down:M1": 50.23e6 + 1.3e3,                # profiles/gemv_sk_down_5120x17408_M1.md
+    "gemv:gate_up:M32": 103.055872e6 + 3.15008e6,   # profiles/dram_traffic_one_pass.md
+    "gemv:down:M32": 51.427328e6 + 30.464e3,        # profiles/dram_traffic_one_pass.md
     "gemm:M512": 55.41e6 + 3.43e6,                  # profiles/gemm_prefill_17408x5120.md
     "gemm:M4096": 368.32e6 + 237.22e6,              # profiles/gemm_prefill_17408x5120.md
+    "moe_pre:M4096:gate_up": 261.251328e6 + 38.374912e6,  # profiles/dram_traffic_one_pass.md
+    "moe_pre:M4096:down": 163.623168e6 + 208.747264e6,    # profiles/dram_traffic_one_pass.md
 }
 
 

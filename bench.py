@@ -275,9 +275,11 @@ def moe_buffers(torch, q, d, M, dims, topk=8):
 
 
 def moe_layer_calls(q, d, M, dims, topk=8, stage=None):
-    """Issue one MoE layer on the current stream: routing + permutation, gate_up
-    grouped GEMV with SwiGLU, down grouped GEMV, combine. `stage(name, fn)` wraps
-    each call (timing); None runs them plainly (also under CUDA-graph capture)."""
+    """Issue one MoE layer on the current stream: routing + permutation and the gate_up
+    grouped GEMV with SwiGLU (up to 8 tokens in one launch, moe_route_gate_up: its eight
+    routing warps then take one token each; beyond that the one-CTA routing kernel routes
+    the tokens in parallel, then the grouped GEMV), the down grouped GEMV, the combine. `stage(name, fn)` wraps each call (timing); None
+    runs them plainly (also under CUDA-graph capture)."""
     import torch
     E, H, F = dims
     rows = M * topk
@@ -285,10 +287,14 @@ def moe_layer_calls(q, d, M, dims, topk=8, stage=None):
     logits, X = d["logits"][:M], d["X"][:M]
     ws = d.get("ws") if M <= 32 else None
     stage = stage or (lambda k, fn: fn())
-    r = stage("route", lambda: q.moe_route_permute(logits, topk, out=b["route"], ws=b["route_ws"]))
-    h = stage("gate_up", lambda: q.moe_q4k_grouped(d["W_gate_up"], E, 2 * F, H, X, r["expert_offsets"],
-                                                  rows, M, q.ACT_SWIGLU, row_gather=r["row_token"],
-                                                  out=b["h"], ws=ws))
+    if M <= 8:
+        r, h = stage("route_gate_up", lambda: q.moe_route_gate_up(logits, topk, d["W_gate_up"], 2 * F, H, X,
+                                                                  out=b["route"], h=b["h"]))
+    else:
+        r = stage("route", lambda: q.moe_route_permute(logits, topk, out=b["route"], ws=b["route_ws"]))
+        h = stage("gate_up", lambda: q.moe_q4k_grouped(d["W_gate_up"], E, 2 * F, H, X, r["expert_offsets"],
+                                                      rows, M, q.ACT_SWIGLU, row_gather=r["row_token"],
+                                                      out=b["h"], ws=ws))
     o = stage("down", lambda: q.moe_q4k_grouped(d["W_down"], E, H, F, h, r["expert_offsets"], rows, M,
                                                q.ACT_NONE, out=b["o"], ws=ws))
     y = stage("combine", lambda: q.moe_combine(o, r["inv_perm"], r["topk_w"], M, topk, H, Y=b["y"]))
@@ -370,12 +376,12 @@ def run_step(q, tm, W):
     for staged in (True, False):
         for M in (1, 8, 32):
             moe_layer_gpu(q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"], staged=staged)
-            launches += 4  # routing+permutation, grouped gate_up GEMV (+SwiGLU), grouped down GEMV, combine
+            launches += 3 if M <= 8 else 4  # routing (+ grouped gate_up GEMV with SwiGLU), down GEMV, combine
         moe_layer_gpu(q, tm, "moe_pre:M4096", W["moe_pre"], 4096, W["moe_dims"], staged=staged)
         launches += 5  # routing, permutation, 2 grouped GEMMs, combine
     for M in (1, 8, 32):
         moe_layer_graph(torch, q, tm, f"moe_dec:M{M}", W["moe_dec"], M, W["moe_dims"])
-        launches += 4
+        launches += 3 if M <= 8 else 4
     return launches
 
 
@@ -482,10 +488,11 @@ def summarize(tm, W, peaks):
         comp[f"gemm_M{M}_TFLOPS"] = round(2.0 * M * N * K / t / 1e12, 1)
         comp[f"gemm_M{M}_us"] = round(t * 1e6, 1)
     for key, M in (("moe_dec", 1), ("moe_dec", 8), ("moe_dec", 32), ("moe_pre", 4096)):
-        parts = [T[f"{key}:M{M}:{s}"] for s in ("route", "gate_up", "down", "combine")]
+        names = ("route_gate_up", "down", "combine") if M <= 8 else ("route", "gate_up", "down", "combine")
+        parts = [T[f"{key}:M{M}:{s}"] for s in names]
         comp[f"{key}_M{M}_tokens_per_s"] = round(M / T[f"{key}:M{M}:layer"], 1)
         comp[f"{key}_M{M}_layer_us"] = round(T[f"{key}:M{M}:layer"] * 1e6, 2)
-        comp[f"{key}_M{M}_stage_us"] = {s: round(x * 1e6, 2) for s, x in zip(("route", "gate_up", "down", "combine"), parts)}
+        comp[f"{key}_M{M}_stage_us"] = {s: round(x * 1e6, 2) for s, x in zip(names, parts)}
         if f"{key}:M{M}:graph" in T:
             comp[f"{key}_M{M}_graph_us"] = round(T[f"{key}:M{M}:graph"] * 1e6, 2)
             comp[f"{key}_M{M}_graph_tokens_per_s"] = round(M / T[f"{key}:M{M}:graph"], 1)

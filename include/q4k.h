@@ -272,6 +272,26 @@ q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uin
                            int rows, int max_rows_hint, int act, void* out,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* Routing and the grouped gate_up GEMV of the decode MoE layer in one launch
+ * (hipEngine 0.3.0 README, "Core principles": the route composite fused with the
+ * expert matmul that follows it). Equivalent to
+ *   moe_route_permute(logits, M, E, topk, topk_ids, topk_w, expert_offsets, perm,
+ *                     inv_perm, row_token, ...)  and then
+ *   moe_q4k_grouped(W_gate_up, E, N, K, X, row_gather = row_token, expert_offsets,
+ *                   M*topk, M, Q4K_ACT_SWIGLU, h, ...),
+ * bit for bit (every CTA of the GEMV routes all tokens with the same code and order
+ * as the routing kernel; one writes the routing outputs).
+ *   logits fp32 [M][E]; X bf16 [M][K]; W_gate_up Q4_K [E][N][K/256] (gate rows
+ *   first, then up rows); h bf16 [M*topk][N/2]; the routing outputs as in
+ *   moe_route_permute (all device, caller-owned, written).
+ * Supported: 1 <= M <= 32, E <= 256, topk <= 16, 1536 <= K <= 5120 (at least six
+ * consumer warps to host the routing warps), N % 32 == 0; anything else returns
+ * Q4K_ERR_UNSUPPORTED (use the two calls). No workspace.
+ * M == 0 only clears expert_offsets. Device errors as the two calls. */
+q4k_status moe_route_gate_up(const float* logits, int M, int E, int topk, int32_t* topk_ids, float* topk_w,
+                             int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm, int32_t* row_token,
+                             const void* W_gate_up, int N, int K, const uint16_t* X, void* h, void* stream);
+
 /* Weighted combine of the expert outputs back into token order
  * (hipEngine 0.3.0 README, "Core principles": the gate_combine part of the
  * fused gate_combine_residual composite).

@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "Q4KError", "lib", "q4k_dequant", "q4k_gemv", "q4k_gemv_q8", "q5k_gemv", "q80_gemv", "q6k_gemv", "q4k_repack", "q4k_gemv_repacked", "q4k_gemm", "bf16w_gemm",
     "moe_route_permute",
-    "moe_route_permute_noalloc", "moe_route_permute_hidden",
+    "moe_route_permute_noalloc", "moe_route_permute_hidden", "moe_route_gate_up",
     "moe_q4k_grouped", "moe_combine", "moe_combine_residual", "q4k_workspace_bytes", "q4k_last_device_status",
     "q4k_test_wait_fault",
     "ACT_NONE", "ACT_SWIGLU", "OP_GEMM", "OP_ROUTE", "OP_GROUPED", "OP_GEMV", "EXPORTS",
@@ -45,6 +45,7 @@ EXPORTS = {
     "moe_route_permute_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
     "moe_route_permute_hidden": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_q4k_grouped": (_i, [_p, _i, _i, _i, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
+    "moe_route_gate_up": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _i, _i, _p, _p, _p]),
     "moe_combine": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_combine_residual": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "q4k_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -308,6 +309,30 @@ def moe_q4k_grouped(W_experts, E: int, N: int, K: int, A, expert_offsets, rows: 
                                0 if ws is None else ws.numel(), _stream(stream))
     _check("moe_q4k_grouped", st)
     return out
+
+
+def moe_route_gate_up(logits, topk: int, W_gate_up, N: int, K: int, X, out=None, h=None, stream=None):
+    """Routing + permutation and the grouped gate_up SwiGLU GEMV in one launch (decode,
+    M <= 32; see include/q4k.h). Returns (routing dict as moe_route_permute's, h)."""
+    M, E = logits.shape
+    dev = logits.device
+    if out is None:
+        out = dict(
+            topk_ids=torch.empty(M, topk, dtype=torch.int32, device=dev),
+            topk_w=torch.empty(M, topk, dtype=torch.float32, device=dev),
+            expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            perm=torch.empty(M * topk, dtype=torch.int32, device=dev),
+            inv_perm=torch.empty(M * topk, dtype=torch.int32, device=dev),
+            row_token=torch.empty(M * topk, dtype=torch.int32, device=dev),
+        )
+    if h is None:
+        h = torch.empty(M * topk, N // 2, dtype=torch.bfloat16, device=dev)
+    st = lib().moe_route_gate_up(_ptr(logits), M, E, topk, _ptr(out["topk_ids"]), _ptr(out["topk_w"]),
+                                 _ptr(out["expert_offsets"]), _ptr(out["perm"]), _ptr(out["inv_perm"]),
+                                 _ptr(out["row_token"]), _ptr(W_gate_up), N, K, _ptr(_bits16(X)), _ptr(h),
+                                 _stream(stream))
+    _check("moe_route_gate_up", st)
+    return out, h
 
 
 def moe_combine(O, inv_perm, topk_w, M: int, topk: int, H: int, Y=None, stream=None):

@@ -28,6 +28,7 @@
 //    sequence inside [0, rows] latch Q4K_ERR_DEVICE_BOUNDS and nothing is computed.
 #pragma once
 #include "gemv_sk.cuh"
+#include "moe.cuh"  // route_tile, route_scan_place_one (the routing prologue)
 
 namespace q4k {
 
@@ -41,21 +42,42 @@ struct SkgParams {
   int CW;                  // consumer warps = ceil(nkb / KPW)
   int pitch;               // shared-memory bytes per staged row (>= nkb * 144)
   int stages;              // weight ring depth
+  // routing prologue (PL > 0): top-k routing and permutation of the M <= 32 tokens
+  // in every CTA; CTA 0 writes the routing outputs (offsets and gather come from it)
+  const float* logits;     // fp32 [M][E]
+  int M, topk;
+  int32_t* topk_ids;       // [M][topk]
+  float* topk_w;           // [M][topk]
+  int32_t* offsets_out;    // [E+1]
+  int32_t* perm;           // [rows]
+  int32_t* inv_perm;       // [rows]
+  int32_t* row_token;      // [rows]
 };
 
+// Warps that route in the routing prologue (route_tile deals the <= 32 tokens to them).
+constexpr int kSkgRouteWarps = 8;
+
 // Shared memory: ring [stages][16][pitch], partials [2][CW][8 tokens x 20], the
-// expert offsets [E+1] and unit starts [E+2] (each padded to 16 B), barriers, abort flag.
+// expert offsets [E+1] and unit starts [E+2] (each padded to 16 B), with the routing
+// prologue its arrays (per-expert totals, starts and token masks [E], warp sums [32],
+// the tile's expert ids and the sorted rows' tokens [32 x 16] each), barriers, abort flag.
 struct SkgSmem {
   static __host__ __device__ size_t red_off(int pitch, int stages) { return (size_t)stages * kSkRows * pitch; }
   static __host__ __device__ size_t tab_off(int pitch, int stages, int CW) {
     return red_off(pitch, stages) + (size_t)kSkRedSlots * CW * kSkPartial * 4;
   }
   static __host__ __device__ size_t tab_bytes(int E) { return ((size_t)(E + 2) * 4 + 15) & ~(size_t)15; }
-  static __host__ __device__ size_t bar_off(int pitch, int stages, int CW, int E) {
+  static __host__ __device__ size_t route_off(int pitch, int stages, int CW, int E) {
     return tab_off(pitch, stages, CW) + 2 * tab_bytes(E);
   }
-  static __host__ __device__ size_t total(int pitch, int stages, int CW, int E) {
-    return bar_off(pitch, stages, CW, E) + 8 * (2 * stages + 2 * kSkRedSlots) + 16;
+  static __host__ __device__ size_t route_bytes(int E) {
+    return (size_t)3 * ((E * 4 + 15) & ~15) + 128 + (size_t)2 * kRouteTokPerCta * kMaxTopk * 4;
+  }
+  static __host__ __device__ size_t bar_off(int pitch, int stages, int CW, int E, bool route) {
+    return route_off(pitch, stages, CW, E) + (route ? route_bytes(E) : 0);
+  }
+  static __host__ __device__ size_t total(int pitch, int stages, int CW, int E, bool route = false) {
+    return bar_off(pitch, stages, CW, E, route) + 8 * (2 * stages + 2 * kSkRedSlots) + 16;
   }
 };
 
@@ -106,9 +128,13 @@ __device__ __forceinline__ void skg_next(SkgPos& s, const int* ustart, const int
   s.nr = min(8, s.oe - s.r0);
 }
 
-template <int KPW, bool SWIGLU>
+// PL > 0: the routing prologue (route_tile with PL logits per lane, E <= 32 * PL),
+// run by every CTA with the same code and order as the one-CTA routing kernel, so its
+// results are bit-identical to moe_route_permute's.
+template <int KPW, bool SWIGLU, int PL = 0>
 __global__ void __launch_bounds__(SkMax<KPW>::threads, 1) gemv_skg_kernel(const SkgParams p) {
   using L = SkgSmem;
+  constexpr bool ROUTE = PL > 0;
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -122,9 +148,18 @@ __global__ void __launch_bounds__(SkMax<KPW>::threads, 1) gemv_skg_kernel(const 
   float* red = reinterpret_cast<float*>(smem + L::red_off(p.pitch, S));
   int* eoff = reinterpret_cast<int*>(smem + L::tab_off(p.pitch, S, CW));  // expert offsets [E+1]
   int* ustart = eoff + L::tab_bytes(E) / 4;  // unit starts [E+1], then the unit total
-  const uint32_t bar0 = smem_u32(smem + L::bar_off(p.pitch, S, CW, E));
+  const uint32_t bar0 = smem_u32(smem + L::bar_off(p.pitch, S, CW, E, ROUTE));
   volatile int* abort_flag =
-      reinterpret_cast<volatile int*>(smem + L::bar_off(p.pitch, S, CW, E) + 8 * (2 * S + 2 * kSkRedSlots));
+      reinterpret_cast<volatile int*>(smem + L::bar_off(p.pitch, S, CW, E, ROUTE) + 8 * (2 * S + 2 * kSkRedSlots));
+  // routing prologue arrays (ROUTE)
+  uint8_t* rbase = smem + L::route_off(p.pitch, S, CW, E);
+  const size_t ea = (size_t)((E * 4 + 15) & ~15);
+  int* r_total = reinterpret_cast<int*>(rbase);
+  int* r_start = reinterpret_cast<int*>(rbase + ea);
+  unsigned* r_tmask = reinterpret_cast<unsigned*>(rbase + 2 * ea);
+  int* r_wsum = reinterpret_cast<int*>(rbase + 3 * ea);
+  int* r_sids = reinterpret_cast<int*>(rbase + 3 * ea + 128);
+  int* r_rtok = r_sids + kRouteTokPerCta * kMaxTopk;  // token of each sorted row
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (S + s); };
   auto redfull = [&](int r) { return bar0 + 8u * (2 * S + r); };
@@ -145,14 +180,33 @@ __global__ void __launch_bounds__(SkMax<KPW>::threads, 1) gemv_skg_kernel(const 
   // Dependents may launch now; each waits (griddepcontrol.wait) for this grid to
   // complete before it touches anything this grid reads or writes.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // the offsets, the gather indices and A come from the previous kernels
+  // the offsets, the gather indices (or the logits) and A come from the previous kernels
   asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  if (ROUTE) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      r_total[e] = 0;
+      r_tmask[e] = 0u;
+    }
+    __syncthreads();
+    const bool out = blockIdx.x == 0;  // CTA 0 writes the routing outputs
+    if (warp < kSkgRouteWarps)
+      route_tile<(ROUTE ? PL : 1), kSkgRouteWarps>(p.logits, p.M, E, p.topk, out ? p.topk_ids : nullptr,
+                                                   out ? p.topk_w : nullptr, r_total, r_sids, r_tmask, 0);
+    __syncthreads();
+    route_scan_place_one(r_total, r_start, r_wsum, E, p.M, p.topk, r_sids, r_tmask, out ? p.offsets_out : nullptr,
+                         out ? p.perm : nullptr, out ? p.inv_perm : nullptr, out ? p.row_token : nullptr, eoff,
+                         r_rtok);
+    __syncthreads();
+  }
 
   if (warp == 0) {
     // unit starts: ustart[e] = U * (token groups of experts 0..e-1); the checks
     // make every later index lie inside [0, rows)
+    if (!ROUTE) {
 #pragma unroll 4
-    for (int e = lane; e <= E; e += 32) eoff[e] = __ldg(p.offsets + e);  // all loads in flight at once
+      for (int e = lane; e <= E; e += 32) eoff[e] = __ldg(p.offsets + e);  // all loads in flight at once
+    }
     __syncwarp();
     bool bad = false;
     for (int e = lane; e < E; e += 32) {  // token groups of expert e, in ustart[e + 1] for now
@@ -287,7 +341,8 @@ __global__ void __launch_bounds__(SkMax<KPW>::threads, 1) gemv_skg_kernel(const 
       if (pos.r0 != cur) {  // a new token group: its fragments, from A rows (gathered)
         cur = pos.r0;
         const bool mine = g < pos.nr;
-        const int64_t arow = mine ? (p.gather ? __ldg(p.gather + pos.r0 + g) : pos.r0 + g) : 0;
+        const int64_t arow =
+            mine ? (ROUTE ? r_rtok[pos.r0 + g] : (p.gather ? __ldg(p.gather + pos.r0 + g) : pos.r0 + g)) : 0;
 #pragma unroll
         for (int kk = 0; kk < KPW; ++kk)
           sk_load_act(act[kk], p.A + arow * p.K + (int64_t)(KPW * w + kk) * QK + 8 * t, has[kk] && mine, t);
@@ -332,16 +387,16 @@ struct SkgCfg {
   size_t smem;
 };
 
-inline bool skg_shape(int nkb, int E, size_t smem_budget, SkgCfg* c) {
+inline bool skg_shape(int nkb, int E, size_t smem_budget, SkgCfg* c, bool route = false) {
   c->kpw = nkb > 10 ? 2 : 1;
   const int KU = c->kpw == 2 ? SkMax<2>::KU : SkMax<1>::KU;
   if (nkb > KU) return false;
   c->CW = (nkb + c->kpw - 1) / c->kpw;
   c->pitch = sk_pitch(nkb);
   int st = 8;
-  while (st > 2 && SkgSmem::total(c->pitch, st, c->CW, E) > smem_budget) --st;
+  while (st > 2 && SkgSmem::total(c->pitch, st, c->CW, E, route) > smem_budget) --st;
   c->stages = st;
-  c->smem = SkgSmem::total(c->pitch, st, c->CW, E);
+  c->smem = SkgSmem::total(c->pitch, st, c->CW, E, route);
   return c->smem <= smem_budget;
 }
 

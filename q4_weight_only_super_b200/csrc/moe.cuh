@@ -90,8 +90,8 @@ __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int
 #pragma unroll
       for (int k = 0; k < kMaxTopk; ++k)
         if (k == lane) { num = expf(sel_v[k] - sel_v[0]); id = sel_i[k]; }
-      ids[(int64_t)tok * topk + lane] = id;
-      wts[(int64_t)tok * topk + lane] = num / den;
+      if (ids) ids[(int64_t)tok * topk + lane] = id;  // (null: not written)
+      if (wts) wts[(int64_t)tok * topk + lane] = num / den;
       if (sids) sids[tl * topk + lane] = id;
       if (tmask) atomicOr(&tmask[id], 1u << tl);
       atomicAdd(&hist[id], 1);
@@ -214,6 +214,70 @@ permute_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ coun
                  min(M, (b + 1) * kRouteTokPerCta) * topk, topk, perm, inv_perm, row_token);
 }
 
+// After route_tile over a CTA's single tile (all threads of the CTA call this): the
+// exclusive scan of the per-expert totals into the expert offsets and each expert's
+// start, then the stable place of every (token, slot) pair f = t*topk + j: a token
+// selects an expert at most once, so f's rank among expert e's pairs is the number of
+// earlier tokens that selected e (the popcount of e's token mask below bit t). Each of
+// the outputs may be null (not written): global (g_*) and shared-memory copies (s_offsets
+// [E+1], s_row_token [M*topk]).
+__device__ __forceinline__ void route_scan_place_one(const int* total, int* start, int* warp_sums, int E, int M,
+                                                     int topk, const int* sids, const unsigned* tmask,
+                                                     int32_t* __restrict__ g_offsets, int32_t* __restrict__ g_perm,
+                                                     int32_t* __restrict__ g_inv_perm,
+                                                     int32_t* __restrict__ g_row_token, int* s_offsets,
+                                                     int* s_row_token) {
+  {
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = threadIdx.x * per;
+    int run = 0;
+    for (int e = e0; e < e0 + per && e < E; ++e) run += total[e];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = run;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int nw = blockDim.x / 32;
+      int ws = lane < nw ? warp_sums[lane] : 0;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, ws, off);
+        if (lane >= off) ws += o;
+      }
+      if (lane < nw) warp_sums[lane] = ws;
+    }
+    __syncthreads();
+    int excl = incl - run + (warp > 0 ? warp_sums[warp - 1] : 0);
+    for (int e = e0; e < e0 + per && e < E; ++e) {
+      if (g_offsets) g_offsets[e] = excl;
+      if (s_offsets) s_offsets[e] = excl;
+      start[e] = excl;
+      excl += total[e];
+    }
+    if (threadIdx.x == blockDim.x - 1) {
+      if (g_offsets) g_offsets[E] = excl;
+      if (s_offsets) s_offsets[E] = excl;
+    }
+  }
+  __syncthreads();
+  for (int f = threadIdx.x; f < M * topk; f += blockDim.x) {
+    const int t = f / topk;
+    const int e = sids[f];
+    if (e < 0 || e >= E) {
+      latch_status(Q4K_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    const int pos = start[e] + __popc(tmask[e] & ((1u << t) - 1u));
+    if (g_perm) g_perm[pos] = f;
+    if (g_inv_perm) g_inv_perm[f] = pos;
+    if (g_row_token) g_row_token[pos] = t;
+    if (s_row_token) s_row_token[pos] = t;
+  }
+}
+
 // Routing and permutation of at most kRouteTokPerCta tokens in one CTA (one
 // launch instead of two; the histogram, the ids and the per-expert token masks
 // stay in shared memory). A token selects an expert at most once, so the rank
@@ -243,51 +307,8 @@ route_permute_one_kernel(const float* __restrict__ logits, int M, int E, int top
   __syncthreads();
   route_tile<PL, kRouteOneWarps>(logits, M, E, topk, ids, wts, total, sids, tmask, 0);
   __syncthreads();
-  // exclusive scan of the per-expert totals -> expert_offsets and start[e]
-  {
-    const int per = (E + blockDim.x - 1) / blockDim.x;
-    const int e0 = threadIdx.x * per;
-    int run = 0;
-    for (int e = e0; e < e0 + per && e < E; ++e) run += total[e];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = run;
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int nw = blockDim.x / 32;
-      int ws = lane < nw ? warp_sums[lane] : 0;
-      for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, ws, off);
-        if (lane >= off) ws += o;
-      }
-      if (lane < nw) warp_sums[lane] = ws;
-    }
-    __syncthreads();
-    int excl = incl - run + (warp > 0 ? warp_sums[warp - 1] : 0);
-    for (int e = e0; e < e0 + per && e < E; ++e) {
-      expert_offsets[e] = excl;
-      start[e] = excl;
-      excl += total[e];
-    }
-    if (threadIdx.x == blockDim.x - 1) expert_offsets[E] = excl;
-  }
-  __syncthreads();
-  for (int f = threadIdx.x; f < M * topk; f += blockDim.x) {
-    const int t = f / topk;
-    const int e = sids[f];
-    if (e < 0 || e >= E) {
-      latch_status(Q4K_ERR_DEVICE_BOUNDS);
-      continue;
-    }
-    const int pos = start[e] + __popc(tmask[e] & ((1u << t) - 1u));
-    perm[pos] = f;
-    inv_perm[f] = pos;
-    row_token[pos] = t;
-  }
+  route_scan_place_one(total, start, warp_sums, E, M, topk, sids, tmask, expert_offsets, perm, inv_perm,
+                       row_token, nullptr, nullptr);
 }
 
 // y[t][h] = sum_j w[t][j] * O[inv_perm[t*topk + j]][h], j in increasing order.

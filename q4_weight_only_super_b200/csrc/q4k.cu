@@ -326,9 +326,9 @@ size_t skg_budget(int nkb) {
 }
 
 // Every CTA resident at once: the kernel deals the units over the whole grid.
-template <int KPW, bool SWIGLU>
+template <int KPW, bool SWIGLU, int PL = 0>
 q4k_status launch_skg_t(const SkgCfg& c, const SkgParams& p, cudaStream_t s) {
-  auto* k = gemv_skg_kernel<KPW, SWIGLU>;
+  auto* k = gemv_skg_kernel<KPW, SWIGLU, PL>;
   static std::atomic<size_t> smem_set[kMaxDevices];
   // resident CTAs per SM for the last (threads, smem) asked on each device, packed
   // as (threads << 40) | (smem << 8) | count
@@ -364,6 +364,12 @@ q4k_status launch_skg(const SkgCfg& c, const SkgParams& p, bool swiglu, cudaStre
   if (c.kpw == 2)
     return swiglu ? launch_skg_t<2, true>(c, p, s) : launch_skg_t<2, false>(c, p, s);
   return swiglu ? launch_skg_t<1, true>(c, p, s) : launch_skg_t<1, false>(c, p, s);
+}
+
+// The grouped gate_up + SwiGLU GEMV with the routing prologue; PL = logits per lane.
+template <int PL>
+q4k_status launch_skg_route_t(const SkgCfg& c, const SkgParams& p, cudaStream_t s) {
+  return c.kpw == 2 ? launch_skg_t<2, true, PL>(c, p, s) : launch_skg_t<1, true, PL>(c, p, s);
 }
 
 // Routing kernels keep each lane's share of a logit row in registers: pick the
@@ -797,6 +803,58 @@ q4k_status moe_q4k_grouped(const void* W_experts, int E, int N, int K, const uin
   p.act = act;
   p.expert_stride = (int64_t)N * nkb * BLOCK_BYTES;
   return launch_gemm_tc_grouped(p, s);
+}
+
+q4k_status moe_route_gate_up(const float* logits, int M, int E, int topk, int32_t* topk_ids, float* topk_w,
+                             int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm, int32_t* row_token,
+                             const void* W_gate_up, int N, int K, const uint16_t* X, void* h, void* stream) {
+  if (M < 0 || E <= 0 || topk <= 0 || N <= 0 || K <= 0 || K % QK) return Q4K_ERR_SHAPE;
+  if (M > kRouteTokPerCta || E > 256 || topk > kMaxTopk || topk > E) return Q4K_ERR_UNSUPPORTED;
+  if (N % 32) return Q4K_ERR_UNSUPPORTED;
+  if (!expert_offsets) return Q4K_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    return cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), s) == cudaSuccess ? Q4K_OK
+                                                                                          : Q4K_ERR_CUDA;
+  }
+  if (!logits || !topk_ids || !topk_w || !perm || !inv_perm || !row_token || !W_gate_up || !X || !h)
+    return Q4K_ERR_NULL;
+  if (!aligned16(logits) || !aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(expert_offsets) ||
+      !aligned16(perm) || !aligned16(inv_perm) || !aligned16(row_token) || !aligned16(W_gate_up) ||
+      !aligned16(X) || !aligned16(h))
+    return Q4K_ERR_ALIGN;
+  const int nkb = K / QK;
+  const int rows = M * topk;
+  SkgCfg sc;
+  // the routing warps of the prologue must exist: CW + 2 >= kSkgRouteWarps
+  if (!skg_shape(nkb, E, skg_budget(nkb), &sc, true) || sc.CW + 2 < kSkgRouteWarps ||
+      ((int64_t)(rows + 7) / 8 + E) * (N / kSkRows) >= 0x7fffffffLL)
+    return Q4K_ERR_UNSUPPORTED;  // use moe_route_permute and moe_q4k_grouped
+  SkgParams sp = {};
+  sp.W = static_cast<const uint8_t*>(W_gate_up);
+  sp.A = X;
+  sp.out = h;
+  sp.E = E;
+  sp.N = N;
+  sp.K = K;
+  sp.nkb = nkb;
+  sp.rows = rows;
+  sp.CW = sc.CW;
+  sp.pitch = sc.pitch;
+  sp.stages = sc.stages;
+  sp.logits = logits;
+  sp.M = M;
+  sp.topk = topk;
+  sp.topk_ids = topk_ids;
+  sp.topk_w = topk_w;
+  sp.offsets_out = expert_offsets;
+  sp.perm = perm;
+  sp.inv_perm = inv_perm;
+  sp.row_token = row_token;
+  if (E <= 32) return launch_skg_route_t<1>(sc, sp, s);
+  if (E <= 64) return launch_skg_route_t<2>(sc, sp, s);
+  if (E <= 128) return launch_skg_route_t<4>(sc, sp, s);
+  return launch_skg_route_t<8>(sc, sp, s);
 }
 
 q4k_status moe_combine(const float* O, const int32_t* inv_perm, const float* topk_w, int M,

@@ -94,6 +94,15 @@ def test_argument_errors_return_before_launch(L):
     assert L.moe_combine_residual(fake, fake, fake, fake, 2, 2, 6, fake, None) == 4
     assert L.moe_combine_residual(fake, fake, fake, None, 2, 2, 8, fake, None) == 1
     assert L.moe_combine_residual(None, None, None, None, 0, 2, 8, None, None) == 0
+    # routing + gate_up in one launch: more than 32 tokens, more than 256 experts, K below
+    # six super-blocks or above 5120, K not a multiple of 256 (no fallback)
+    rg = L.moe_route_gate_up
+    assert rg(fake, 33, 128, 8, fake, fake, fake, fake, fake, fake, fake, 1536, 2048, fake, fake, None) == 4
+    assert rg(fake, 4, 512, 8, fake, fake, fake, fake, fake, fake, fake, 1536, 2048, fake, fake, None) == 4
+    assert rg(fake, 4, 128, 8, fake, fake, fake, fake, fake, fake, fake, 1536, 1280, fake, fake, None) == 4
+    assert rg(fake, 4, 128, 8, fake, fake, fake, fake, fake, fake, fake, 1536, 24 * 256, fake, fake, None) == 4
+    assert rg(fake, 4, 128, 8, fake, fake, fake, fake, fake, fake, fake, 1536, 2000, fake, fake, None) == 3
+    assert rg(fake, 4, 128, 8, fake, fake, None, fake, fake, fake, fake, 1536, 2048, fake, fake, None) == 1
     # empty problems are no-ops
     assert L.q4k_gemv(None, None, None, 0, 16, 256, None, 0, None) == 0
     assert L.moe_combine(None, None, None, 0, 2, 8, None, None) == 0

@@ -159,3 +159,45 @@ def test_grouped_decode_bad_offsets_latch(bad):
     y = host(q.moe_q4k_grouped(Wd, 3, 256, 2048, Ad, dev(offs), rows, 8, q.ACT_NONE, row_gather=gd))
     assert q.q4k_last_device_status() == 0
     _assert_tol(y, *O.grouped_ref(W, A, offs, row_gather=gather), "after the latch")
+
+
+# ------------------------------------------------ routing + gate_up, one launch --
+
+@pytest.mark.parametrize("case", ["M1", "M8", "M32", "E16_top3", "E256_top8"])
+def test_route_gate_up_equals_the_two_calls(case):
+    """moe_route_gate_up == moe_route_permute then moe_q4k_grouped (SwiGLU), bit for bit:
+    every routing output and the bf16 h."""
+    if case == "E16_top3":
+        M, topk, inp = 20, 3, synth.moe_layer(21, 20, E=16, H=1536, F=512)
+    elif case == "E256_top8":
+        M, topk, inp = 12, 8, synth.moe_layer(22, 12, E=256, H=1536, F=256)
+    else:
+        M, topk = int(case[1:]), 8
+        inp = synth.moe_decode(3, M)
+    E, H, F = inp["E"], inp["H"], inp["F"]
+    L, X, Wgu = dev(inp["logits"]), dev(inp["X"]), dev(inp["W_gate_up"])
+    r = q.moe_route_permute(L, topk)
+    h_ref = host(q.moe_q4k_grouped(Wgu, E, 2 * F, H, X, r["expert_offsets"], M * topk, M, q.ACT_SWIGLU,
+                                   row_gather=r["row_token"]))
+    for _ in range(2):
+        rr, h = q.moe_route_gate_up(L, topk, Wgu, 2 * F, H, X)
+        for k in ("topk_ids", "expert_offsets", "perm", "inv_perm", "row_token"):
+            assert np.array_equal(host(rr[k]), host(r[k])), k
+        assert np.array_equal(host(rr["topk_w"]).view(np.uint32), host(r["topk_w"]).view(np.uint32))
+        assert np.array_equal(host(h).view(np.uint16), h_ref.view(np.uint16))
+    assert q.q4k_last_device_status() == 0
+
+
+def test_route_gate_up_no_tokens():
+    """M == 0: only the expert offsets are cleared."""
+    E = 128
+    offs = torch.full((E + 1,), 7, dtype=torch.int32, device="cuda")
+    L = torch.empty(0, E, dtype=torch.float32, device="cuda")
+    W = torch.empty(16, dtype=torch.uint8, device="cuda")
+    X = torch.empty(0, 2048, dtype=torch.int16, device="cuda")
+    out = {k: torch.empty(16, dtype=torch.int32, device="cuda")
+           for k in ("topk_ids", "perm", "inv_perm", "row_token")}
+    out["topk_w"] = torch.empty(16, dtype=torch.float32, device="cuda")
+    out["expert_offsets"] = offs
+    q.moe_route_gate_up(L, 8, W, 1536, 2048, X, out=out, h=torch.empty(16, dtype=torch.bfloat16, device="cuda"))
+    assert int(torch.count_nonzero(offs)) == 0

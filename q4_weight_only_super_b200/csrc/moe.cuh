@@ -43,18 +43,28 @@ __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int
                                            int* sids, unsigned* tmask, int tile) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   static_assert(kRouteTokPerCta % NW == 0, "whole tokens per warp");
+  // the warp's next token's logits are loaded while it routes the current one
+  float nxt[PL];
+  auto load = [&](int tt) {
+    const int tok = tile * kRouteTokPerCta + tt * NW + warp;
+    const float* row = logits + (int64_t)tok * E;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+      const int e = i * 32 + lane;
+      nxt[i] = (tok < M && e < E) ? row[e] : 0.f;
+    }
+  };
+  load(0);
+#pragma unroll 1
   for (int tt = 0; tt < kRouteTokPerCta / NW; ++tt) {
     const int tl = tt * NW + warp;  // token within the tile
     const int tok = tile * kRouteTokPerCta + tl;
     if (tok >= M) break;  // uniform per warp
-    const float* row = logits + (int64_t)tok * E;
     float v[PL];
     uint32_t taken = 0;
 #pragma unroll
-    for (int i = 0; i < PL; ++i) {
-      const int e = i * 32 + lane;
-      v[i] = e < E ? row[e] : 0.f;
-    }
+    for (int i = 0; i < PL; ++i) v[i] = nxt[i];
+    if (tt + 1 < kRouteTokPerCta / NW) load(tt + 1);
     float sel_v[kMaxTopk];  // fully unrolled below, so these stay in registers
     int sel_i[kMaxTopk];
 #pragma unroll

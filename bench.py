@@ -401,39 +401,57 @@ def read_roof(torch, tm, W):
 
 
 def e2e_gemv(torch, q, W, steps, warmup):
-    """GEMV through the C ABI with host activations: H2D copy, kernel, D2H copy, all timed."""
+    """The step's ten decode GEMVs through the C ABI from host activations to host results,
+    as a serving loop issues them: one timed region per step holds every input's copy in
+    (pinned host -> device, on a copy stream, ahead of its GEMV), the GEMVs (each on rotating
+    weight copies, as the device-timed line, so none finds its weights in L2) and every
+    result's copy out (device -> pinned host, on the copy stream as soon as its GEMV ends,
+    overlapping the next GEMV); the step ends when the last result is on the host."""
     total_bytes, h2d, d2h = 0, 0, 0
     outs = {}
-    for M in (1, 4, 8, 16, 32):
-        for p in ("gate_up", "down"):
-            N, K = W["dec_shapes"][p]
-            outs[(p, M)] = (torch.empty(M, K, dtype=torch.int16, device="cuda"),
-                            torch.empty(M, N, dtype=torch.float32, device="cuda"),
-                            torch.empty(M, N, dtype=torch.float32).pin_memory())
+    order = [(M, p) for M in (1, 4, 8, 16, 32) for p in ("gate_up", "down")]
+    for M, p in order:
+        N, K = W["dec_shapes"][p]
+        outs[(p, M)] = (torch.empty(M, K, dtype=torch.int16, device="cuda"),
+                        torch.empty(M, N, dtype=torch.float32, device="cuda"),
+                        torch.empty(M, N, dtype=torch.float32).pin_memory())
+        total_bytes += N * (K // 256) * BLOCK
+        h2d += M * K * 2
+        d2h += M * N * 4
+    comp = torch.cuda.current_stream()
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     times = []
     for it in range(warmup + steps):
-        t_step = 0.0
-        for M in (1, 4, 8, 16, 32):
-            for p in ("gate_up", "down"):
-                N, K = W["dec_shapes"][p]
-                xd, yd, yh = outs[(p, M)]
-                xh = W["dec_host_X"][p][:M]
-                flush.fill_(1)
-                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                s.record()
-                xd.copy_(xh, non_blocking=True)
-                q.q4k_gemv(W["dec"][f"W_{p}"], xd, N, K, Y=yd, ws=W["ws"])
+        flush.fill_(1)  # nothing of the previous step left in L2
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(comp)
+        cin.wait_event(s)
+        cout.wait_event(s)
+        x_ready = {}
+        with torch.cuda.stream(cin):  # every input in, in the order the GEMVs need them
+            for M, p in order:
+                xd, _, _ = outs[(p, M)]
+                xd.copy_(W["dec_host_X"][p][:M], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(cin)
+                x_ready[(p, M)] = ev
+        for i, (M, p) in enumerate(order):
+            N, K = W["dec_shapes"][p]
+            xd, yd, yh = outs[(p, M)]
+            copies = W["dec_copies"][p]
+            comp.wait_event(x_ready[(p, M)])
+            q.q4k_gemv(copies[i % len(copies)], xd, N, K, Y=yd, ws=W["ws"])
+            done = torch.cuda.Event()
+            done.record(comp)
+            cout.wait_event(done)
+            with torch.cuda.stream(cout):
                 yh.copy_(yd, non_blocking=True)
-                e.record()
-                e.synchronize()
-                t_step += s.elapsed_time(e) * 1e-3
-                if it == 0:
-                    total_bytes += N * (K // 256) * BLOCK
-                    h2d += xh.numel() * 2
-                    d2h += yd.numel() * 4
+        comp.wait_stream(cout)
+        e.record(comp)
+        e.synchronize()
         if it >= warmup:
-            times.append(t_step)
+            times.append(s.elapsed_time(e) * 1e-3)
     return total_bytes, h2d, d2h, times
 
 

@@ -17,7 +17,7 @@
 //  * A warp owns a 16-row tile and a part of K; eight warps per CTA cover
 //    8/P tiles x P parts, and the CTA sums the parts in part order through shared
 //    memory (deterministic). P is the smallest power of two that gives at least
-//    2048 warps, so short matrices still fill the GPU.
+//    8192 warps, so many loads are in flight and short matrices still fill the GPU.
 //  * One mma.sync m16n8k16 per 16-weight sub-block (n, u, lh) and token group:
 //    thread t takes the sub-block's weights 16lh + 4t + {0,1,2,3}, which makes its
 //    four ql bytes, four qh bytes (and the activations) one word each. The six
@@ -167,11 +167,15 @@ __global__ void __launch_bounds__(32 * kQ6Warps) q6k_gemv_kernel(const Q6Params 
   }
 }
 
-// K parts per tile: the smallest power of two (at most 8) giving 2048 warps or more.
+// K parts per tile: the smallest power of two (at most 8) giving 8192 warps or more.
+// The warps' word loads are the bound (long-scoreboard stalls), so more of them in
+// flight is the lever: gate+up (2176 tiles) with four parts instead of one took
+// 89.4 -> 78.6 us at 1 token and 209 -> 175 us at 32 (eight parts: no better at 1
+// token, 205 us at 32).
 inline int q6_parts(int N, int nkb) {
   const int tiles = N / 16;
   int P = 1;
-  while (P < 8 && (int64_t)tiles * P < 2048 && P * 2 <= nkb) P *= 2;
+  while (P < 8 && (int64_t)tiles * P < 8192 && P * 2 <= nkb) P *= 2;
   return P;
 }
 

@@ -32,6 +32,12 @@ def _gpu(cuda_ok):
 
 
 def _run(op):
+    if op == "moe_route_gate_up":  # routing inside the grouped GEMV (MoE decode, one launch)
+        inp = synth.moe_layer(997, 4, E=16, H=1536, F=256)
+        E, H, F = inp["E"], inp["H"], inp["F"]
+        Lg, Xd, Wd = dev(inp["logits"]), dev(inp["X"]), dev(inp["W_gate_up"])
+        call = lambda: q.moe_route_gate_up(Lg, 2, Wd, 2 * F, H, Xd)[1]
+        return call, inp, None
     if op == "moe_dec":  # grouped stationary GEMV (MoE decode)
         rng = np.random.default_rng(996)
         E, N, K = 4, 256, 2048
@@ -51,7 +57,7 @@ def _run(op):
     return (lambda: q.q4k_gemm(dev(W), dev(X), N, K)), W, X
 
 
-@pytest.mark.parametrize("op", ["gemv_1tok", "gemv_17tok", "gemm", "moe_dec"])
+@pytest.mark.parametrize("op", ["gemv_1tok", "gemv_17tok", "gemm", "moe_dec", "moe_route_gate_up"])
 def test_bounded_wait_expires_and_recovers(op):
     call, W, X = _run(op)
     assert q.q4k_last_device_status() == 0
@@ -64,6 +70,13 @@ def test_bounded_wait_expires_and_recovers(op):
     assert q.q4k_last_device_status() == 0
     y = host(call())
     assert q.q4k_last_device_status() == 0
+    if op == "moe_route_gate_up":  # h after the timeout equals the two-call path's
+        inp = W
+        r = q.moe_route_permute(dev(inp["logits"]), 2)
+        h_ref = host(q.moe_q4k_grouped(dev(inp["W_gate_up"]), inp["E"], 2 * inp["F"], inp["H"], dev(inp["X"]),
+                                       r["expert_offsets"], 8, 4, q.ACT_SWIGLU, row_gather=r["row_token"]))
+        assert np.array_equal(y.view(np.uint16), h_ref.view(np.uint16))
+        return
     Y, S = O.grouped_ref(W[0], X, W[1]) if op == "moe_dec" else O.matmul_ref(W, X)
     ok, ratio = O.check_tolerance(y, Y, S)
     assert ok, f"{op} after a timeout: worst err/S = {ratio:.3e}"

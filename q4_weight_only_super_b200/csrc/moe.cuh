@@ -33,7 +33,8 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 // remaining (logit, id), the warp takes the largest logit (a reduce-max over
 // order keys) and, among lanes holding it, the smallest id (a reduce-min) --
 // the order "higher logit first, equal logits to the lower id". Softmax over
-// the selected logits in fp32. `hist` (shared, E entries, zeroed by the caller)
+// the selected logits in fp32 (lane k holds winner k: one exp per lane, the sum
+// over the lanes in a fixed butterfly order). `hist` (shared, E entries, zeroed by the caller)
 // receives the tile's expert histogram; `sids` (shared, or nullptr) a copy of
 // the tile's ids [token in tile][topk]; `tmask` (shared, or nullptr) bit t of
 // entry e set when token t of the tile selected expert e.
@@ -43,68 +44,142 @@ __device__ __forceinline__ void route_tile(const float* __restrict__ logits, int
                                            int* sids, unsigned* tmask, int tile) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   static_assert(kRouteTokPerCta % NW == 0, "whole tokens per warp");
-  // the warp's next token's logits are loaded while it routes the current one
-  float nxt[PL];
-  auto load = [&](int tt) {
-    const int tok = tile * kRouteTokPerCta + tt * NW + warp;
-    const float* row = logits + (int64_t)tok * E;
+  constexpr int TPW = kRouteTokPerCta / NW;  // tokens per warp
+  if constexpr (TPW == 1) {
+    // One token a warp (the one-CTA routing kernel): its logits loaded at once, the
+    // selection rounds unrolled where the registers allow. Winner k is kept by lane k.
+    float v[TPW][PL];
+    uint32_t taken[TPW];
+    float my_v[TPW];
+    int my_i[TPW];
 #pragma unroll
-    for (int i = 0; i < PL; ++i) {
-      const int e = i * 32 + lane;
-      nxt[i] = (tok < M && e < E) ? row[e] : 0.f;
-    }
-  };
-  load(0);
-#pragma unroll 1
-  for (int tt = 0; tt < kRouteTokPerCta / NW; ++tt) {
-    const int tl = tt * NW + warp;  // token within the tile
-    const int tok = tile * kRouteTokPerCta + tl;
-    if (tok >= M) break;  // uniform per warp
-    float v[PL];
-    uint32_t taken = 0;
-#pragma unroll
-    for (int i = 0; i < PL; ++i) v[i] = nxt[i];
-    if (tt + 1 < kRouteTokPerCta / NW) load(tt + 1);
-    float sel_v[kMaxTopk];  // fully unrolled below, so these stay in registers
-    int sel_i[kMaxTopk];
-#pragma unroll
-    for (int k = 0; k < kMaxTopk; ++k) {
-      sel_v[k] = 0.f;
-      sel_i[k] = 0;
-      if (k >= topk) continue;
-      float bv = -INFINITY;  // a lane with no candidate left never wins
-      int bi = 0x7fffffff;
+    for (int tt = 0; tt < TPW; ++tt) {
+      const int tok = tile * kRouteTokPerCta + tt * NW + warp;
+      const float* row = logits + (int64_t)tok * E;
 #pragma unroll
       for (int i = 0; i < PL; ++i) {
         const int e = i * 32 + lane;
-        if (e < E && !((taken >> i) & 1u) && ranks_before(v[i], e, bv, bi)) {
-          bv = v[i];
-          bi = e;
+        v[tt][i] = (tok < M && e < E) ? row[e] : 0.f;
+      }
+      taken[tt] = 0u;
+      my_v[tt] = 0.f;
+      my_i[tt] = 0;
+    }
+    // this warp's tokens in the tile (tokens past M take no rounds)
+    const int ntok = min(TPW, max(0, (M - tile * kRouteTokPerCta - warp + NW - 1) / NW));
+    auto round = [&](int k) {
+#pragma unroll
+      for (int tt = 0; tt < TPW; ++tt) {
+        if (tt >= ntok) break;  // uniform per warp
+        float bv = -INFINITY;  // a lane with no candidate left never wins
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+          const int e = i * 32 + lane;
+          if (e < E && !((taken[tt] >> i) & 1u) && ranks_before(v[tt][i], e, bv, bi)) {
+            bv = v[tt][i];
+            bi = e;
+          }
+        }
+        const uint32_t key = bi == 0x7fffffff ? 0u : order_key(bv);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const int wi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0x7fffffffu);
+        if ((wi & 31) == lane) taken[tt] |= 1u << (wi >> 5);
+        if (lane == k) {
+          my_v[tt] = key_value(kmax);
+          my_i[tt] = wi;
         }
       }
-      const uint32_t key = bi == 0x7fffffff ? 0u : order_key(bv);
-      const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
-      const int wi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0x7fffffffu);
-      if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
-      sel_v[k] = key_value(kmax);
-      sel_i[k] = wi;
+    };
+    if constexpr (PL <= 8) {  // the rounds unrolled (few logits a lane: registers to spare)
+#pragma unroll
+      for (int k = 0; k < kMaxTopk; ++k) {
+        if (k >= topk) break;
+        round(k);
+      }
+    } else {
+      for (int k = 0; k < topk; ++k) round(k);
     }
-    // softmax over the selected logits; sel_v[0] is the largest
-    float den = 0.f;
+    // softmax over each token's selected logits (lane 0 holds the largest): one exp
+    // per lane, the sum over the lanes in a fixed butterfly order
 #pragma unroll
-    for (int k = 0; k < kMaxTopk; ++k)
-      if (k < topk) den += expf(sel_v[k] - sel_v[0]);
-    if (lane < topk) {
-      float num = 0.f;
-      int id = 0;
+    for (int tt = 0; tt < TPW; ++tt) {
+      const int tl = tt * NW + warp;  // token within the tile
+      const int tok = tile * kRouteTokPerCta + tl;
+      if (tok >= M) break;  // uniform per warp
+      const float v0 = __shfl_sync(0xffffffffu, my_v[tt], 0);
+      const float ek = lane < topk ? expf(my_v[tt] - v0) : 0.f;
+      float den = ek;
 #pragma unroll
-      for (int k = 0; k < kMaxTopk; ++k)
-        if (k == lane) { num = expf(sel_v[k] - sel_v[0]); id = sel_i[k]; }
-      if (ids) ids[(int64_t)tok * topk + lane] = id;  // (null: not written)
-      if (wts) wts[(int64_t)tok * topk + lane] = num / den;
-      if (sids) sids[tl * topk + lane] = id;
-      if (tmask) atomicOr(&tmask[id], 1u << tl);
-      atomicAdd(&hist[id], 1);
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      if (lane < topk) {
+        const int id = my_i[tt];
+        if (ids) ids[(int64_t)tok * topk + lane] = id;  // (null: not written)
+        if (wts) wts[(int64_t)tok * topk + lane] = ek / den;
+        if (sids) sids[tl * topk + lane] = id;
+        if (tmask) atomicOr(&tmask[id], 1u << tl);
+        atomicAdd(&hist[id], 1);
+      }
+    }
+  } else {
+    // Several tokens a warp: one after another (the next token's logits load while the
+    // warp routes the current one; one copy of the rounds, so the code stays small).
+    float nxt[PL];
+    auto load = [&](int tt) {
+      const int tok = tile * kRouteTokPerCta + tt * NW + warp;
+      const float* row = logits + (int64_t)tok * E;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) {
+        const int e = i * 32 + lane;
+        nxt[i] = (tok < M && e < E) ? row[e] : 0.f;
+      }
+    };
+    load(0);
+#pragma unroll 1
+    for (int tt = 0; tt < TPW; ++tt) {
+      const int tl = tt * NW + warp;  // token within the tile
+      const int tok = tile * kRouteTokPerCta + tl;
+      if (tok >= M) break;  // uniform per warp
+      float v[PL];
+      uint32_t taken = 0;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) v[i] = nxt[i];
+      if (tt + 1 < TPW) load(tt + 1);
+      float my_v = 0.f;
+      int my_i = 0;
+      for (int k = 0; k < topk; ++k) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+          const int e = i * 32 + lane;
+          if (e < E && !((taken >> i) & 1u) && ranks_before(v[i], e, bv, bi)) {
+            bv = v[i];
+            bi = e;
+          }
+        }
+        const uint32_t key = bi == 0x7fffffff ? 0u : order_key(bv);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const int wi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0x7fffffffu);
+        if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
+        if (lane == k) {
+          my_v = key_value(kmax);
+          my_i = wi;
+        }
+      }
+      const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
+      const float ek = lane < topk ? expf(my_v - v0) : 0.f;
+      float den = ek;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      if (lane < topk) {
+        const int id = my_i;
+        if (ids) ids[(int64_t)tok * topk + lane] = id;
+        if (wts) wts[(int64_t)tok * topk + lane] = ek / den;
+        if (sids) sids[tl * topk + lane] = id;
+        if (tmask) atomicOr(&tmask[id], 1u << tl);
+        atomicAdd(&hist[id], 1);
+      }
     }
   }
 }

@@ -13,6 +13,7 @@
 #include "gemv.cuh"
 #include "gemv_q6.cuh"
 #include "gemv_sk.cuh"
+#include "gemv_sk6.cuh"
 #include "gemv_skg.cuh"
 #include "moe.cuh"
 
@@ -217,17 +218,18 @@ q4k_status launch_gemv(const GemvCfg& c, GemvParams p, const uint16_t* X, const 
 
 // sk_fit[d][kpw-1][P]: clusters of P stationary-GEMV CTAs (one per SM) resident at
 // once on device d.
-std::atomic<int> g_sk_fit[kMaxDevices][2][9];
-std::atomic<size_t> g_sk_smem_set[2][kMaxDevices];
+// Q6: the Q6_K form of the kernel (gemv_sk6_kernel), with its own tables.
+std::atomic<int> g_sk_fit[2][kMaxDevices][2][9];
+std::atomic<size_t> g_sk_smem_set[2][2][kMaxDevices];
 
-template <int KPW>
+template <int KPW, bool Q6 = false>
 q4k_status sk_cluster_fit_t(int P, int* fit) {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices || P < 1 || P > 8) return Q4K_ERR_CUDA;
-  int v = g_sk_fit[dev][KPW - 1][P].load();
+  int v = g_sk_fit[Q6][dev][KPW - 1][P].load();
   if (v <= 0) {
-    auto* k = gemv_sk_kernel<KPW>;
-    if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[KPW - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
+    auto* k = Q6 ? gemv_sk6_kernel<KPW> : gemv_sk_kernel<KPW>;
+    if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[Q6][KPW - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(P * 64), 1, 1);
     cfg.blockDim = dim3(SkMax<KPW>::threads, 1, 1);
@@ -243,29 +245,30 @@ q4k_status sk_cluster_fit_t(int P, int* fit) {
       cudaGetLastError();
       return Q4K_ERR_CUDA;
     }
-    g_sk_fit[dev][KPW - 1][P].store(v);
+    g_sk_fit[Q6][dev][KPW - 1][P].store(v);
   }
   *fit = v;
   return Q4K_OK;
 }
 
 // The stationary GEMV's launch shape for an N x K matrix; *ok = false when the shape
-// is outside what it covers (more than 8 K parts).
-q4k_status pick_sk(int N, int nkb, SkCfg* c, bool* ok) {
+// is outside what it covers (more than 8 K parts). q6: the Q6_K form.
+q4k_status pick_sk(int N, int nkb, SkCfg* c, bool* ok, bool q6 = false) {
   *ok = false;
-  if (!sk_shape(N, nkb, c)) return Q4K_OK;
+  if (!(q6 ? sk6_shape(N, nkb, c) : sk_shape(N, nkb, c))) return Q4K_OK;
   int fit = 0;
-  const q4k_status st = c->kpw == 2 ? sk_cluster_fit_t<2>(c->P, &fit) : sk_cluster_fit_t<1>(c->P, &fit);
+  const q4k_status st = q6 ? (c->kpw == 2 ? sk_cluster_fit_t<2, true>(c->P, &fit) : sk_cluster_fit_t<1, true>(c->P, &fit))
+                           : (c->kpw == 2 ? sk_cluster_fit_t<2>(c->P, &fit) : sk_cluster_fit_t<1>(c->P, &fit));
   if (st != Q4K_OK) return Q4K_OK;  // not resident on this device: the ring kernel takes the shape
   *ok = sk_finish(fit, c);
   return Q4K_OK;
 }
 
-template <int KPW>
+template <int KPW, bool Q6 = false>
 q4k_status launch_sk_t(const SkCfg& c, const void* W, const uint16_t* X, float* Y, int M, int N, int K,
                        cudaStream_t s) {
-  auto* k = gemv_sk_kernel<KPW>;
-  if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[KPW - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
+  auto* k = Q6 ? gemv_sk6_kernel<KPW> : gemv_sk_kernel<KPW>;
+  if (ensure_smem(k, kSkSmemBudget, g_sk_smem_set[Q6][KPW - 1]) != cudaSuccess) return Q4K_ERR_LAUNCH;
   SkParams p = {};
   p.W = static_cast<const uint8_t*>(W);
   p.X = X;
@@ -299,7 +302,9 @@ q4k_status launch_sk_t(const SkCfg& c, const void* W, const uint16_t* X, float* 
 }
 
 q4k_status launch_sk(const SkCfg& c, const void* W, const uint16_t* X, float* Y, int M, int N, int K,
-                     cudaStream_t s) {
+                     cudaStream_t s, bool q6 = false) {
+  if (q6)
+    return c.kpw == 2 ? launch_sk_t<2, true>(c, W, X, Y, M, N, K, s) : launch_sk_t<1, true>(c, W, X, Y, M, N, K, s);
   return c.kpw == 2 ? launch_sk_t<2>(c, W, X, Y, M, N, K, s) : launch_sk_t<1>(c, W, X, Y, M, N, K, s);
 }
 
@@ -558,6 +563,13 @@ q4k_status q6k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
   if (ws_bytes < gemv_ws_bytes(M, K)) return Q4K_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int nkb = K / QK;
+  if (M <= 8) {  // 1..8 tokens: the stationary form, one launch, no pre-pass
+    SkCfg sc;
+    bool ok = false;
+    const q4k_status st = pick_sk(N, nkb, &sc, &ok, true);
+    if (st != Q4K_OK) return st;
+    if (ok) return launch_sk(sc, W, X, Y, M, N, K, s, true);
+  }
   Q6Params p = {};
   p.W = static_cast<const uint8_t*>(W);
   p.xprep = static_cast<const uint8_t*>(ws);

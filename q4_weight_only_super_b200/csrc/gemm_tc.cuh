@@ -63,8 +63,6 @@ constexpr uint32_t kSmemB = kSmemA + kStagesAW * kATileBytes;
 static_assert(kDqWarps * 32 * kEpiPitch * 4 <= kStagesAW * kATileBytes, "epilogue staging fits the A stages");
 constexpr uint32_t kSmemW = kSmemB + kStagesB * kBTileBytes;
 constexpr uint32_t kSmemBar = kSmemW + kStagesAW * kWRawBytes;
-constexpr uint32_t kSmemTotal = kSmemBar + 256;
-constexpr size_t kGemmSmemLaunch = kSmemTotal + 1024;  // + alignment slack
 
 // Shared-memory layout of one CTA. PAIR: a CTA pair (a cluster of two) computes a
 // 512-token x 256-weight-row tile with tcgen05.mma.cta_group::2 (M = 256, N = 256):
@@ -307,12 +305,6 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, uint32_t rank) 
       " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}" ::"r"(bar),
       "r"(rank)
       : "memory");
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
 }
 
 // All threads of both CTAs of the cluster (release / acquire).

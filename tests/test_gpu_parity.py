@@ -203,10 +203,11 @@ def test_q6k_gemv_odd_block_count_rows():
     _assert_tol(y, Y, S, "Q6_K odd block count")
 
 
-def test_q6k_gemv_edge_blocks():
+@pytest.mark.parametrize("M", [3, 9])  # the stationary form (1..8 tokens) and the 9..16 class
+def test_q6k_gemv_edge_blocks(M):
     """Extreme Q6_K blocks: d = +-65504, subnormal d, zero; scales -128, 127, 0; q = -32, 31, 0."""
     rng = np.random.default_rng(830)
-    N, K, M = 272, 256 * 5, 9
+    N, K = 272, 256 * 5
     pool = np.stack([O.make_block_q6(d, sc, qv) for d in (65504.0, -65504.0, 6e-8, 0.0, -1.5)
                      for sc in ([-128] * 16, [127] * 16, [0] * 16, list(range(-8, 8)))
                      for qv in ([-32] * 256, [31] * 256, [0] * 256, list(rng.integers(-32, 32, 256)))])

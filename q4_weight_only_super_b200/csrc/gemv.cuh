@@ -273,9 +273,18 @@ constexpr int kQ5QsOff = 48;   // the 128 nibble bytes, ordered as in Q4_K
 // GEMV reads them eight at a time (one 256-wide column of the matrix, 272 bytes
 // per row), and block j of a group plays the part of Q4_K's sub-block j
 constexpr int kQ80GroupBytes = 272;
+// Q6_K: 210-byte super-blocks (ql[128], qh[64], sixteen signed byte scales at 192, fp16
+// d at 208). Rows are then only 2-byte aligned, out of reach of a TMA box, so each row's
+// block of a stage is one 224-byte bulk copy of its 16-byte-aligned superset (the block
+// starts 0..14 bytes in; 224 = 14 * 16 also ends each copy at or before the next block's
+// end, and the last copy of the matrix exactly at its end, the matrix being a multiple of
+// 16 bytes long)
+constexpr int kQ6BB = 210;
+constexpr int kQ6Copy = 224;
 // weight formats of the GEMV kernel
 constexpr int kQtQ4K = 0, kQtQ5K = 1, kQtQ80 = 2;
 constexpr int kQtQ4KxQ8 = 3;  // Q4_K weights, int8 activations (the Q8 lane)
+constexpr int kQtQ6K = 4;
 
 // Shared memory layout (dynamic):
 //   wring [wstages][WARPS][16*TILES rows][160 B]   weight tiles (TMA destination)
@@ -291,7 +300,9 @@ template <int MT, int WARPS, int TILES, bool REPACK = false, int QT = kQtQ4K>
 struct GemvSmem {
   static constexpr int TOK = 8 * MT;
   static constexpr int pitch =
-      QT == kQtQ80 ? kQ80GroupBytes : (QT == kQtQ5K ? kQ5BlockBytes : (REPACK ? BLOCK_BYTES : kGemvPitch));
+      QT == kQtQ6K ? kQ6Copy
+                   : (QT == kQtQ80 ? kQ80GroupBytes
+                                   : (QT == kQtQ5K ? kQ5BlockBytes : (REPACK ? BLOCK_BYTES : kGemvPitch)));
   // Q8_0 (272-byte rows): the reduction buffer lies in the weight ring, which is
   // free once every stage has been consumed, so 32 tokens still fit two CTAs per SM
   static constexpr bool red_in_ring = QT == kQtQ80;
@@ -326,6 +337,111 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
       : "memory");
 }
 
+// The 4 bytes at a 2-byte-aligned shared-memory address (its row has slack after it).
+__device__ __forceinline__ uint32_t lds_word_a2(const uint8_t* p) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  const uint32_t* q = reinterpret_cast<const uint32_t*>(a & ~static_cast<uintptr_t>(3));
+  return __funnelshift_r(q[0], q[1], (uint32_t)(a & 3) * 8u);
+}
+
+// Signed scale byte j (0..3) of a word, as an exact fp32: (2^23 + 128 + s) - (2^23 + 128).
+__device__ __forceinline__ float s8_to_f32(uint32_t w, int j) {
+  return __uint_as_float(__byte_perm(w ^ 0x80808080u, 0x4B000000u, 0x7650u | (uint32_t)j)) - 8388736.f;
+}
+
+// One Q6_K stage of a consumer warp: its rows g + 8r (r < 2*TILES) of the warp tile wt,
+// row r's block starting off[r] bytes into its copy, times the stage's activation
+// records xb for MT token groups; acc += d * 2^-k * sum_i scale_i * (q . x)_i.
+// One mma.sync m16n8k16 per 16-weight sub-block (n, u, lh), tile and token group: thread
+// t takes weights 16lh + 4t + {0..3}, so its ql and qh data are one word each per row;
+// the six bits go into the low byte of 0x6400 = 1024 + (q + 32) and one fp16 add of
+// -1056 leaves q itself, exact. The signed scale multiplies the fp32 MMA result. The
+// record holds the matching activations in the 8-byte half t%2 of chunk
+// 4(4n + u) + 2lh + t/2 (the order the pre-pass gives every 32-wide column).
+template <int MT, int TILES>
+__device__ __forceinline__ void q6_stage(float (&acc)[TILES][MT][4], const uint8_t* wt, const int (&off)[2 * TILES],
+                                         const uint8_t* xb, int g, int t) {
+  constexpr int R = 2 * TILES;
+  const uint8_t* rb[R];
+  uint32_t sc[R][4];
+  float d[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    rb[r] = wt + (g + 8 * r) * kQ6Copy + off[r];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[r][i] = lds_word_a2(rb[r] + 192 + 4 * i);
+    d[r] = __half2float(*reinterpret_cast<const __half*>(rb[r] + 208));
+  }
+  const __half2 m1056 = __float2half2_rn(-1056.f);
+  float C[TILES][MT][4];
+#pragma unroll
+  for (int n = 0; n < 2; ++n) {
+#pragma unroll
+    for (int lh = 0; lh < 2; ++lh) {
+      const int o = 64 * n + 16 * lh + 4 * t;
+      uint32_t la[R], lb[R], hq[R];  // ql words for u = 0, 2 and u = 1, 3; qh for all four
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        la[r] = lds_word_a2(rb[r] + o);
+        lb[r] = lds_word_a2(rb[r] + o + 32);
+        hq[r] = lds_word_a2(rb[r] + 128 + 32 * n + 16 * lh + 4 * t);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int si = 8 * n + 2 * u + lh;  // scale index (weight / 16)
+        uint32_t lo[R], hi[R];
+        float s[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          // six-bit values q + 32 of the four weights, one per byte
+          const uint32_t v = ((((u & 1) ? lb[r] : la[r]) >> (4 * (u >> 1))) & 0x0F0F0F0Fu) |
+                             (((hq[r] >> (2 * u)) & 0x03030303u) << 4);
+          lo[r] = h2_bits(__hadd2(bits_h2(__byte_perm(v, 0x64646464u, 0x4240u)), m1056));  // weights 4t, 4t+2
+          hi[r] = h2_bits(__hadd2(bits_h2(__byte_perm(v, 0x64646464u, 0x4341u)), m1056));  // 4t+1, 4t+3
+          s[r] = s8_to_f32(sc[r][si >> 2], si & 3);
+        }
+        const int boff = (4 * (4 * n + u) + 2 * lh + (t >> 1)) * 16 + 8 * (t & 1);
+#pragma unroll
+        for (int f = 0; f < MT; ++f) {
+          const uint2 bx = *reinterpret_cast<const uint2*>(xb + (8 * f + g) * kXRec + boff);
+#pragma unroll
+          for (int tt = 0; tt < TILES; ++tt) {
+            // A: rows g (regs 0, 2) and g+8 (regs 1, 3) of tile tt
+            float Cj[4];
+            mma_f16_16816(Cj, lo[2 * tt], lo[2 * tt + 1], hi[2 * tt], hi[2 * tt + 1], bx.x, bx.y, true);
+            const float sa = s[2 * tt], sb = s[2 * tt + 1];
+            if (si == 0) {
+              C[tt][f][0] = sa * Cj[0];
+              C[tt][f][1] = sa * Cj[1];
+              C[tt][f][2] = sb * Cj[2];
+              C[tt][f][3] = sb * Cj[3];
+            } else {
+              C[tt][f][0] = fmaf(sa, Cj[0], C[tt][f][0]);
+              C[tt][f][1] = fmaf(sa, Cj[1], C[tt][f][1]);
+              C[tt][f][2] = fmaf(sb, Cj[2], C[tt][f][2]);
+              C[tt][f][3] = fmaf(sb, Cj[3], C[tt][f][3]);
+            }
+          }
+        }
+      }
+    }
+  }
+  // y += d * 2^-k * C (2^-k of tokens 2t and 2t+1 of each group, from the records)
+#pragma unroll
+  for (int f = 0; f < MT; ++f) {
+    const float k0 = *reinterpret_cast<const float*>(xb + (8 * f + 2 * t) * kXRec + 544);
+    const float k1 = *reinterpret_cast<const float*>(xb + (8 * f + 2 * t + 1) * kXRec + 544);
+#pragma unroll
+    for (int tt = 0; tt < TILES; ++tt) {
+      const float da = d[2 * tt], db = d[2 * tt + 1];
+      acc[tt][f][0] = fmaf(da * k0, C[tt][f][0], acc[tt][f][0]);
+      acc[tt][f][1] = fmaf(da * k1, C[tt][f][1], acc[tt][f][1]);
+      acc[tt][f][2] = fmaf(db * k0, C[tt][f][2], acc[tt][f][2]);
+      acc[tt][f][3] = fmaf(db * k1, C[tt][f][3], acc[tt][f][3]);
+    }
+  }
+}
+
 // Roles: warps 0..WARPS-1 consume (16*TILES weight rows each); warp WARPS issues
 // the weight TMA; warp WARPS+1 copies the activation records.
 // GROUPED: blockIdx.y enumerates non-empty experts (the y-th expert with a
@@ -339,13 +455,18 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
 //    of the subnormal form at every token count, with A = the signed q itself as
 //    an fp16 integer (-128..127, exact) and the block's d as the sub-block scale;
 //    no min term.
+//  * Q6_K (210-byte super-blocks): the weight producer warp issues one 224-byte
+//    bulk copy per row (the block's 16-byte-aligned superset) instead of a TMA
+//    box, and the consumers run q6_stage on each row from its own offset; no min
+//    term.
 template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK = false, int QT = kQtQ4K>
 __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                                    GemvParams p) {
   using L = GemvSmem<MT, WARPS, TILES, REPACK, QT>;
   static_assert(!REPACK || (!GROUPED && 16 * TILES * WARPS == kRepackRows), "repacked: dense, 128-row tiles");
-  static_assert(QT == kQtQ4K || (!GROUPED && !REPACK), "Q5_K, Q8_0: dense raw layout");
-  constexpr bool Q5 = QT == kQtQ5K, Q80 = QT == kQtQ80, Q8X = QT == kQtQ4KxQ8;
+  static_assert(QT == kQtQ4K || (!GROUPED && !REPACK), "Q5_K, Q8_0, Q6_K: dense raw layout");
+  static_assert(QT != kQtQ6K || !SWIGLU, "Q6_K: plain output");
+  constexpr bool Q5 = QT == kQtQ5K, Q80 = QT == kQtQ80, Q8X = QT == kQtQ4KxQ8, Q6 = QT == kQtQ6K;
   constexpr int BB = Q80 ? kQ80GroupBytes : (Q5 ? kQ5BlockBytes : BLOCK_BYTES);  // bytes per 256-wide column
   constexpr int QO = Q5 ? kQ5QsOff : 16;                                         // offset of the nibble bytes
   constexpr int TOK = 8 * MT;
@@ -359,7 +480,7 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int SW = p.wstages, SX = p.xstages;
-  if (!REPACK && threadIdx.x == 32 * WARPS)  // the weight-TMA thread: fetch the descriptor while the rest sets up
+  if (!REPACK && !Q6 && threadIdx.x == 32 * WARPS)  // the weight-TMA thread: fetch the descriptor meanwhile
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
 
   const int rank = (int)(blockIdx.x % (unsigned)p.ksplit);
@@ -432,8 +553,51 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
   __syncthreads();
 
   if (warp == WARPS) {
-    // ---------------- weight producer: TMA ----------------
-    if (lane == 0) {
+    if (Q6) {
+      // ---------------- weight producer, Q6_K: one 224-byte bulk copy per row ----------------
+      // lane l copies row l of every warp tile; rows past N are not copied (no MMA tile
+      // mixes them with real rows, and their results are never written)
+      static_assert(!Q6 || 16 * TILES == 32, "Q6_K: one row per lane and warp tile");
+      const int drop = g_test_drop_stage;  // test hook; -1 in normal use
+      const int64_t row_bytes = (int64_t)p.nkb * kQ6BB;
+      const int rbase = tile * ROWS + lane;
+      uint32_t nrows = 0;
+#pragma unroll
+      for (int w = 0; w < WARPS; ++w) nrows += rbase + WROWS * w < p.N ? 1u : 0u;
+      const uint32_t tx = __reduce_add_sync(0xffffffffu, nrows) * (uint32_t)kQ6Copy;
+      int issued = 0, s = 0;
+      uint32_t ph = 0;
+      for (int ks = 0; ks < nk; ++ks) {
+        int ok = 1;
+        if (lane == 0) {
+          if (ks >= SW) mbar_wait(wempty(s), ph ^ 1u, abort_flag);
+          ok = !*abort_flag;
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if (ks != drop) {
+          if (lane == 0) mbar_arrive_expect_tx(wfull(s), tx);
+          __syncwarp();
+          const int64_t kofs = (int64_t)(kb0 + ks) * kQ6BB;
+          const uint32_t dst = smem_u32(smem) + (uint32_t)(s * L::wstage) + (uint32_t)(lane * kQ6Copy);
+#pragma unroll
+          for (int w = 0; w < WARPS; ++w) {
+            const int r = rbase + WROWS * w;
+            if (r < p.N)
+              bulk_copy_g2s(dst + (uint32_t)(w * L::warp_tile), p.W + (((int64_t)r * row_bytes + kofs) & ~(int64_t)15),
+                            (uint32_t)kQ6Copy, wfull(s));
+          }
+        }
+        ++issued;
+        if (++s == SW) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (lane == 0)
+        for (int ks = (issued > SW ? issued - SW : 0); ks < issued; ++ks)
+          if (ks != drop) mbar_wait_drain(wfull(ks % SW), (ks / SW) & 1);
+    } else if (lane == 0) {
+      // ---------------- weight producer: TMA ----------------
       const int lim = SWIGLU ? p.N / 2 : p.N;
       const int drop = g_test_drop_stage;  // test hook; -1 in normal use
       int issued = 0;
@@ -514,12 +678,42 @@ __global__ void __launch_bounds__(32 * (WARPS + 2), 2) gemv_kernel(const __grid_
     const __half2 sixteenth = __float2half2_rn(0.0625f);
     const __half2 neg64 = __float2half2_rn(-64.f);
 
+    // Q6_K: row g + 8r of this warp starts (its offset + 210 kb) mod 16 bytes into its copy
+    int q6off[Q6 ? 2 * TILES : 1];
+#pragma unroll
+    for (int r = 0; r < (Q6 ? 2 * TILES : 0); ++r)
+      q6off[r] = (int)(((int64_t)(r0 + g + 8 * r) * ((int64_t)p.nkb * kQ6BB)) & 15);
     int sw = 0, sx = 0;
     uint32_t pw = 0, px = 0;  // ring stage indices and phase parities (no divisions)
     for (int ks = 0; ks < nk; ++ks) {
       mbar_wait(wfull(sw), pw, abort_flag);
       const int sw_cur = sw;
       const uint8_t* wt = smem + sw * L::wstage + warp * L::warp_tile;
+      if (Q6) {
+        // the stage's weights are read from shared memory until the end: both rings are
+        // released together
+        mbar_wait(xfull(sx), px, abort_flag);
+        if (valid) {
+          int off[2 * TILES];
+#pragma unroll
+          for (int r = 0; r < 2 * TILES; ++r) off[r] = (q6off[r] + (kb0 + ks) * kQ6BB) & 15;
+          q6_stage<MT, TILES>(acc, wt, off, xring + (size_t)sx * L::xstage, g, t);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(wempty(sw));
+          mbar_arrive(xempty(sx));
+        }
+        if (++sw == SW) {
+          sw = 0;
+          pw ^= 1u;
+        }
+        if (++sx == SX) {
+          sx = 0;
+          px ^= 1u;
+        }
+        continue;
+      }
       // rows g, g+8 (tile 0), g+16, g+24 (tile 1), ... of this warp's rows
       constexpr int R = 2 * TILES;
       uint32_t hdx[R];

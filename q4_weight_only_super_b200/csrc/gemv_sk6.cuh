@@ -27,8 +27,6 @@
 
 namespace q4k {
 
-constexpr int kQ6BB = 210;  // bytes per Q6_K super-block
-
 // Row pitch in shared memory for runs of KU super-blocks: the aligned superset (up to
 // 30 bytes more), padded to 32 or 96 modulo 128 (rows g = 0..7 in distinct banks) with
 // 8 bytes of slack for the second load of the last word.
@@ -76,18 +74,6 @@ __device__ __forceinline__ void sk6_load_act(Sk6Act& a, const uint16_t* xc, bool
   }
   a.s0 = __shfl_sync(0xffffffffu, kinv, 8 * t);
   a.s1 = __shfl_sync(0xffffffffu, kinv, 8 * t + 4);
-}
-
-// The 4 bytes at a 2-byte-aligned shared-memory address (its row has slack after it).
-__device__ __forceinline__ uint32_t lds_word_a2(const uint8_t* p) {
-  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
-  const uint32_t* q = reinterpret_cast<const uint32_t*>(a & ~static_cast<uintptr_t>(3));
-  return __funnelshift_r(q[0], q[1], (uint32_t)(a & 3) * 8u);
-}
-
-// Signed scale byte j (0..3) of a word, as an exact fp32: (2^23 + 128 + s) - (2^23 + 128).
-__device__ __forceinline__ float s8_to_f32(uint32_t w, int j) {
-  return __uint_as_float(__byte_perm(w ^ 0x80808080u, 0x4B000000u, 0x7650u | (uint32_t)j)) - 8388736.f;
 }
 
 // One 16 x 256 Q6_K block (rows g, g+8 start at b0, b1 in shared memory, 2-byte aligned)

@@ -11,7 +11,6 @@
 #include "dequant.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
-#include "gemv_q6.cuh"
 #include "gemv_sk.cuh"
 #include "gemv_sk6.cuh"
 #include "gemv_skg.cuh"
@@ -97,6 +96,11 @@ static_assert(GemvSmem<2, 4, 2, false, kQtQ80>::total(kGemvStagesQ80[1][0], kGem
 static_assert(GemvSmem<4, 4, 2, false, kQtQ80>::total(kGemvStagesQ80[2][0], kGemvStagesQ80[2][1]) <= kGemvTwoPerSm, "q8 mt 4");
 static_assert(GemvSmem<4, 4, 2, false, kQtQ80>::red_bytes <= 2 * GemvSmem<4, 4, 2, false, kQtQ80>::wstage,
               "q8: reduction buffer inside the weight ring");
+// Q6_K: 224-byte row copies, two or three weight stages
+constexpr int kGemvStagesQ6[3][2] = {{3, 5}, {3, 2}, {2, 2}};
+static_assert(GemvSmem<1, 4, 2, false, kQtQ6K>::total(kGemvStagesQ6[0][0], kGemvStagesQ6[0][1]) <= kGemvTwoPerSm, "q6 mt 1");
+static_assert(GemvSmem<2, 4, 2, false, kQtQ6K>::total(kGemvStagesQ6[1][0], kGemvStagesQ6[1][1]) <= kGemvTwoPerSm, "q6 mt 2");
+static_assert(GemvSmem<4, 4, 2, false, kQtQ6K>::total(kGemvStagesQ6[2][0], kGemvStagesQ6[2][1]) <= kGemvTwoPerSm, "q6 mt 4");
 
 // fit[d][ks]: clusters of ks GEMV CTAs that can be resident at once on device d
 // (a cluster must sit inside one GPC, so this is below 2 * SMs / ks).
@@ -166,10 +170,10 @@ template <int MT, int WARPS, int TILES, bool GROUPED, bool SWIGLU, bool REPACK =
 q4k_status launch_gemv_t(const GemvParams& p, int rows_total, int tiles, int groups, cudaStream_t s) {
   auto* k = gemv_kernel<MT, WARPS, TILES, GROUPED, SWIGLU, REPACK, QT>;
   static std::atomic<size_t> smem_set[kMaxDevices];  // one per instantiation
-  CUtensorMap tmap = {};  // repacked weights stream by plain bulk copies: no tensor map
+  CUtensorMap tmap = {};  // repacked and Q6_K weights stream by plain bulk copies: no tensor map
   using LS = GemvSmem<MT, WARPS, TILES, REPACK, QT>;
   const int bb = QT == kQtQ80 ? kQ80GroupBytes : (QT == kQtQ5K ? kQ5BlockBytes : BLOCK_BYTES);
-  if (!REPACK && !make_tmap_w_rowgroup(&tmap, p.W, rows_total, (int64_t)p.nkb * bb, 16 * TILES, LS::pitch,
+  if (!REPACK && QT != kQtQ6K && !make_tmap_w_rowgroup(&tmap, p.W, rows_total, (int64_t)p.nkb * bb, 16 * TILES, LS::pitch,
                                        QT == kQtQ80 ? 2 : 1))
     return Q4K_ERR_CUDA;
   const size_t smem = GemvSmem<MT, WARPS, TILES, REPACK, QT>::total(p.wstages, p.xstages);
@@ -570,24 +574,21 @@ q4k_status q6k_gemv(const void* W, const uint16_t* X, float* Y, int M, int N, in
     if (st != Q4K_OK) return st;
     if (ok) return launch_sk(sc, W, X, Y, M, N, K, s, true);
   }
-  Q6Params p = {};
+  // 9..32 tokens (and shapes the stationary form does not cover): the ring GEMV, the
+  // weights streamed by per-row bulk copies
+  GemvParams p = {};
   p.W = static_cast<const uint8_t*>(W);
-  p.xprep = static_cast<const uint8_t*>(ws);
-  p.Y = Y;
+  p.out = Y;
   p.M = M;
   p.N = N;
   p.nkb = nkb;
-  p.rows_pad = M + kXPadRows;
-  p.P = q6_parts(N, nkb);
-  const int64_t recs = (int64_t)p.rows_pad * nkb;
-  q4k_status st = launch_pdl(gemv_prep_kernel, dim3((unsigned)((recs + 7) / 8)), dim3(256), s, X,
-                             static_cast<const int32_t*>(nullptr), M, p.rows_pad, K, nkb, static_cast<uint8_t*>(ws));
+  GemvCfg c;
+  const q4k_status st = pick_gemv(M, N, nkb, 1, &c);  // the Q4_K K split: same cluster fit
   if (st != Q4K_OK) return st;
-  const int T = kQ6Warps / p.P;
-  const dim3 grid((unsigned)((N / 16 + T - 1) / T));
-  if (M <= 8) return launch_pdl(q6k_gemv_kernel<1>, grid, dim3(32 * kQ6Warps), s, p);
-  if (M <= 16) return launch_pdl(q6k_gemv_kernel<2>, grid, dim3(32 * kQ6Warps), s, p);
-  return launch_pdl(q6k_gemv_kernel<4>, grid, dim3(32 * kQ6Warps), s, p);
+  const int cls = c.mt == 1 ? 0 : (c.mt == 2 ? 1 : 2);
+  c.wstages = kGemvStagesQ6[cls][0];
+  c.xstages = kGemvStagesQ6[cls][1];
+  return launch_gemv<false, false, false, kQtQ6K>(c, p, X, nullptr, M, K, ws, N, 1, s);
 }
 
 q4k_status q4k_repack(const void* W, int N, int K, void* Wr, void* stream) {
